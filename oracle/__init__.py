@@ -1,0 +1,135 @@
+"""Double-precision CPU oracle of causal multi-head attention (fwd + bwd).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline leg may import this package.  The product path (the CUDA
+library and its Python binding) never imports it and shares no code with it.
+
+The arithmetic lives in ``attn_oracle.c`` (plain loops in double, OpenMP over
+heads); this module compiles it with gcc on first use and marshals numpy
+float64 arrays through ctypes.  Every function takes [B, H, T, D] arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libattn_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library (gcc -O2 -fopenmp, IEEE math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class OracleLib:
+    """ctypes view of one compiled oracle library (the default one, or a
+    variant a test builds from edited source to check that the pins bite)."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        i = ctypes.c_int
+        lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double]
+        lib.oracle_attn_fwd.restype = None
+        lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, ctypes.c_double]
+        lib.oracle_attn_probs.restype = None
+        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double]
+        lib.oracle_attn_bwd.restype = None
+        lib.oracle_threads.argtypes = []
+        lib.oracle_threads.restype = i
+        self.lib = lib
+
+    def attn_fwd(self, q, k, v, scale=None):
+        """Returns (O [B,H,T,D], lse [B,H,T]) in float64."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, T, D = _shape(q)
+        scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+        o = np.empty_like(q)
+        lse = np.empty((B, H, T), dtype=np.float64)
+        self.lib.oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D, scale)
+        return o, lse
+
+    def attn_probs(self, q, k, scale=None):
+        """The causal softmax matrices P [B,H,T,T] (zero above the diagonal)."""
+        q, k = _f64(q), _f64(k)
+        B, H, T, D = _shape(q)
+        scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+        p = np.empty((B, H, T, T), dtype=np.float64)
+        self.lib.oracle_attn_probs(_ptr(q), _ptr(k), _ptr(p), B, H, T, D, scale)
+        return p
+
+    def attn_bwd(self, q, k, v, do, scale=None):
+        """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
+        q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+        B, H, T, D = _shape(q)
+        scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        self.lib.oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                                 B, H, T, D, scale)
+        return dq, dk, dv
+
+    def threads_used(self) -> int:
+        """OpenMP threads the most recent call ran on."""
+        return int(self.lib.oracle_threads())
+
+
+def _load() -> OracleLib:
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = OracleLib(build())
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):  # a torch tensor: upcast exactly on the CPU
+        import torch
+        a = a.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _shape(q: np.ndarray):
+    if q.ndim != 4:
+        raise ValueError("expected [B, H, T, D]")
+    return tuple(int(s) for s in q.shape)
+
+
+def attn_fwd(q, k, v, scale=None):
+    """Returns (O [B,H,T,D], lse [B,H,T]) in float64."""
+    return _load().attn_fwd(q, k, v, scale)
+
+
+def attn_probs(q, k, scale=None):
+    """The causal softmax matrices P [B,H,T,T] (zero above the diagonal)."""
+    return _load().attn_probs(q, k, scale)
+
+
+def attn_bwd(q, k, v, do, scale=None):
+    """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
+    return _load().attn_bwd(q, k, v, do, scale)
+
+
+def threads_used() -> int:
+    """OpenMP threads the most recent oracle call ran on."""
+    return _load().threads_used()
+
+
+def source_path() -> str:
+    return _SRC

@@ -1,0 +1,196 @@
+/*
+ * attn_oracle.c -- plain, slow, double-precision CPU oracle of multi-head
+ * causal scaled dot-product self-attention, forward and backward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call this:
+ * only the tests, the smoke check and the bench's CPU-baseline leg load it.
+ * It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes, per head (b, h), for rows i and columns j of [T, T]:
+ *
+ *   S_ij = scale * <q_i, k_j>              affinity = dot product of a token's
+ *                                          query with the keys of the tokens
+ *                                          up to it, divided by sqrt(head dim)
+ *   S_ij = -inf for j > i                  upper triangle masked before the
+ *                                          softmax: no look into the future
+ *   P_i. = softmax(S_i.)                   row-normalised weights
+ *   O_i  = sum_j P_ij v_j                  values aggregated by the weights
+ *   lse_i = ln sum_{j<=i} exp(S_ij)        natural log, of the scaled scores
+ *
+ * Sources: "How Andrej Karpathy built GPT from 200 lines of code" (rdly.ru
+ * summary of the "Let's build GPT" video), section "Self-Attention: the
+ * mathematical trick" [43:56]-[55:20] (tril, row normalisation, -inf upper
+ * triangle, softmax) and section "Implementing the attention heads (Query,
+ * Key, Value)" [1:04:00]-[1:22:27] (query/key affinities, values, division by
+ * the square root of the head size, heads in parallel).  Heads are independent
+ * and dropout is 0 (nanoGPT skill card, Workflow 2 config: dropout = 0.0).
+ *
+ * The backward pass is the exact derivative of the forward for the loss
+ * L = sum(O * dO); the pages do not spell it out, so it is the textbook
+ * chain rule through O = P V and the row softmax:
+ *
+ *   dV_j  = sum_{i>=j} P_ij dO_i
+ *   dP_ij = <dO_i, v_j>
+ *   Delta_i = <dO_i, O_i>              (= sum_j P_ij dP_ij)
+ *   dS_ij = P_ij (dP_ij - Delta_i)
+ *   dQ_i  = scale * sum_{j<=i} dS_ij k_j
+ *   dK_j  = scale * sum_{i>=j} dS_ij q_i
+ *
+ * Layout: every tensor is [B, H, T, D] contiguous float64; lse is [B, H, T].
+ * No blocking, no fusion, no reordering beyond the definition.  The softmax
+ * subtracts the row maximum before exponentiating, which changes nothing in
+ * exact arithmetic and keeps exp() finite.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Row i of the causal softmax of one head: fills p[0..i] (p[j>i] untouched),
+ * returns lse_i.  q_i is one query row, kh the head's keys. */
+static double causal_softmax_row(const double *qi, const double *kh, int i, int D,
+                                 double scale, double *p)
+{
+    double m = -INFINITY;
+    for (int j = 0; j <= i; ++j) {
+        double s = 0.0;
+        for (int d = 0; d < D; ++d) s += qi[d] * kh[(int64_t)j * D + d];
+        s *= scale;
+        p[j] = s;
+        if (s > m) m = s;
+    }
+    double l = 0.0;
+    for (int j = 0; j <= i; ++j) {
+        p[j] = exp(p[j] - m);
+        l += p[j];
+    }
+    for (int j = 0; j <= i; ++j) p[j] /= l;
+    return m + log(l);
+}
+
+static int num_threads_used = 1;
+
+/* Number of OpenMP threads the last call ran on. */
+int oracle_threads(void) { return num_threads_used; }
+
+/* Forward: o [B,H,T,D], lse [B,H,T] (lse may be NULL). */
+void oracle_attn_fwd(const double *q, const double *k, const double *v,
+                     double *o, double *lse, int B, int H, int T, int D, double scale)
+{
+    const int64_t heads = (int64_t)B * H;
+    const int64_t hs = (int64_t)T * D;
+#pragma omp parallel
+    {
+#ifdef _OPENMP
+#pragma omp single
+        num_threads_used = omp_get_num_threads();
+#endif
+        double *p = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < heads; ++bh) {
+            const double *qh = q + bh * hs, *kh = k + bh * hs, *vh = v + bh * hs;
+            double *oh = o + bh * hs;
+            for (int i = 0; i < T; ++i) {
+                double li = causal_softmax_row(qh + (int64_t)i * D, kh, i, D, scale, p);
+                if (lse) lse[bh * T + i] = li;
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int j = 0; j <= i; ++j) acc += p[j] * vh[(int64_t)j * D + d];
+                    oh[(int64_t)i * D + d] = acc;
+                }
+            }
+        }
+        free(p);
+    }
+}
+
+/* The full probability matrices P [B,H,T,T] (zeros above the diagonal). */
+void oracle_attn_probs(const double *q, const double *k, double *p,
+                       int B, int H, int T, int D, double scale)
+{
+    const int64_t heads = (int64_t)B * H;
+    const int64_t hs = (int64_t)T * D;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < heads; ++bh) {
+        double *ph = p + bh * (int64_t)T * T;
+        memset(ph, 0, sizeof(double) * (size_t)T * (size_t)T);
+        for (int i = 0; i < T; ++i)
+            causal_softmax_row(q + bh * hs + (int64_t)i * D, k + bh * hs, i, D, scale,
+                               ph + (int64_t)i * T);
+    }
+}
+
+/* Backward: dq, dk, dv [B,H,T,D] from q, k, v and the upstream gradient dO.
+ * The forward (P, O) is recomputed here from q, k, v in double. */
+void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
+                     double *dq, double *dk, double *dv,
+                     int B, int H, int T, int D, double scale)
+{
+    const int64_t heads = (int64_t)B * H;
+    const int64_t hs = (int64_t)T * D;
+#pragma omp parallel
+    {
+#ifdef _OPENMP
+#pragma omp single
+        num_threads_used = omp_get_num_threads();
+#endif
+        const size_t tt = (size_t)(T > 0 ? T : 1) * (size_t)(T > 0 ? T : 1);
+        double *P = (double *)malloc(sizeof(double) * tt);    /* P_ij  */
+        double *dS = (double *)malloc(sizeof(double) * tt);   /* dS_ij */
+        double *O = (double *)malloc(sizeof(double) * (size_t)(hs > 0 ? hs : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < heads; ++bh) {
+            const double *qh = q + bh * hs, *kh = k + bh * hs, *vh = v + bh * hs;
+            const double *gh = dO + bh * hs;
+            double *dqh = dq + bh * hs, *dkh = dk + bh * hs, *dvh = dv + bh * hs;
+            memset(P, 0, sizeof(double) * tt);
+            memset(dS, 0, sizeof(double) * tt);
+            /* forward recompute: P and O */
+            for (int i = 0; i < T; ++i) {
+                causal_softmax_row(qh + (int64_t)i * D, kh, i, D, scale, P + (int64_t)i * T);
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int j = 0; j <= i; ++j) acc += P[(int64_t)i * T + j] * vh[(int64_t)j * D + d];
+                    O[(int64_t)i * D + d] = acc;
+                }
+            }
+            /* dV_j = sum_{i>=j} P_ij dO_i */
+            for (int j = 0; j < T; ++j)
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int i = j; i < T; ++i) acc += P[(int64_t)i * T + j] * gh[(int64_t)i * D + d];
+                    dvh[(int64_t)j * D + d] = acc;
+                }
+            /* dS_ij = P_ij (dP_ij - Delta_i), dP_ij = <dO_i, v_j>, Delta_i = <dO_i, O_i> */
+            for (int i = 0; i < T; ++i) {
+                double delta = 0.0;
+                for (int d = 0; d < D; ++d) delta += gh[(int64_t)i * D + d] * O[(int64_t)i * D + d];
+                for (int j = 0; j <= i; ++j) {
+                    double dp = 0.0;
+                    for (int d = 0; d < D; ++d) dp += gh[(int64_t)i * D + d] * vh[(int64_t)j * D + d];
+                    dS[(int64_t)i * T + j] = P[(int64_t)i * T + j] * (dp - delta);
+                }
+            }
+            /* dQ_i = scale * sum_{j<=i} dS_ij k_j */
+            for (int i = 0; i < T; ++i)
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int j = 0; j <= i; ++j) acc += dS[(int64_t)i * T + j] * kh[(int64_t)j * D + d];
+                    dqh[(int64_t)i * D + d] = scale * acc;
+                }
+            /* dK_j = scale * sum_{i>=j} dS_ij q_i */
+            for (int j = 0; j < T; ++j)
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int i = j; i < T; ++i) acc += dS[(int64_t)i * T + j] * qh[(int64_t)i * D + d];
+                    dkh[(int64_t)j * D + d] = scale * acc;
+                }
+        }
+        free(P);
+        free(dS);
+        free(O);
+    }
+}

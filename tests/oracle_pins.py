@@ -1,0 +1,200 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each check takes an oracle implementation (an object with ``attn_fwd``,
+``attn_bwd`` and ``attn_probs``) and raises AssertionError on a violation, so
+that the same checks run on the committed oracle and on deliberately broken
+variants of it (see test_oracle_mutations.py).
+
+What pins what:
+
+* rows of P sum to 1 and P is zero above the diagonal -- the softmax replaces
+  the row-normalised lower-triangular matrix ("How Andrej Karpathy built GPT
+  from 200 lines of code", section "Self-Attention: the mathematical trick",
+  [51:04] and [55:20]);
+* Q = 0 (or K = 0) turns causal attention into the averaging trick: every
+  token gets the mean of the values of the tokens up to it (same section,
+  [43:56]-[51:04]); closed forms follow for O, lse, dV, dK and dQ;
+* perturbing tokens after t leaves O, lse and dQ at rows <= t bit-identical
+  (the -inf upper triangle, [55:20]);
+* T = 1 returns V exactly and lse = scale * <q, k>;
+* adding one vector u to every key leaves P, O, dV, dK, dQ unchanged and adds
+  scale * <q_i, u> to lse_i (softmax shift invariance);
+* central finite differences of L = sum(O * dO) match dQ, dK, dV;
+* torch's float64 CPU ``scaled_dot_product_attention(is_causal=True)`` and its
+  autograd, a library routine used as an independent witness;
+* small hand-derived golden examples under tests/golden/.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def check_probs_rows(impl, seed=1):
+    r = _rng(seed)
+    B, H, T, D = 2, 3, 17, 5
+    q, k = r.standard_normal((B, H, T, D)), r.standard_normal((B, H, T, D)) * 3.0
+    p = impl.attn_probs(q, k)
+    assert np.all(np.abs(p.sum(-1) - 1.0) <= 1e-14), "rows of P must sum to 1"
+    upper = np.triu(np.ones((T, T), dtype=bool), 1)
+    assert np.all(p[..., upper] == 0.0), "P must be zero above the diagonal"
+    assert np.all(p[..., ~upper] > 0.0), "P must be positive on and below the diagonal"
+
+
+def check_averaging_trick(impl, seed=2):
+    """Q = 0 (then K = 0): all scores equal, so P is the row-normalised tril."""
+    r = _rng(seed)
+    B, H, T, D = 2, 2, 11, 6
+    k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(3))
+    scale = 1.0 / math.sqrt(D)
+    n = np.arange(1, T + 1, dtype=np.float64)              # i + 1
+    prefix_mean = np.cumsum(v, axis=2) / n[:, None]
+
+    zero = np.zeros_like(k)
+    o, lse = impl.attn_fwd(zero, k, v)
+    np.testing.assert_allclose(o, prefix_mean, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, np.broadcast_to(np.log(n), lse.shape), rtol=0, atol=1e-14)
+
+    dq, dk, dv = impl.attn_bwd(zero, k, v, do)
+    # dV_j = sum_{i >= j} dO_i / (i + 1): a reversed cumulative sum
+    w = do / n[:, None]
+    dv_ref = np.flip(np.cumsum(np.flip(w, axis=2), axis=2), axis=2)
+    np.testing.assert_allclose(dv, dv_ref, rtol=0, atol=1e-13)
+    assert np.all(dk == 0.0), "Q = 0 must give dK = 0 exactly"
+    # dQ_i = scale/(i+1) * sum_{j<=i} (<dO_i, v_j> - <dO_i, O_i>) k_j
+    g = np.einsum("bhid,bhjd->bhij", do, v)                # <dO_i, v_j>
+    delta = np.einsum("bhid,bhid->bhi", do, prefix_mean)
+    tril = np.tril(np.ones((T, T)))
+    ds = (g - delta[..., None]) * tril / n[:, None]
+    dq_ref = scale * np.einsum("bhij,bhjd->bhid", ds, k)
+    np.testing.assert_allclose(dq, dq_ref, rtol=0, atol=1e-13)
+
+    # K = 0: the same uniform weights; dQ = 0 exactly, dK by the transposed sum
+    q = r.standard_normal((B, H, T, D))
+    o2, lse2 = impl.attn_fwd(q, zero, v)
+    np.testing.assert_allclose(o2, prefix_mean, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse2, np.broadcast_to(np.log(n), lse2.shape), rtol=0, atol=1e-14)
+    dq2, dk2, dv2 = impl.attn_bwd(q, zero, v, do)
+    assert np.all(dq2 == 0.0), "K = 0 must give dQ = 0 exactly"
+    np.testing.assert_allclose(dv2, dv_ref, rtol=0, atol=1e-13)
+    dk_ref = scale * np.einsum("bhij,bhid->bhjd", ds, q)
+    np.testing.assert_allclose(dk2, dk_ref, rtol=0, atol=1e-13)
+
+
+def check_causality(impl, seed=3):
+    r = _rng(seed)
+    B, H, T, D = 1, 3, 13, 4
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    o, lse = impl.attn_fwd(q, k, v)
+    dq, _, _ = impl.attn_bwd(q, k, v, do)
+    for t in (0, 5, T - 2):
+        q2, k2, v2, do2 = (a.copy() for a in (q, k, v, do))
+        for a in (q2, k2, v2, do2):
+            a[:, :, t + 1:] += 10.0 * r.standard_normal(a[:, :, t + 1:].shape)
+        o2, lse2 = impl.attn_fwd(q2, k2, v2)
+        dq2, _, _ = impl.attn_bwd(q2, k2, v2, do2)
+        assert np.array_equal(o2[:, :, :t + 1], o[:, :, :t + 1]), f"O_<= {t} saw the future"
+        assert np.array_equal(lse2[:, :, :t + 1], lse[:, :, :t + 1]), f"lse_<= {t} saw the future"
+        assert np.array_equal(dq2[:, :, :t + 1], dq[:, :, :t + 1]), f"dQ_<= {t} saw the future"
+        assert not np.array_equal(o2[:, :, t + 1:], o[:, :, t + 1:])
+
+
+def check_single_token(impl, seed=4):
+    r = _rng(seed)
+    B, H, T, D = 3, 2, 1, 7
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    scale = 1.0 / math.sqrt(D)
+    o, lse = impl.attn_fwd(q, k, v)
+    assert np.array_equal(o, v), "T = 1 must return V exactly"
+    np.testing.assert_allclose(lse, scale * np.sum(q * k, -1), rtol=1e-15, atol=1e-15)
+    dq, dk, dv = impl.attn_bwd(q, k, v, do)
+    assert np.array_equal(dv, do), "T = 1 must give dV = dO"
+    np.testing.assert_allclose(dq, 0.0, atol=1e-15)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-15)
+
+
+def check_shift_invariance(impl, seed=5):
+    r = _rng(seed)
+    B, H, T, D = 2, 2, 9, 5
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    u = 4.0 * r.standard_normal((B, H, 1, D))
+    scale = 1.0 / math.sqrt(D)
+    o, lse = impl.attn_fwd(q, k, v)
+    o2, lse2 = impl.attn_fwd(q, k + u, v)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse2, lse + scale * np.sum(q * u, -1), rtol=0, atol=1e-12)
+    g, g2 = impl.attn_bwd(q, k, v, do), impl.attn_bwd(q, k + u, v, do)
+    for a, b in zip(g, g2):
+        np.testing.assert_allclose(b, a, rtol=0, atol=1e-12)
+
+
+def check_finite_differences(impl, seed=6):
+    r = _rng(seed)
+    B, H, T, D = 1, 2, 5, 3
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    dq, dk, dv = impl.attn_bwd(q, k, v, do)
+
+    def loss(q_, k_, v_):
+        return float(np.sum(impl.attn_fwd(q_, k_, v_)[0] * do))
+
+    h = 1e-6
+    for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+        fd = np.zeros_like(grad)
+        for idx in np.ndindex(*grad.shape):
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[which][idx] += h
+            lp = loss(args["q"], args["k"], args["v"])
+            args[which][idx] -= 2 * h
+            lm = loss(args["q"], args["k"], args["v"])
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.linalg.norm(fd - grad) / max(np.linalg.norm(grad), 1e-300)
+        assert err <= 1e-7, f"d{which}: finite differences disagree (rel {err:.2e})"
+
+
+def check_torch_witness(impl, seed=7):
+    import torch
+    r = _rng(seed)
+    B, H, T, D = 2, 3, 33, 16
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True)
+    to.backward(torch.tensor(do))
+    o, lse = impl.attn_fwd(q, k, v)
+    dq, dk, dv = impl.attn_bwd(q, k, v, do)
+    np.testing.assert_allclose(o, to.detach().numpy(), rtol=0, atol=1e-12)
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-12)
+    s = torch.tensor(q) @ torch.tensor(k).transpose(-1, -2) / math.sqrt(D)
+    s = s.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), rtol=0, atol=1e-12)
+
+
+def check_golden(impl):
+    for name in sorted(os.listdir(GOLDEN)):
+        if not name.endswith(".json"):
+            continue
+        with open(os.path.join(GOLDEN, name)) as f:
+            g = json.load(f)
+        arr = lambda key: np.asarray(g[key], dtype=np.float64)[None, None]
+        q, k, v = arr("q"), arr("k"), arr("v")
+        o, lse = impl.attn_fwd(q, k, v, g.get("scale"))
+        np.testing.assert_allclose(o[0, 0], np.asarray(g["o"]), rtol=0, atol=g["atol"], err_msg=name)
+        np.testing.assert_allclose(lse[0, 0], np.asarray(g["lse"]), rtol=0, atol=g["atol"], err_msg=name)
+        if "do" in g:
+            dq, dk, dv = impl.attn_bwd(q, k, v, arr("do"), g.get("scale"))
+            for key, got in (("dq", dq), ("dk", dk), ("dv", dv)):
+                np.testing.assert_allclose(got[0, 0], np.asarray(g[key]), rtol=0, atol=g["atol"],
+                                           err_msg=f"{name}:{key}")
+
+
+ALL_PINS = [check_probs_rows, check_averaging_trick, check_causality, check_single_token,
+            check_shift_invariance, check_finite_differences, check_torch_witness, check_golden]

@@ -1,0 +1,45 @@
+"""Plant plausible mistakes in a copy of the oracle's C source, on the CPU,
+and check that the pins catch every one of them."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+MUTATIONS = {
+    "scale_dropped": ("s *= scale;", "s *= 1.0;"),
+    "lse_log2": ("return m + log(l);", "return m + log2(l);"),
+    "softmax_not_normalised": ("for (int j = 0; j <= i; ++j) p[j] /= l;", ""),
+    "pv_wrong_value_row": ("acc += p[j] * vh[(int64_t)j * D + d];", "acc += p[j] * vh[(int64_t)i * D + d];"),
+    "dv_transposed_p": ("acc += P[(int64_t)i * T + j] * gh[(int64_t)i * D + d];",
+                        "acc += P[(int64_t)j * T + i] * gh[(int64_t)i * D + d];"),
+    "ds_sign_flipped": ("(dp - delta)", "(delta - dp)"),
+    "ds_delta_dropped": ("(dp - delta)", "(dp)"),
+    "dk_uses_k": ("acc += dS[(int64_t)i * T + j] * qh[(int64_t)i * D + d];",
+                  "acc += dS[(int64_t)i * T + j] * kh[(int64_t)i * D + d];"),
+    "dq_scale_dropped": ("dqh[(int64_t)i * D + d] = scale * acc;", "dqh[(int64_t)i * D + d] = acc;"),
+    "dq_transposed_ds": ("acc += dS[(int64_t)i * T + j] * kh[(int64_t)j * D + d];",
+                         "acc += dS[(int64_t)j * T + i] * kh[(int64_t)j * D + d];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(oracle.source_path()).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} must be unique"
+    path = tmp_path / "mut.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / f"libmut_{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", str(lib),
+                           str(path), "-lm"])
+    impl = oracle.OracleLib(str(lib))
+    caught = []
+    for check in oracle_pins.ALL_PINS:
+        try:
+            check(impl)
+        except AssertionError:
+            caught.append(check.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
