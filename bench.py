@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Throughput of multi-head causal attention, forward + backward, on B200.
+
+One step = the GPT-2 124M attention workload of one training step: 12
+independent layer instances (B=12, H=12, T=1024, D=64, bf16), 12 forwards
+(layer 1 -> 12) then 12 backwards (layer 12 -> 1) on one stream, every
+layer on its own buffers (inputs and outputs of a step touch ~2.3 GB, far
+more than the 126 MB L2, so no L2 flush is needed between steps).
+
+FLOPs are the algorithmic causal count 12 * D per attended pair (4 D forward:
+QK^T, PV; 8 D backward: dV, dP, dK, dQ), i.e. the causal half of the
+12 * L * H * Q * T per-token attention term of nanoGPT's estimate_mfu; the
+backward's recompute of P is not credited.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  Under torchrun every rank runs an independent
+replica on its own inputs (attention has no cross-rank exchange), the time is
+the max over ranks and the value is the total FLOPs of all ranks / that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal attention fwd+bwd TFLOP/s (bf16, GPT-2-124M shape), % of tensor peak"
+WORKLOAD = "gpt2_124m"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--e2e-steps", type=int, default=5, help="steps of the host-buffer end-to-end leg")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w, layers):
+    return {
+        "workload": f"{w.name}: causal multi-head attention fwd+bwd, B={w.B} H={w.H} T={w.T} "
+                    f"D={w.D}, {layers} independent layer instances per step",
+        "B": w.B, "H": w.H, "T": w.T, "D": w.D, "layers": layers,
+        "flops_per_step": w.flops() * layers,
+        "flop_convention": "12*D per causal pair (4D fwd + 8D bwd), P recompute not credited",
+        "l2": "inputs larger than L2 (each step touches ~2.3 GB of distinct buffers)",
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+        self.first = threading.Event()
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            self.first.set()
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        self.first.wait(timeout=10)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+            self.first.set()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0: float, t1: float):
+        sm, smax, reasons = [], None, set()
+        for ts, line in self.lines:
+            if ts < t0 or ts > t1 + 0.15:
+                continue
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "decoder_only_transformer_sdpa_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------ CPU oracle leg
+
+def oracle_sample(w, seed, n_heads):
+    """Inputs of n_heads whole heads of layer 0 of the workload (float64)."""
+    import numpy as np
+    from workloads import make_inputs
+    inp = make_inputs(w, seed=seed, layer=0)
+    B, H, T, D = w.B, w.H, w.T, w.D
+    idx = np.linspace(0, B * H - 1, n_heads).round().astype(int)
+    return {n: t.double().numpy().reshape(B * H, T, D)[idx][None] for n, t in inp.items()}
+
+
+def time_oracle_step(sample):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.attn_fwd(sample["q"], sample["k"], sample["v"])
+    oracle.attn_bwd(sample["q"], sample["k"], sample["v"], sample["do"])
+    return time.perf_counter() - t0, oracle.threads_used()
+
+
+def cpu_baseline(w, seed):
+    """The oracle as it stands, timed on this host's cores on a bounded
+    sample of the workload (about four whole heads per core)."""
+    import oracle
+    oracle.build()
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    n_heads = max(1, min(w.B * w.H, 4 * threads))
+    sample = oracle_sample(w, seed, n_heads)
+    dt, cores = time_oracle_step(sample)
+    flops = 12 * w.D * n_heads * w.T * (w.T + 1) // 2
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_heads} of {w.B * w.H} heads of layer 1 (T={w.T}, D={w.D}), fwd+bwd in "
+                      f"float64, {dt:.1f} s"}
+
+
+def run_reference(args, w):
+    """The reference arm: the CPU oracle (plain double-precision C) timed as
+    it stands on this host, on the same workload config, one bounded sample
+    of whole heads per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    n_heads = max(1, min(w.B * w.H, threads))
+    sample = oracle_sample(w, args.seed, n_heads)
+    for _ in range(args.warmup):
+        time_oracle_step(sample)
+    times, cores = [], 1
+    for _ in range(args.steps):
+        dt, cores = time_oracle_step(sample)
+        times.append(dt)
+    total = sum(times)
+    flops = 12 * w.D * n_heads * w.T * (w.T + 1) // 2 * len(times)
+    value = flops / total / 1e12
+    desc = (f"{n_heads} of {w.B * w.H} heads of layer 1 per step (T={w.T}, D={w.D}), fwd+bwd in "
+            f"float64 on {cores} threads")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, w.layers), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU leg
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    import decoder_only_transformer_sdpa_b200 as A
+    from workloads import make_inputs
+
+    L = w.layers
+    peaks, peak_kind = load_peaks()
+    # ---- inputs, outputs and workspaces of every layer, resident in HBM
+    layers = []
+    for l in range(L):
+        inp = make_inputs(w, seed=args.seed + 7919 * rank, layer=l)
+        q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+        layers.append(dict(
+            q=q, k=k, v=v, do=do, o=torch.empty_like(q),
+            lse=torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev),
+            dq=torch.empty_like(q), dk=torch.empty_like(q), dv=torch.empty_like(q),
+            ws=torch.empty(A.attn_bwd_workspace_bytes(w.B, w.H, w.T, w.D), dtype=torch.uint8,
+                           device=dev)))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_fwd=None, ev_bwd=None):
+        launches = 0
+        for l, b in enumerate(layers):
+            if ev_fwd is not None:
+                A.attn_profile_next_call(*ev_fwd[l])
+            A.attn_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"])
+            launches += A.attn_last_launch_count()
+        for l in range(L - 1, -1, -1):
+            b = layers[l]
+            if ev_bwd is not None:
+                A.attn_profile_next_call(*ev_bwd[l])
+            A.attn_bwd(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"], b["dv"],
+                       workspace=b["ws"])
+            launches += A.attn_last_launch_count()
+        return launches
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    barrier()
+    if A.attn_device_error() != 0:
+        raise RuntimeError("a bounded in-kernel wait timed out during warm-up")
+
+    # ---- timed region: K steps, events on the launching stream
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [([(mk(), mk()) for _ in range(L)], [(mk(), mk()) for _ in range(L)]) for _ in range(args.steps)]
+    sampler = ClockSampler(gpu_uuid(torch, dev))
+    sampler.start()
+    barrier()
+    t_wall0 = time.time()
+    start, end = mk(), mk()
+    start.record(stream)
+    launches = 0
+    for s in range(args.steps):
+        launches += step(*ev[s])
+    end.record(stream)
+    barrier()
+    t_wall1 = time.time()
+    sampler.stop()
+    ms = start.elapsed_time(end)
+    if A.attn_device_error() != 0:
+        raise RuntimeError("a bounded in-kernel wait timed out in the timed region")
+
+    fwd_ms = [a.elapsed_time(b) for e in ev for a, b in e[0]]
+    bwd_ms = [a.elapsed_time(b) for e in ev for a, b in e[1]]
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    flops_step = w.flops() * L
+    value = flops_step * world * args.steps / (ms_max * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel (the one with the larger total time)
+    pairs = w.causal_pairs()
+    kern = {
+        "attn_fwd": dict(ms=statistics.mean(fwd_ms), flops=4 * w.D * pairs, total=sum(fwd_ms)),
+        "attn_bwd": dict(ms=statistics.mean(bwd_ms), flops=8 * w.D * pairs, total=sum(bwd_ms)),
+    }
+    dom = max(kern, key=lambda n: kern[n]["total"])
+    peak = float(peaks.get("bf16_tflops"))
+    achieved = kern[dom]["flops"] / (kern[dom]["ms"] * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": f"{dom} main kernel", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                "traffic": measured_traffic(dom),
+                "algorithmic_flops_per_launch": kern[dom]["flops"],
+                "avg_launch_ms": kern[dom]["ms"],
+                "other": {n: {"avg_launch_ms": kern[n]["ms"],
+                              "tflops": kern[n]["flops"] / (kern[n]["ms"] * 1e-3) / 1e12}
+                          for n in kern}}
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        host = [{n: b[n].cpu().pin_memory() for n in ("q", "k", "v", "do")} for b in layers]
+        out_host = [{n: torch.empty(b["q"].shape, dtype=b["q"].dtype).pin_memory()
+                     for n in ("o", "dq", "dk", "dv")} for b in layers]
+        h2d = sum(t.numel() * t.element_size() for hb in host for t in hb.values())
+        d2h = sum(t.numel() * t.element_size() for hb in out_host for t in hb.values())
+
+        def e2e_step():
+            for l, b in enumerate(layers):
+                for n in ("q", "k", "v", "do"):
+                    b[n].copy_(host[l][n], non_blocking=True)
+                A.attn_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"])
+            for l in range(L - 1, -1, -1):
+                b = layers[l]
+                A.attn_bwd(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"],
+                           b["dv"], workspace=b["ws"])
+                for n in ("o", "dq", "dk", "dv"):
+                    out_host[l][n].copy_(b[n], non_blocking=True)
+        e2e_step()
+        barrier()
+        s0, s1 = mk(), mk()
+        s0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        barrier()
+        te = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item())
+        e2e = {"value": flops_step * world * args.e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.seed)
+
+    if rank == 0:
+        clocks = sampler.summary(t_wall0, t_wall1)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(w, L),
+            "pct_of_peak": {"measured_burst": value / world / peak,
+                            "measured_sustained": value / world / float(peaks.get("bf16_tflops_sustained", peak)),
+                            "datasheet_2250": value / world / 2250.0},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    from workloads import WORKLOADS
+    w = WORKLOADS[WORKLOAD]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,199 @@
+"""Python binding of libattn.so: multi-head causal scaled dot-product
+self-attention, forward and backward, on B200 (sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/attn.h.  PyTorch supplies device
+memory and the current CUDA stream.  There is no CPU or library fallback: if
+the shared library is missing, importing this package raises ImportError.
+
+Functions mirror the C entry points and take [B, H, T, D] contiguous CUDA
+tensors (bf16 for ``attn_fwd``/``attn_bwd``, float32 for the ``_f32`` pair);
+outputs may be passed in or are allocated.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is not built; run `python decoder_only_transformer_sdpa_b200/build.py` "
+        "(nvcc, sm_100a). There is no fallback implementation.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _fp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_lib.attn_status_string.argtypes = [_i]
+_lib.attn_status_string.restype = ctypes.c_char_p
+_lib.attn_version.restype = _i
+_lib.attn_last_launch_count.restype = _i
+_lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _f, _vp]
+_lib.attn_fwd.restype = _i
+_lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
+_lib.attn_bwd_workspace_bytes.restype = _sz
+_lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]
+_lib.attn_bwd.restype = _i
+_lib.attn_fwd_f32.argtypes = [_fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _vp]
+_lib.attn_fwd_f32.restype = _i
+_lib.attn_bwd_f32_workspace_bytes.argtypes = [_i, _i, _i, _i]
+_lib.attn_bwd_f32_workspace_bytes.restype = _sz
+_lib.attn_bwd_f32.argtypes = [_fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _vp, _sz, _vp]
+_lib.attn_bwd_f32.restype = _i
+_lib.attn_device_error.argtypes = [_vp]
+_lib.attn_device_error.restype = _i
+_lib.attn_profile_next_call.argtypes = [_vp, _vp]
+_lib.attn_profile_next_call.restype = _i
+
+EXPORTED = ("attn_status_string", "attn_version", "attn_last_launch_count", "attn_fwd",
+            "attn_bwd_workspace_bytes", "attn_bwd", "attn_fwd_f32", "attn_bwd_f32_workspace_bytes",
+            "attn_bwd_f32", "attn_device_error", "attn_profile_next_call")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {attn_status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The raw ctypes handle of libattn.so."""
+    return _lib
+
+
+def attn_status_string(status: int) -> str:
+    return _lib.attn_status_string(int(status)).decode()
+
+
+def attn_version() -> int:
+    return int(_lib.attn_version())
+
+
+def attn_last_launch_count() -> int:
+    """Kernels enqueued by the most recent successful call on this thread."""
+    return int(_lib.attn_last_launch_count())
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> int:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check(t, name, dtype, shape=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _shape4(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, T, D]")
+    return tuple(int(s) for s in q.shape)
+
+
+def _raise(status: int, where: str):
+    if status != 0:
+        raise AttnError(status, where)
+
+
+def _fwd(cfn, dtype, q, k, v, o, lse, scale, stream):
+    torch = _torch()
+    B, H, T, D = _shape4(q)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    ptrs = [_check(q, "q", dtype), _check(k, "k", dtype, q.shape), _check(v, "v", dtype, q.shape),
+            _check(o, "o", dtype, q.shape), _check(lse, "lse", torch.float32, (B, H, T))]
+    with torch.cuda.device(q.device):
+        _raise(cfn(*ptrs, B, H, T, D, scale, _stream_handle(stream)), cfn.__name__)
+    return o, lse
+
+
+def _bwd(cfn, ws_fn, dtype, q, k, v, o, lse, dO, dq, dk, dv, scale, workspace, stream):
+    torch = _torch()
+    B, H, T, D = _shape4(q)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    need = int(ws_fn(B, H, T, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ptrs = [_check(q, "q", dtype), _check(k, "k", dtype, q.shape), _check(v, "v", dtype, q.shape),
+            _check(o, "o", dtype, q.shape), _check(lse, "lse", torch.float32, (B, H, T)),
+            _check(dO, "dO", dtype, q.shape), _check(dq, "dq", dtype, q.shape),
+            _check(dk, "dk", dtype, q.shape), _check(dv, "dv", dtype, q.shape)]
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        _raise(cfn(*ptrs, B, H, T, D, scale, workspace.data_ptr(), ws_bytes, _stream_handle(stream)),
+               cfn.__name__)
+    return dq, dk, dv
+
+
+def attn_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, stream=None):
+    """bf16 forward on the tensor cores: returns (O bf16, lse float32 [B,H,T])."""
+    return _fwd(_lib.attn_fwd, _torch().bfloat16, q, k, v, o, lse, scale, stream)
+
+
+def attn_bwd_workspace_bytes(B: int, H: int, T: int, D: int) -> int:
+    return int(_lib.attn_bwd_workspace_bytes(B, H, T, D))
+
+
+def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[float] = None,
+             workspace=None, stream=None):
+    """bf16 backward: returns (dQ, dK, dV) bf16."""
+    return _bwd(_lib.attn_bwd, _lib.attn_bwd_workspace_bytes, _torch().bfloat16, q, k, v, o, lse,
+                dO, dq, dk, dv, scale, workspace, stream)
+
+
+def attn_fwd_f32(q, k, v, o=None, lse=None, scale: Optional[float] = None, stream=None):
+    """float32 forward on CUDA cores: returns (O, lse)."""
+    return _fwd(_lib.attn_fwd_f32, _torch().float32, q, k, v, o, lse, scale, stream)
+
+
+def attn_bwd_f32_workspace_bytes(B: int, H: int, T: int, D: int) -> int:
+    return int(_lib.attn_bwd_f32_workspace_bytes(B, H, T, D))
+
+
+def attn_bwd_f32(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[float] = None,
+                 workspace=None, stream=None):
+    """float32 backward: returns (dQ, dK, dV)."""
+    return _bwd(_lib.attn_bwd_f32, _lib.attn_bwd_f32_workspace_bytes, _torch().float32, q, k, v, o,
+                lse, dO, dq, dk, dv, scale, workspace, stream)
+
+
+def attn_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the in-kernel error flag
+    status: 0, or the timeout status if a bounded wait ran out."""
+    return int(_lib.attn_device_error(_stream_handle(stream)))
+
+
+def attn_profile_next_call(start=None, end=None) -> None:
+    """Arm the next attn_fwd/attn_bwd call on this thread to record the two
+    torch.cuda.Event objects around its main kernel, on the call's stream."""
+    h = lambda ev: None if ev is None else int(ev.cuda_event)
+    _raise(_lib.attn_profile_next_call(h(start), h(end)), "attn_profile_next_call")

@@ -1,0 +1,251 @@
+// attn_api.cu -- the extern "C" entry points of libattn.so (declared in
+// include/attn.h): argument validation, workspace carving and dispatch to the
+// kernels.  Nothing here computes attention; every step runs in a kernel.
+#include "../../include/attn.h"
+#include "internal.h"
+
+#include <math.h>
+#include <mutex>
+
+#define ATTN_API extern "C" __attribute__((visibility("default")))
+
+namespace attn {
+namespace {
+
+// Device-side error word.  Kernels receive its address as an argument (one
+// address per device, looked up once) and set it when a bounded wait runs out.
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int *g_err_addr[kMaxDevices];
+int g_cc_major[kMaxDevices];  // 0 = not yet queried
+
+thread_local int t_last_launches = 0;
+thread_local cudaEvent_t t_prof_start = nullptr, t_prof_end = nullptr;
+
+// Takes the armed profiling events (if any) for the call being made.
+LaunchInfo take_launch_info() {
+    LaunchInfo li;
+    li.main_start = t_prof_start;
+    li.main_end = t_prof_end;
+    t_prof_start = t_prof_end = nullptr;
+    return li;
+}
+
+int current_device(int &dev) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_DEVICE;
+    return ATTN_OK;
+}
+
+// Checks the current device is sm_100 and returns its error-word address.
+int device_setup(int **err_addr) {
+    int dev;
+    int st = current_device(dev);
+    if (st != ATTN_OK) return st;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_cc_major[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        if (major != 10 || minor != 0) {
+            g_cc_major[dev] = -1;
+        } else {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return ATTN_ERR_CUDA;
+            g_err_addr[dev] = static_cast<int *>(p);
+            g_cc_major[dev] = major;
+        }
+    }
+    if (g_cc_major[dev] < 0) return ATTN_ERR_DEVICE;
+    if (err_addr) *err_addr = g_err_addr[dev];
+    return ATTN_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(int B, int H, int T, int D, int dmax) {
+    if (B < 1 || H < 1 || T < 1) return ATTN_ERR_SHAPE;
+    if (D < 1 || D > dmax) return ATTN_ERR_UNSUPPORTED_D;
+    const long double n = (long double)B * H * T * D;
+    if (n > (long double)(1ll << 40)) return ATTN_ERR_SHAPE;
+    if ((long long)B * H > 0x7fffffffLL / 8) return ATTN_ERR_SHAPE;
+    return ATTN_OK;
+}
+
+int check_scale(float scale) {
+    return (isfinite(scale) && scale > 0.f) ? ATTN_OK : ATTN_ERR_SCALE;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int finish(cudaError_t e, const LaunchInfo &li) {
+    if (e != cudaSuccess) {
+        cudaGetLastError();  // clear a sticky launch error of this call
+        return ATTN_ERR_CUDA;
+    }
+    t_last_launches = li.kernels;
+    return ATTN_OK;
+}
+
+bool bf16_d_supported(int D) { return D == 32 || D == 64; }
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+ATTN_API const char *attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_NULL: return "a required pointer is NULL";
+        case ATTN_ERR_SHAPE: return "invalid shape (B, H, T must be >= 1; size overflow)";
+        case ATTN_ERR_UNSUPPORTED_D: return "unsupported head_dim";
+        case ATTN_ERR_ALIGN: return "pointer misaligned (bf16: 16 bytes, float32: 4 bytes)";
+        case ATTN_ERR_CUDA: return "CUDA error";
+        case ATTN_ERR_TIMEOUT: return "a bounded in-kernel wait timed out";
+        case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case ATTN_ERR_DEVICE: return "current device is not sm_100 (B200 class)";
+        case ATTN_ERR_SCALE: return "scale must be finite and positive";
+        default: return "unknown status";
+    }
+}
+
+ATTN_API int attn_version(void) { return 1; }
+
+ATTN_API int attn_profile_next_call(cudaEvent_t start, cudaEvent_t end) {
+    if ((start == nullptr) != (end == nullptr)) return ATTN_ERR_NULL;
+    t_prof_start = start;
+    t_prof_end = end;
+    return ATTN_OK;
+}
+
+ATTN_API int attn_last_launch_count(void) { return t_last_launches; }
+
+ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                      int H, int T, int D, float scale, cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    int st = check_shape(B, H, T, D, 64);
+    if (st != ATTN_OK) return st;
+    if (!bf16_d_supported(D)) return ATTN_ERR_UNSUPPORTED_D;
+    if ((st = check_scale(scale)) != ATTN_OK) return st;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return ATTN_ERR_ALIGN;
+    int *err = nullptr;
+    if ((st = device_setup(&err)) != ATTN_OK) return st;
+    cudaError_t e = sm100_fwd(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                              static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), lse,
+                              Shape{B, H, T, D, scale}, err, stream, li);
+    return finish(e, li);
+}
+
+// Workspace of the bf16 backward: dQ float32 accumulator, then Delta.
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
+    if (check_shape(B, H, T, D, 64) != ATTN_OK || !bf16_d_supported(D)) return 0;
+    const size_t rows = (size_t)B * H * T;
+    return round_up(rows * D * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+}
+
+ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                      const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D,
+                      float scale, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
+    int st = check_shape(B, H, T, D, 64);
+    if (st != ATTN_OK) return st;
+    if (!bf16_d_supported(D)) return ATTN_ERR_UNSUPPORTED_D;
+    if ((st = check_scale(scale)) != ATTN_OK) return st;
+    const void *ptrs[] = {q, k, v, o, dO, dq, dk, dv};
+    for (const void *p : ptrs)
+        if (!aligned(p, 16)) return ATTN_ERR_ALIGN;
+    if (!aligned(lse, 4)) return ATTN_ERR_ALIGN;
+    const size_t need = attn_bwd_workspace_bytes(B, H, T, D);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
+    int *err = nullptr;
+    if ((st = device_setup(&err)) != ATTN_OK) return st;
+    const size_t rows = (size_t)B * H * T;
+    float *dq_acc = static_cast<float *>(workspace);
+    float *delta = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                             round_up(rows * D * sizeof(float), 256));
+    cudaError_t e = sm100_bwd(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(o), lse,
+        static_cast<const __nv_bfloat16 *>(dO), static_cast<__nv_bfloat16 *>(dq),
+        static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv), dq_acc, delta,
+        Shape{B, H, T, D, scale}, err, stream, li);
+    return finish(e, li);
+}
+
+ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
+                          int B, int H, int T, int D, float scale, cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    int st = check_shape(B, H, T, D, 128);
+    if (st != ATTN_OK) return st;
+    if ((st = check_scale(scale)) != ATTN_OK) return st;
+    if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(o, 4) || !aligned(lse, 4))
+        return ATTN_ERR_ALIGN;
+    if ((st = device_setup(nullptr)) != ATTN_OK) return st;
+    cudaError_t e = simt_fwd<float>(q, k, v, o, lse, Shape{B, H, T, D, scale}, stream, li);
+    return finish(e, li);
+}
+
+ATTN_API size_t attn_bwd_f32_workspace_bytes(int B, int H, int T, int D) {
+    if (check_shape(B, H, T, D, 128) != ATTN_OK) return 0;
+    return round_up((size_t)B * H * T * sizeof(float), 256);
+}
+
+ATTN_API int attn_bwd_f32(const float *q, const float *k, const float *v, const float *o,
+                          const float *lse, const float *dO, float *dq, float *dk, float *dv, int B,
+                          int H, int T, int D, float scale, void *workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
+    int st = check_shape(B, H, T, D, 128);
+    if (st != ATTN_OK) return st;
+    if ((st = check_scale(scale)) != ATTN_OK) return st;
+    const void *ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
+    for (const void *p : ptrs)
+        if (!aligned(p, 4)) return ATTN_ERR_ALIGN;
+    const size_t need = attn_bwd_f32_workspace_bytes(B, H, T, D);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
+    if ((st = device_setup(nullptr)) != ATTN_OK) return st;
+    cudaError_t e = simt_bwd<float>(q, k, v, o, lse, dO, dq, dk, dv, static_cast<float *>(workspace),
+                                    Shape{B, H, T, D, scale}, stream, li);
+    return finish(e, li);
+}
+
+ATTN_API int attn_device_error(cudaStream_t stream) {
+    int *err = nullptr;
+    int st = device_setup(&err);
+    if (st != ATTN_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (h != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        return ATTN_ERR_TIMEOUT;
+    }
+    return ATTN_OK;
+}
+
+namespace attn {
+void *tensor_map_encoder() {
+    static void *fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = p;
+    });
+    return fn;
+}
+}  // namespace attn

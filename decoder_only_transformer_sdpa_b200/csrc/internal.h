@@ -1,0 +1,63 @@
+// internal.h -- declarations shared by the library's translation units (not
+// part of the public ABI; every symbol here has hidden visibility).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace attn {
+
+// Upper bound on the polls of any in-kernel wait (mbarrier or flag).  A wait
+// that runs out sets the device error word to kErrTimeout and the kernel
+// leaves by its normal exit path.  At ~1 poll per 20-100 ns this bounds a
+// stuck wait to a fraction of a second up to a few seconds.
+constexpr uint32_t kWaitLimit = 1u << 25;
+constexpr int kErrTimeout = 1;
+
+struct Shape {
+    int B, H, T, D;
+    float scale;
+};
+
+// Per-call bookkeeping: kernels enqueued, and the optional event pair to
+// record around the call's main kernel (see attn_profile_next_call).
+struct LaunchInfo {
+    int kernels = 0;
+    cudaEvent_t main_start = nullptr;
+    cudaEvent_t main_end = nullptr;
+};
+
+// Records li.main_start / li.main_end (when armed) around a main kernel.
+inline cudaError_t mark_main_start(const LaunchInfo &li, cudaStream_t st) {
+    return li.main_start ? cudaEventRecord(li.main_start, st) : cudaSuccess;
+}
+inline cudaError_t mark_main_end(const LaunchInfo &li, cudaStream_t st) {
+    return li.main_end ? cudaEventRecord(li.main_end, st) : cudaSuccess;
+}
+
+// ---- SIMT kernels (float32 math on CUDA cores), element type float or bf16
+template <typename T>
+cudaError_t simt_fwd(const T *q, const T *k, const T *v, T *o, float *lse, Shape s,
+                     cudaStream_t st, LaunchInfo &li);
+template <typename T>
+cudaError_t simt_bwd(const T *q, const T *k, const T *v, const T *o, const float *lse,
+                     const T *dO, T *dq, T *dk, T *dv, float *delta, Shape s,
+                     cudaStream_t st, LaunchInfo &li);
+
+// ---- tcgen05 / TMA kernels for bf16, D in {32, 64}
+cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                      __nv_bfloat16 *o, float *lse, Shape s, int *err, cudaStream_t st,
+                      LaunchInfo &li);
+cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                      const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
+                      __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv,
+                      float *dq_acc, float *delta, Shape s, int *err, cudaStream_t st,
+                      LaunchInfo &li);
+
+// Driver entry point for cuTensorMapEncodeTiled, resolved once at run time
+// through the runtime (so the library does not link libcuda directly).
+void *tensor_map_encoder();
+
+}  // namespace attn

@@ -1,0 +1,134 @@
+/*
+ * attn.h -- C ABI of libattn.so: multi-head causal scaled dot-product
+ * self-attention, forward and backward, on NVIDIA B200 (sm_100a).
+ *
+ * What it computes (per head, rows i and columns j of a T x T tile):
+ *
+ *   S_ij = scale * <q_i, k_j>  for j <= i, -inf above the diagonal
+ *   P    = row softmax of S,  O = P V,  lse_i = ln sum_{j<=i} exp(S_ij)
+ *
+ * "How Andrej Karpathy built GPT from 200 lines of code" (rdly.ru summary of
+ * the "Let's build GPT" video): section "Implementing the attention heads
+ * (Query, Key, Value)" -- affinities are the dot product of a token's query
+ * with the keys of the tokens up to it [1:06:16], divided by the square root
+ * of the head size [1:17:18], used to aggregate the values [1:10:15], several
+ * heads in parallel [1:22:27]; section "Self-Attention: the mathematical
+ * trick" -- the upper triangle is set to -inf before the softmax so a token
+ * cannot look into the future [55:20].  Dropout is 0 ("Model Architecture
+ * Nanogpt" skill card, Workflow 2 config), so there is no dropout argument.
+ * The backward pass is the exact derivative of the forward (the pages give no
+ * formula for it): dV = P^T dO, dS = P o (dO V^T - Delta), Delta_i =
+ * <dO_i, O_i>, dQ = scale dS K, dK = scale dS^T Q.
+ *
+ * Common rules for every entry point:
+ *
+ *  - Layout: q, k, v, o, dO, dq, dk, dv are [B, H, T, D] contiguous row-major
+ *    (D fastest); lse is [B, H, T] contiguous float32.
+ *  - All pointers are device pointers owned by the caller.  The library
+ *    allocates no device memory, never synchronises the stream and only
+ *    enqueues work on `stream` (NULL = the legacy default stream).
+ *  - bf16 entry points take __nv_bfloat16 data through `void *`; every tensor
+ *    pointer must be 16-byte aligned (TMA requirement).  float32 entry points
+ *    need 4-byte alignment.
+ *  - `scale` is normally 1/sqrt(D); any finite positive value is accepted.
+ *  - Argument errors are reported before anything is launched; a failed
+ *    launch is reported as ATTN_ERR_CUDA.  Faults inside a kernel surface
+ *    asynchronously at the caller's next synchronisation.  Every internal wait
+ *    of the kernels is bounded: a wait that runs out records a flag that
+ *    attn_device_error() returns as ATTN_ERR_TIMEOUT.
+ *  - Calls are thread-safe; tensor descriptors travel as kernel parameters.
+ *    Calls that write the same output buffers race like any CUDA work.
+ */
+#ifndef ATTN_H
+#define ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's own stream handle type (an opaque pointer). */
+typedef struct CUstream_st *cudaStream_t;
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = -1,          /* a required pointer is NULL                      */
+    ATTN_ERR_SHAPE = -2,         /* B, H or T < 1, or B*H*T*D overflows             */
+    ATTN_ERR_UNSUPPORTED_D = -3, /* head_dim outside the supported set              */
+    ATTN_ERR_ALIGN = -4,         /* a pointer misses its required alignment         */
+    ATTN_ERR_CUDA = -5,          /* a CUDA runtime/driver call or launch failed     */
+    ATTN_ERR_TIMEOUT = -6,       /* a bounded in-kernel wait ran out                */
+    ATTN_ERR_WORKSPACE = -7,     /* workspace NULL or smaller than required         */
+    ATTN_ERR_DEVICE = -8,        /* current device is not sm_100 (B200 class)       */
+    ATTN_ERR_SCALE = -9          /* scale is not finite and positive                */
+} attn_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *attn_status_string(int status);
+
+/* ---------------- bf16 path: tcgen05 tensor cores + TMA ------------------ */
+
+/* Forward.  q, k, v: bf16 inputs; o: bf16 output; lse: float32 output, the
+ * natural-log log-sum-exp of each row's scaled, masked scores (needed by
+ * attn_bwd).  D must be 32 or 64.  Any T >= 1. */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int H, int T, int D, float scale, cudaStream_t stream);
+
+/* Bytes of device workspace attn_bwd needs: a float32 dQ accumulator
+ * [B,H,T,D] plus Delta [B,H,T], each 256-byte aligned.  0 on a bad shape. */
+size_t attn_bwd_workspace_bytes(int B, int H, int T, int D);
+
+/* Backward.  q, k, v, o, lse: as given to / returned by attn_fwd; dO: bf16
+ * upstream gradient; dq, dk, dv: bf16 outputs (fully overwritten).
+ * workspace: caller-owned device scratch of at least
+ * attn_bwd_workspace_bytes(B,H,T,D) bytes, 256-byte aligned; its contents on
+ * entry do not matter and are clobbered.  D must be 32 or 64. */
+int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const void *dO, void *dq, void *dk, void *dv,
+             int B, int H, int T, int D, float scale,
+             void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------- float32 path: CUDA cores, IEEE expf -------------------- */
+
+/* Forward in float32 (all tensors float32).  1 <= D <= 128. */
+int attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
+                 int B, int H, int T, int D, float scale, cudaStream_t stream);
+
+/* Bytes of device workspace attn_bwd_f32 needs (Delta [B,H,T], float32). */
+size_t attn_bwd_f32_workspace_bytes(int B, int H, int T, int D);
+
+/* Backward in float32.  Same arguments as attn_bwd with float32 tensors. */
+int attn_bwd_f32(const float *q, const float *k, const float *v, const float *o,
+                 const float *lse, const float *dO, float *dq, float *dk, float *dv,
+                 int B, int H, int T, int D, float scale,
+                 void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------- diagnostics ------------------------------------------- */
+
+/* Synchronises `stream`, then reads and clears the current device's
+ * in-kernel error flag.  Returns ATTN_OK, ATTN_ERR_TIMEOUT (a bounded wait
+ * ran out since the last call) or ATTN_ERR_CUDA (the sync itself failed). */
+int attn_device_error(cudaStream_t stream);
+
+/* Number of kernels the most recent successful call on this host thread
+ * enqueued (for launch accounting). */
+int attn_last_launch_count(void);
+
+/* Timing hook: arms the next attn_fwd / attn_bwd call made on this host
+ * thread to record `start` just before and `end` just after enqueueing its
+ * main kernel (the forward kernel, or the backward's tile kernel), on the
+ * call's stream.  Both are cudaEvent_t handles owned by the caller; the call
+ * consumes the arming whether or not it succeeds.  Pass NULLs to disarm. */
+typedef struct CUevent_st *cudaEvent_t;
+int attn_profile_next_call(cudaEvent_t start, cudaEvent_t end);
+
+/* Library ABI version: 1. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H */

@@ -1,0 +1,115 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+symbol include/attn.h declares, and rejects bad arguments before touching
+CUDA (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decoder_only_transformer_sdpa_b200 as lib_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+OK, E_NULL, E_SHAPE, E_D, E_ALIGN, E_CUDA, E_TIMEOUT, E_WS, E_DEV, E_SCALE = 0, -1, -2, -3, -4, -5, -6, -7, -8, -9
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert {"attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_f32", "attn_bwd_f32",
+            "attn_status_string"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = lib_mod.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libattn.so does not export {name}"
+    assert set(declared_functions()) == set(lib_mod.EXPORTED)
+
+
+def test_exports_nothing_else():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_mod.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    funcs = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert funcs == set(declared_functions())
+
+
+def test_status_strings():
+    for s in (OK, E_NULL, E_SHAPE, E_D, E_ALIGN, E_CUDA, E_TIMEOUT, E_WS, E_DEV, E_SCALE, 12345):
+        assert isinstance(lib_mod.attn_status_string(s), str) and lib_mod.attn_status_string(s)
+    assert lib_mod.attn_version() == 1
+
+
+def test_workspace_sizes():
+    B, H, T, D = 12, 12, 1024, 64
+    rows = B * H * T
+    rnd = lambda x: (x + 255) // 256 * 256
+    assert lib_mod.attn_bwd_workspace_bytes(B, H, T, D) == rnd(rows * D * 4) + rnd(rows * 4)
+    assert lib_mod.attn_bwd_workspace_bytes(1, 1, 1, 32) == 256 + 256
+    assert lib_mod.attn_bwd_workspace_bytes(1, 1, 1, 48) == 0       # unsupported D
+    assert lib_mod.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0       # bad shape
+    assert lib_mod.attn_bwd_f32_workspace_bytes(4, 4, 8, 8) == rnd(4 * 4 * 8 * 4)
+    assert lib_mod.attn_bwd_f32_workspace_bytes(1, 1, 1, 129) == 0
+
+
+# Fake but well-aligned device addresses: every call below fails validation
+# before the library makes any CUDA call.
+P = 1 << 20
+
+
+def fwd(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, T=8, D=64, scale=0.125):
+    return lib_mod.lib().attn_fwd(q, k, v, o, lse, B, H, T, D, scale, None)
+
+
+def bwd(ptrs=None, B=1, H=1, T=8, D=64, scale=0.125, ws=P, ws_bytes=1 << 30):
+    p = [P] * 9 if ptrs is None else ptrs
+    return lib_mod.lib().attn_bwd(*p, B, H, T, D, scale, ws, ws_bytes, None)
+
+
+def fwd32(q=P, o=P, B=1, H=1, T=8, D=8, scale=0.3):
+    return lib_mod.lib().attn_fwd_f32(q, P, P, o, P, B, H, T, D, scale, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), E_NULL), (dict(lse=None), E_NULL),
+    (dict(B=0), E_SHAPE), (dict(H=-1), E_SHAPE), (dict(T=0), E_SHAPE),
+    (dict(D=48), E_D), (dict(D=128), E_D), (dict(D=0), E_D), (dict(D=16), E_D),
+    (dict(scale=0.0), E_SCALE), (dict(scale=float("nan")), E_SCALE), (dict(scale=-1.0), E_SCALE),
+    (dict(scale=float("inf")), E_SCALE),
+    (dict(q=P + 8), E_ALIGN), (dict(o=P + 2), E_ALIGN), (dict(lse=P + 2), E_ALIGN),
+    (dict(B=1 << 20, H=1 << 10, T=1 << 12), E_SHAPE),
+])
+def test_fwd_argument_errors(kw, expect):
+    assert fwd(**kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ptrs=[P] * 8 + [None]), E_NULL),
+    (dict(ptrs=[P] * 5 + [P + 8] + [P] * 3), E_ALIGN),
+    (dict(D=100), E_D),
+    (dict(ws=None), E_WS), (dict(ws_bytes=16), E_WS), (dict(ws=P + 16), E_WS),
+    (dict(T=0), E_SHAPE), (dict(scale=float("nan")), E_SCALE),
+])
+def test_bwd_argument_errors(kw, expect):
+    assert bwd(**kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), E_NULL), (dict(D=129), E_D), (dict(D=0), E_D), (dict(q=P + 2), E_ALIGN),
+    (dict(B=0), E_SHAPE), (dict(scale=-2.0), E_SCALE),
+])
+def test_fwd_f32_argument_errors(kw, expect):
+    assert fwd32(**kw) == expect
+
+
+def test_bwd_f32_workspace_error():
+    lib = lib_mod.lib()
+    assert lib.attn_bwd_f32(*([P] * 9), 1, 1, 8, 8, 0.3, P, 8, None) == E_WS
