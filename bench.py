@@ -303,6 +303,10 @@ def run_ours(args, w):
     # ---- timed region: K steps, events on the launching stream
     mk = lambda: torch.cuda.Event(enable_timing=True)
     ev = [([(mk(), mk()) for _ in range(L)], [(mk(), mk()) for _ in range(L)]) for _ in range(args.steps)]
+    for e in ev:  # torch creates the CUDA event on first record; the library re-records it
+        for pair in e[0] + e[1]:
+            for x in pair:
+                x.record(stream)
     sampler = ClockSampler(gpu_uuid(torch, dev))
     sampler.start()
     barrier()

@@ -46,12 +46,15 @@ _lib.attn_bwd_f32.argtypes = [_fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _i, _
 _lib.attn_bwd_f32.restype = _i
 _lib.attn_device_error.argtypes = [_vp]
 _lib.attn_device_error.restype = _i
+_lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _vp]
+_lib.attn_selftest_wait_timeout.restype = _i
 _lib.attn_profile_next_call.argtypes = [_vp, _vp]
 _lib.attn_profile_next_call.restype = _i
 
 EXPORTED = ("attn_status_string", "attn_version", "attn_last_launch_count", "attn_fwd",
             "attn_bwd_workspace_bytes", "attn_bwd", "attn_fwd_f32", "attn_bwd_f32_workspace_bytes",
-            "attn_bwd_f32", "attn_device_error", "attn_profile_next_call")
+            "attn_bwd_f32", "attn_device_error", "attn_profile_next_call",
+            "attn_selftest_wait_timeout")
 
 
 class AttnError(RuntimeError):
@@ -195,5 +198,17 @@ def attn_device_error(stream=None) -> int:
 def attn_profile_next_call(start=None, end=None) -> None:
     """Arm the next attn_fwd/attn_bwd call on this thread to record the two
     torch.cuda.Event objects around its main kernel, on the call's stream."""
-    h = lambda ev: None if ev is None else int(ev.cuda_event)
+    def h(ev):
+        if ev is None:
+            return None
+        handle = int(ev.cuda_event)
+        if handle == 0:
+            raise ValueError("the torch.cuda.Event has no CUDA event yet: record it once first")
+        return handle
     _raise(_lib.attn_profile_next_call(h(start), h(end)), "attn_profile_next_call")
+
+
+def attn_selftest_wait_timeout(polls: int = 1024, stream=None) -> None:
+    """Enqueue the bounded-wait failure self test (see include/attn.h)."""
+    _raise(_lib.attn_selftest_wait_timeout(int(polls), _stream_handle(stream)),
+           "attn_selftest_wait_timeout")

@@ -234,6 +234,14 @@ ATTN_API int attn_device_error(cudaStream_t stream) {
     return ATTN_OK;
 }
 
+ATTN_API int attn_selftest_wait_timeout(uint32_t polls, cudaStream_t stream) {
+    if (polls < 1 || polls > (1u << 22)) return ATTN_ERR_SHAPE;
+    int *err = nullptr;
+    int st = device_setup(&err);
+    if (st != ATTN_OK) return st;
+    return selftest_wait_timeout(polls, err, stream) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 namespace attn {
 void *tensor_map_encoder() {
     static void *fn = nullptr;

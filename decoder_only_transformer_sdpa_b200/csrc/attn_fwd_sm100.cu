@@ -1,0 +1,334 @@
+// attn_fwd_sm100.cu -- causal attention forward on B200 tensor cores.
+//
+// Computes, per head, O = softmax(scale * Q K^T with the upper triangle at
+// -inf) V and the natural-log row log-sum-exp ("How Andrej Karpathy built GPT
+// from 200 lines of code": section "Implementing the attention heads (Query,
+// Key, Value)" [1:06:16]-[1:17:18] for the scaled query-key affinities and
+// the value aggregation; section "Self-Attention: the mathematical trick"
+// [55:20] for the -inf upper triangle and the softmax).
+//
+// One CTA per (128-row query tile, head); heaviest tiles (most key tiles
+// under the causal mask) are launched first.  Six warps:
+//   warp 0      TMA producer: Q once, then K_j / V_j tiles into a 3-stage ring
+//   warp 1      tcgen05 issuer: S_j = Q K_j^T into TMEM (double buffered),
+//               O += P_j V_j with P_j read from TMEM; owns the TMEM allocation
+//   warps 2..5  softmax: one query row per thread (TMEM lane), online max and
+//               sum in registers, P_j written back to TMEM as bf16 over S_j,
+//               lazy rescale of the O accumulator, final O / l and lse.
+// Key tiles wholly above the diagonal are never loaded; only the diagonal
+// tile applies the element mask.  The score matrix never leaves the SM.
+//
+// TMEM columns: S_0 [0,128), S_1 [128,256), O [256, 256+D).
+#include "internal.h"
+#include "sm100.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace attn {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;          // query rows per CTA (= TMEM lanes)
+constexpr int kBN = 128;          // key rows per tile
+constexpr int kStages = 3;        // K/V ring depth
+constexpr int kThreads = 192;     // 6 warps
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
+
+template <int D>
+struct FwdSmem {
+    static constexpr int kTileBytes = kBN * D * 2;
+    alignas(1024) __nv_bfloat16 q[kBM * D];
+    alignas(1024) __nv_bfloat16 k[kStages][kBN * D];
+    alignas(1024) __nv_bfloat16 v[kStages][kBN * D];
+    uint64_t q_full;
+    uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
+    uint64_t s_full[2], p_full[2];
+    uint64_t o_done, o_final, drain;
+    uint32_t tmem_slot;
+    int abort;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+               const __grid_constant__ CUtensorMap tv, __nv_bfloat16 *__restrict__ o,
+               float *__restrict__ lse, int T, int BH, int ntiles, float scale_log2, int *err) {
+    using Smem = FwdSmem<D>;
+    constexpr int kRowBytes = D * 2;                      // 128 (D=64) or 64 (D=32)
+    constexpr uint32_t kSwz = (D == 64) ? kSwizzle128B : kSwizzle64B;
+    constexpr uint32_t kAtom = 8 * kRowBytes;             // 8-row swizzle atom
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~uintptr_t(1023));
+    volatile int *abort = &sm.abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qt = ntiles - 1 - (int)(blockIdx.x / BH);  // heaviest first
+    const int bh = (int)(blockIdx.x % BH);
+    const int n_kv = qt + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.v_full[s], 1);
+            mbar_init(&sm.k_empty[s], 1);
+            mbar_init(&sm.v_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.p_full[b], kBM);
+        }
+        mbar_init(&sm.o_done, 1);
+        mbar_init(&sm.o_final, 1);
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_slot;
+    const uint32_t tS[2] = {tmem, tmem + 128};
+    const uint32_t tO = tmem + 256;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tq);
+            prefetch_tensormap(&tk);
+            prefetch_tensormap(&tv);
+            mbar_arrive_expect_tx(&sm.q_full, Smem::kTileBytes);
+            tma_load_3d(sm.q, &tq, &sm.q_full, 0, qt * kBM, bh);
+            int issued = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j % kStages;
+                const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+                if (!mbar_wait(&sm.k_empty[s], ph ^ 1u, err, abort)) break;
+                mbar_arrive_expect_tx(&sm.k_full[s], Smem::kTileBytes);
+                tma_load_3d(sm.k[s], &tk, &sm.k_full[s], 0, j * kBN, bh);
+                if (!mbar_wait(&sm.v_empty[s], ph ^ 1u, err, abort)) {
+                    issued = j + 1;  // K_j is in flight
+                    mbar_wait(&sm.k_full[s], ph, err, abort);
+                    break;
+                }
+                mbar_arrive_expect_tx(&sm.v_full[s], Smem::kTileBytes);
+                tma_load_3d(sm.v[s], &tv, &sm.v_full[s], 0, j * kBN, bh);
+                issued = j + 1;
+            }
+            // Drain: every load this thread issued has landed before exit.
+            for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
+                const int s = j % kStages;
+                const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
+                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.v_full[s], ph); ++i) {}
+            }
+            mbar_wait(&sm.q_full, 0, err, abort);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);  // Q, K both K-major
+            constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);    // P from TMEM, V MN-major
+            const uint32_t q_addr = smem_u32(sm.q);
+            bool ok = mbar_wait(&sm.q_full, 0, err, abort);
+            for (int j = 0; ok && j <= n_kv; ++j) {
+                if (j < n_kv) {
+                    const int s = j % kStages;
+                    if (!(ok = mbar_wait(&sm.k_full[s], (uint32_t)(j / kStages) & 1u, err, abort))) break;
+                    if (j >= 2 && !(ok = mbar_wait(&sm.o_done, (uint32_t)(j - 2) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(sm.k[s]);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tS[j & 1], smem_desc(q_addr + kk * 32, 16, kAtom, kSwz),
+                               smem_desc(k_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
+                    mma_commit(&sm.s_full[j & 1]);
+                    mma_commit(&sm.k_empty[s]);
+                }
+                if (j >= 1) {
+                    const int jj = j - 1;
+                    const int s = jj % kStages;
+                    if (!(ok = mbar_wait(&sm.p_full[jj & 1], (uint32_t)(jj >> 1) & 1u, err, abort))) break;
+                    if (!(ok = mbar_wait(&sm.v_full[s], (uint32_t)(jj / kStages) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(sm.v[s]);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_ts(tO, tS[jj & 1] + kk * 8,
+                               smem_desc(v_addr + kk * 16 * kRowBytes, kBN * kRowBytes, kAtom, kSwz),
+                               idO, (jj > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&sm.o_done);
+                    mma_commit(&sm.v_empty[s]);
+                }
+            }
+            // All MMAs this thread issued are complete once `drain` fires.
+            mma_commit(&sm.o_final);
+            mma_commit(&sm.drain);
+            mbar_wait(&sm.drain, 0, err, abort);
+        }
+    } else {
+        // ------------------------------------------------ softmax warps
+        const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
+        const int row = quad * 32 + lane;          // row within the query tile
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const int b = j & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (uint32_t)(j >> 1) & 1u, err, abort));
+            if (!ok) break;
+            tc_fence_after();
+            float s[kBN];
+#pragma unroll
+            for (int c = 0; c < kBN; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tS[b] + lane_off + c, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) s[c + x] = __uint_as_float(r[x]);
+            }
+            if (j == n_kv - 1) {  // diagonal tile: key column c is visible to row r iff c <= r
+#pragma unroll
+                for (int c = 0; c < kBN; ++c)
+                    if (c > row) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+            const float mxs = mx * scale_log2;
+            // Each row moves its own running max only when its scores exceed
+            // it by more than the threshold; the warp merely decides whether
+            // the TMEM round trip of O is needed (rows that keep their max
+            // scale by exactly 1).  A row's arithmetic thus depends on its own
+            // scores alone.
+            const bool need = mxs > m_used + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, need)) {
+                const float m_new = need ? mxs : m_used;
+                const float alpha = ex2(m_used - m_new);
+                if (j > 0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done, (uint32_t)(j - 1) & 1u, err, abort));
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < D; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(tO + lane_off + c, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+                        tmem_st32(tO + lane_off + c, r);
+                    }
+                }
+                l *= alpha;
+                m_used = m_new;
+            }
+            const float neg_m = -m_used;
+#pragma unroll
+            for (int c = 0; c < kBN; c += 64) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    const float p0 = ex2(fmaf(s[c + 2 * x], scale_log2, neg_m));
+                    const float p1 = ex2(fmaf(s[c + 2 * x + 1], scale_log2, neg_m));
+                    l += p0 + p1;
+                    pk[x] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tS[b] + lane_off + c / 2, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.p_full[b]);
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, 0, err, abort));
+        if (ok) {
+            tc_fence_after();
+            const int t = qt * kBM + row;
+            const float inv = 1.f / l;
+            const size_t grow = (size_t)bh * T + t;
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tO + lane_off + c, r);
+                tmem_wait_ld();
+                if (t < T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(o + grow * D + c);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * inv, __uint_as_float(r[8 * x + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv, __uint_as_float(r[8 * x + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv, __uint_as_float(r[8 * x + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv, __uint_as_float(r[8 * x + 7]) * inv);
+                        dst[x] = w;
+                    }
+                }
+            }
+            if (t < T) lse[grow] = (m_used + log2f(l)) * 0.69314718055994531f;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Encodes a [BH, T, D] bf16 tensor as a 3-D TMA map with 128-row boxes.
+cudaError_t make_map(CUtensorMap *map, const void *ptr, int BH, int T, int D) {
+    auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+    if (!enc) return cudaErrorInitializationError;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)D, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                       __nv_bfloat16 *o, float *lse, Shape s, int *err, cudaStream_t st,
+                       LaunchInfo &li) {
+    const int BH = s.B * s.H;
+    const int ntiles = (s.T + kBM - 1) / kBM;
+    const long long blocks = (long long)ntiles * BH;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    CUtensorMap mq, mk, mv;
+    cudaError_t e;
+    if ((e = make_map(&mq, q, BH, s.T, D)) != cudaSuccess) return e;
+    if ((e = make_map(&mk, k, BH, s.T, D)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, v, BH, s.T, D)) != cudaSuccess) return e;
+    const size_t smem = sizeof(FwdSmem<D>) + 1024;
+    if ((e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+        return e;
+    const float scale_log2 = s.scale * 1.4426950408889634f;
+    if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
+    fwd_kernel<D><<<(unsigned)blocks, kThreads, smem, st>>>(mq, mk, mv, o, lse, s.T, BH, ntiles,
+                                                            scale_log2, err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    li.kernels += 1;
+    return mark_main_end(li, st);
+}
+
+}  // namespace
+
+cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                      __nv_bfloat16 *o, float *lse, Shape s, int *err, cudaStream_t st,
+                      LaunchInfo &li) {
+    if (s.D == 64) return launch_fwd<64>(q, k, v, o, lse, s, err, st, li);
+    if (s.D == 32) return launch_fwd<32>(q, k, v, o, lse, s, err, st, li);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace attn

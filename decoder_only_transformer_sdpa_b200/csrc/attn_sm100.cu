@@ -1,15 +1,8 @@
-// attn_sm100.cu -- bf16 entry of the kernels (provisional: CUDA-core kernels
-// while the tensor-core kernels are brought up).
+// attn_sm100.cu -- bf16 backward entry (provisional: CUDA-core kernels while
+// the tensor-core backward is brought up).
 #include "internal.h"
 
 namespace attn {
-
-cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                      __nv_bfloat16 *o, float *lse, Shape s, int *err, cudaStream_t st,
-                      LaunchInfo &li) {
-    (void)err;
-    return simt_fwd<__nv_bfloat16>(q, k, v, o, lse, s, st, li);
-}
 
 cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,

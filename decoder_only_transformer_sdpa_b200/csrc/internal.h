@@ -11,9 +11,10 @@ namespace attn {
 
 // Upper bound on the polls of any in-kernel wait (mbarrier or flag).  A wait
 // that runs out sets the device error word to kErrTimeout and the kernel
-// leaves by its normal exit path.  At ~1 poll per 20-100 ns this bounds a
-// stuck wait to a fraction of a second up to a few seconds.
-constexpr uint32_t kWaitLimit = 1u << 25;
+// leaves by its normal exit path.  A poll costs from ~20 ns up to ~1 us
+// (try_wait may suspend the thread briefly), so a stuck wait ends after
+// roughly 0.1 s to a few seconds; legitimate waits last microseconds.
+constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr int kErrTimeout = 1;
 
 struct Shape {
@@ -55,6 +56,10 @@ cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv,
                       float *dq_acc, float *delta, Shape s, int *err, cudaStream_t st,
                       LaunchInfo &li);
+
+// Launches one thread that waits on an mbarrier nobody arrives at, polling at
+// most `polls` times, so the timeout path can be exercised without a fault.
+cudaError_t selftest_wait_timeout(uint32_t polls, int *err, cudaStream_t st);
 
 // Driver entry point for cuTensorMapEncodeTiled, resolved once at run time
 // through the runtime (so the library does not link libcuda directly).

@@ -112,6 +112,13 @@ int attn_bwd_f32(const float *q, const float *k, const float *v, const float *o,
  * ran out since the last call) or ATTN_ERR_CUDA (the sync itself failed). */
 int attn_device_error(cudaStream_t stream);
 
+/* Failure-path self test: enqueues one thread that waits on an in-kernel
+ * barrier nothing ever completes, gives up after `polls` polls (1 .. 2^22)
+ * and sets the error flag, as any timed-out wait in the attention kernels
+ * does.  A following attn_device_error() then returns ATTN_ERR_TIMEOUT.
+ * Faults nothing and never hangs. */
+int attn_selftest_wait_timeout(uint32_t polls, cudaStream_t stream);
+
 /* Number of kernels the most recent successful call on this host thread
  * enqueued (for launch accounting). */
 int attn_last_launch_count(void);

@@ -113,3 +113,8 @@ def test_fwd_f32_argument_errors(kw, expect):
 def test_bwd_f32_workspace_error():
     lib = lib_mod.lib()
     assert lib.attn_bwd_f32(*([P] * 9), 1, 1, 8, 8, 0.3, P, 8, None) == E_WS
+
+
+def test_selftest_argument_errors():
+    assert lib_mod.lib().attn_selftest_wait_timeout(0, None) == E_SHAPE
+    assert lib_mod.lib().attn_selftest_wait_timeout((1 << 22) + 1, None) == E_SHAPE
