@@ -142,11 +142,10 @@ ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, floa
     return finish(e, li);
 }
 
-// Workspace of the bf16 backward: dQ float32 accumulator, then Delta.
+// Workspace of the bf16 backward: dQ float32 accumulator, padded lse, Delta.
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
     if (check_shape(B, H, T, D, 64) != ATTN_OK || !bf16_d_supported(D)) return 0;
-    const size_t rows = (size_t)B * H * T;
-    return round_up(rows * D * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+    return bwd_workspace_layout(B, H, T, D).total;
 }
 
 ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -166,15 +165,16 @@ ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
     int *err = nullptr;
     if ((st = device_setup(&err)) != ATTN_OK) return st;
-    const size_t rows = (size_t)B * H * T;
-    float *dq_acc = static_cast<float *>(workspace);
-    float *delta = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                             round_up(rows * D * sizeof(float), 256));
+    const BwdWorkspace wl = bwd_workspace_layout(B, H, T, D);
+    char *ws = static_cast<char *>(workspace);
+    float *dq_acc = reinterpret_cast<float *>(ws + wl.dq_acc);
+    float *lse2 = reinterpret_cast<float *>(ws + wl.lse2);
+    float *delta = reinterpret_cast<float *>(ws + wl.delta);
     cudaError_t e = sm100_bwd(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(o), lse,
         static_cast<const __nv_bfloat16 *>(dO), static_cast<__nv_bfloat16 *>(dq),
-        static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv), dq_acc, delta,
+        static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv), dq_acc, lse2, delta,
         Shape{B, H, T, D, scale}, err, stream, li);
     return finish(e, li);
 }

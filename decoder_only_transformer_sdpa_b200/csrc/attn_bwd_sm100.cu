@@ -1,0 +1,503 @@
+// attn_bwd_sm100.cu -- causal attention backward on B200 tensor cores.
+//
+// The pages define the forward only ("How Andrej Karpathy built GPT from 200
+// lines of code", sections "Self-Attention: the mathematical trick" [55:20]
+// and "Implementing the attention heads (Query, Key, Value)" [1:06:16]-
+// [1:17:18]); the backward is its exact derivative for L = sum(O * dO):
+//
+//   P_ij  = exp(scale q_i.k_j - lse_i)          (recomputed from the saved lse)
+//   dV_j  = sum_{i>=j} P_ij dO_i
+//   dP_ij = dO_i . v_j,   Delta_i = dO_i . O_i
+//   dS_ij = P_ij (dP_ij - Delta_i)
+//   dK_j  = scale sum_{i>=j} dS_ij q_i,   dQ_i = scale sum_{j<=i} dS_ij k_j
+//
+// Three launches on the caller's stream:
+//   prep   Delta_i and lse_i * log2(e) into tile-padded float32 arrays (pad rows
+//          get Delta = 0 and lse = +inf, so they contribute exactly 0), and the
+//          float32 dQ accumulator zeroed;
+//   main   one CTA per (128-row key tile j, head), looping over the query
+//          tiles i >= j; dK_j and dV_j accumulate in TMEM, the partial
+//          dQ_i = dS_ij K_j is added into the float32 accumulator by TMA
+//          reduce-add;
+//   post   dQ = scale * accumulator, rounded to bf16.
+//
+// Main kernel, ten warps:
+//   warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, Delta_i per tile
+//               into a 2-stage ring
+//   warp 1      tcgen05 issuer, TMEM owner
+//   warps 2..5  softmax gradient: one key row per thread (TMEM lane) over the
+//               128 query columns: P^T = exp2(S^T - lse), dS^T = P^T (dP^T -
+//               Delta); P^T to TMEM (bf16), dS^T to shared memory (bf16,
+//               double buffered); final dK, dV epilogue
+//   warps 6..9  dQ drain: TMEM -> swizzled shared staging -> TMA reduce-add
+//
+// Per query tile the issuer runs S^T = K Q^T and dP^T = V dO^T (M = key rows),
+// then, once the softmax gradient of that tile is ready, dV += P^T dO (A from
+// TMEM), dK += dS^T Q and dQ_i = dS K (A read MN-major from the same shared
+// dS^T tile).  The next tile's S^T / dP^T are issued as soon as the current
+// ones have been read out of TMEM, so they overlap the elementwise work.
+//
+// TMEM columns: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D),
+// dQ [256+2D, 256+3D), P^T (bf16 pairs) [256+3D, 256+3D+64).
+#include "internal.h"
+#include "sm100.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace attn {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBT = 128;          // rows per tile (keys and queries)
+constexpr int kThreads = 320;     // 10 warps
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdSmem {
+    static constexpr int kTileBytes = kBT * D * 2;
+    alignas(1024) __nv_bfloat16 q[2][kBT * D];
+    alignas(1024) __nv_bfloat16 dO[2][kBT * D];
+    alignas(1024) __nv_bfloat16 k[kBT * D];
+    alignas(1024) __nv_bfloat16 v[kBT * D];
+    // dS^T, [buffer][query half][key row][64 queries], 128-byte swizzled rows
+    alignas(1024) __nv_bfloat16 ds[2][2][kBT * 64];
+    // dQ staging for the TMA reduce: [32-column box][row][32 floats], swizzled
+    alignas(1024) float stage[D / 32][kBT * 32];
+    alignas(16) float lse2[2][kBT];
+    alignas(16) float delta[2][kBT];
+    uint64_t kv_full, qdo_full[2], qdo_empty[2];
+    uint64_t sdp_full, sdp_free, p_ready[2], ds_ready[2], p_free, ds_free[2];
+    uint64_t dq_full, dq_free, acc_done, drain;
+    uint32_t tmem_slot;
+    int abort;
+};
+
+// ------------------------------------------------------------------ prep
+
+template <int D>
+__global__ void __launch_bounds__(128) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
+                                                       const __nv_bfloat16 *__restrict__ dO,
+                                                       const float *__restrict__ lse,
+                                                       float *__restrict__ lse2,
+                                                       float *__restrict__ delta,
+                                                       float *__restrict__ dq_acc, int T, int Tpad) {
+    const int nt = Tpad / 128;
+    const long long bh = blockIdx.x / nt;
+    const int t = (int)(blockIdx.x - bh * nt) * 128 + threadIdx.x;
+    if (t >= Tpad) return;
+    const size_t prow = (size_t)bh * Tpad + t;
+    if (t < T) {
+        const size_t row = (size_t)bh * T + t;
+        const uint4 *po = reinterpret_cast<const uint4 *>(o + row * D);
+        const uint4 *pg = reinterpret_cast<const uint4 *>(dO + row * D);
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 a = po[c], b = pg[c];
+            const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
+            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&b);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float2 fa = __bfloat1622float2(a2[x]), fb = __bfloat1622float2(b2[x]);
+                acc = fmaf(fa.x, fb.x, acc);
+                acc = fmaf(fa.y, fb.y, acc);
+            }
+        }
+        delta[prow] = acc;
+        lse2[prow] = lse[row] * kLog2e;
+        float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+        delta[prow] = 0.f;
+        lse2[prow] = INFINITY;
+    }
+}
+
+// ------------------------------------------------------------------ post
+
+__global__ void bwd_post_kernel(const float4 *__restrict__ acc, uint2 *__restrict__ dq, long long n4,
+                                float scale) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        const float4 a = acc[i];
+        uint2 r;
+        r.x = pack_bf16x2(a.x * scale, a.y * scale);
+        r.y = pack_bf16x2(a.z * scale, a.w * scale);
+        dq[i] = r;
+    }
+}
+
+// ------------------------------------------------------------------ main
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                    const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                    const __grid_constant__ CUtensorMap tdq, const float *__restrict__ lse2,
+                    const float *__restrict__ delta, __nv_bfloat16 *__restrict__ dk,
+                    __nv_bfloat16 *__restrict__ dv, int T, int Tpad, int BH, int nt,
+                    float scale_log2, float scale, int *err) {
+    using Smem = BwdSmem<D>;
+    constexpr int kRowBytes = D * 2;
+    constexpr uint32_t kSwz = (D == 64) ? kSwizzle128B : kSwizzle64B;
+    constexpr uint32_t kAtom = 8 * kRowBytes;
+    constexpr uint32_t kHalf = kBT * 64 * 2;  // bytes of one 64-query half of dS^T
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~uintptr_t(1023));
+    volatile int *abort = &sm.abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kt = (int)(blockIdx.x / BH);  // key tile; tile 0 sees the most query tiles
+    const int bh = (int)(blockIdx.x % BH);
+    const int n_q = nt - kt;                // query tiles kt .. nt-1
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.qdo_full[s], 1);
+            mbar_init(&sm.qdo_empty[s], 1);
+            mbar_init(&sm.p_ready[s], kBT);
+            mbar_init(&sm.ds_ready[s], kBT);
+            mbar_init(&sm.ds_free[s], 1);
+        }
+        mbar_init(&sm.sdp_full, 1);
+        mbar_init(&sm.sdp_free, kBT);
+        mbar_init(&sm.p_free, 1);
+        mbar_init(&sm.dq_full, 1);
+        mbar_init(&sm.dq_free, kBT);
+        mbar_init(&sm.acc_done, 1);
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_slot;
+    const uint32_t tS = tmem, tdP = tmem + 128;
+    const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D, tdQ = tmem + 256 + 2 * D;
+    const uint32_t tP = tmem + 256 + 3 * D;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tq);
+            prefetch_tensormap(&tk);
+            prefetch_tensormap(&tv);
+            prefetch_tensormap(&tdo);
+            mbar_arrive_expect_tx(&sm.kv_full, 2 * Smem::kTileBytes);
+            tma_load_3d(sm.k, &tk, &sm.kv_full, 0, kt * kBT, bh);
+            tma_load_3d(sm.v, &tv, &sm.kv_full, 0, kt * kBT, bh);
+            int issued = 0;
+            for (int idx = 0; idx < n_q; ++idx) {
+                const int st = idx & 1;
+                const int i = kt + idx;
+                if (!mbar_wait(&sm.qdo_empty[st], (uint32_t)((idx >> 1) & 1) ^ 1u, err, abort)) break;
+                mbar_arrive_expect_tx(&sm.qdo_full[st], 2 * Smem::kTileBytes + 2 * kBT * 4);
+                tma_load_3d(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, bh);
+                tma_load_3d(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, bh);
+                const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
+                bulk_load(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
+                bulk_load(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
+                issued = idx + 1;
+            }
+            for (int idx = (issued > 2 ? issued - 2 : 0); idx < issued; ++idx)
+                for (uint32_t n = 0; n < kWaitLimit && !mbar_try_wait(&sm.qdo_full[idx & 1], (uint32_t)(idx >> 1) & 1u); ++n) {}
+            mbar_wait(&sm.kv_full, 0, err, abort);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(kBT, kBT, 0, 0);  // S^T, dP^T: both K-major
+            constexpr uint32_t idKV = idesc_bf16(kBT, D, 0, 1);   // dV, dK: A K-major/TMEM, B MN-major
+            constexpr uint32_t idQ = idesc_bf16(kBT, D, 1, 1);    // dQ: A (dS) and B (K) MN-major
+            const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+            bool ok = mbar_wait(&sm.kv_full, 0, err, abort);
+            for (int idx = 0; ok && idx <= n_q; ++idx) {
+                if (idx < n_q) {
+                    const int st = idx & 1;
+                    if (!(ok = mbar_wait(&sm.qdo_full[st], (uint32_t)(idx >> 1) & 1u, err, abort))) break;
+                    if (idx >= 1 && !(ok = mbar_wait(&sm.sdp_free, (uint32_t)(idx - 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    const uint32_t q_addr = smem_u32(sm.q[st]), do_addr = smem_u32(sm.dO[st]);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tS, smem_desc(k_addr + kk * 32, 16, kAtom, kSwz),
+                               smem_desc(q_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tdP, smem_desc(v_addr + kk * 32, 16, kAtom, kSwz),
+                               smem_desc(do_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
+                    mma_commit(&sm.sdp_full);
+                }
+                if (idx >= 1) {
+                    const int p = idx - 1;  // the tile whose gradients are now issued
+                    const int st = p & 1, b = p & 1;
+                    const uint32_t q_addr = smem_u32(sm.q[st]), do_addr = smem_u32(sm.dO[st]);
+                    const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
+                    if (!(ok = mbar_wait(&sm.p_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int s = 0; s < kBT / 16; ++s)  // dV += P^T dO, K = 16 queries per step
+                        mma_ts(tdV, tP + s * 8,
+                               smem_desc(do_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
+                               idKV, (p > 0 || s > 0) ? 1u : 0u);
+                    mma_commit(&sm.p_free);
+                    if (!(ok = mbar_wait(&sm.ds_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int s = 0; s < kBT / 16; ++s)  // dK += dS^T Q
+                        mma_ss(tdK,
+                               smem_desc(ds_addr + (s >> 2) * kHalf + (s & 3) * 32, 16, 1024, kSwizzle128B),
+                               smem_desc(q_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
+                               idKV, (p > 0 || s > 0) ? 1u : 0u);
+                    if (p >= 1 && !(ok = mbar_wait(&sm.dq_free, (uint32_t)(p - 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int s = 0; s < kBT / 16; ++s)  // dQ_i = dS K, K = 16 keys per step
+                        mma_ss(tdQ, smem_desc(ds_addr + s * 16 * 128, kHalf, 1024, kSwizzle128B),
+                               smem_desc(k_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
+                               idQ, s > 0 ? 1u : 0u);
+                    mma_commit(&sm.dq_full);
+                    mma_commit(&sm.qdo_empty[st]);
+                    mma_commit(&sm.ds_free[b]);
+                }
+            }
+            mma_commit(&sm.acc_done);
+            mma_commit(&sm.drain);
+            mbar_wait(&sm.drain, 0, err, abort);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ softmax gradient
+        const int quad = warp & 3;
+        const int kr = quad * 32 + lane;                // key row within the tile (TMEM lane)
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t sw = (uint32_t)(kr & 7);
+        bool ok = true;
+        for (int idx = 0; idx < n_q; ++idx) {
+            const int st = idx & 1, b = idx & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.sdp_full, (uint32_t)idx & 1u, err, abort));
+            if (!ok) break;
+            tc_fence_after();
+            const bool diag = (idx == 0);
+            const uint32_t lse_addr = smem_u32(sm.lse2[st]), dl_addr = smem_u32(sm.delta[st]);
+            const uint32_t ds_row = smem_u32(sm.ds[b][0]) + (uint32_t)kr * 128;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {  // 32 query columns per chunk
+                uint32_t rs[32], rp[32];
+                tmem_ld32(tS + lane_off + 32 * c, rs);
+                tmem_ld32(tdP + lane_off + 32 * c, rp);
+                tmem_wait_ld();
+                reg_fence32(rs);
+                reg_fence32(rp);
+                if (c == 3) {  // S^T and dP^T fully read: the next tile may overwrite them
+                    tc_fence_before();
+                    mbar_arrive(&sm.sdp_free);
+                }
+                uint32_t pw[16], dw[16];
+#pragma unroll
+                for (int x = 0; x < 32; x += 4) {
+                    const float4 l4 = ld_shared_f4(lse_addr + (32 * c + x) * 4);
+                    const float4 d4 = ld_shared_f4(dl_addr + (32 * c + x) * 4);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pp[4], dd[4];
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        float pv = ex2(fmaf(__uint_as_float(rs[x + y]), scale_log2, -lv[y]));
+                        if (diag && (32 * c + x + y) < kr) pv = 0.f;  // query before key: masked
+                        pp[y] = pv;
+                        dd[y] = pv * (__uint_as_float(rp[x + y]) - dvv[y]);
+                    }
+                    pw[x / 2] = pack_bf16x2(pp[0], pp[1]);
+                    pw[x / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
+                    dw[x / 2] = pack_bf16x2(dd[0], dd[1]);
+                    dw[x / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
+                }
+                if (c == 0) {
+                    // P^T in TMEM is free once dV of the previous tile completed;
+                    // this dS^T buffer once dK/dQ of two tiles ago completed.
+                    bool w = true;
+                    if (idx >= 1) w = mbar_wait(&sm.p_free, (uint32_t)(idx - 1) & 1u, err, abort);
+                    w = w && mbar_wait(&sm.ds_free[b], (uint32_t)((idx >> 1) & 1) ^ 1u, err, abort);
+                    ok = __all_sync(0xffffffffu, w);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                tmem_st16(tP + lane_off + 16 * c, pw);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {  // four 16-byte chunks = 32 queries
+                    const uint32_t g = 4 * c + u;          // 8-query group 0..15
+                    const uint32_t addr = ds_row + (g >> 3) * kHalf + (((g & 7) ^ sw) << 4);
+                    st_shared_v4(addr, dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
+                }
+            }
+            if (!ok) break;
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&sm.p_ready[b]);
+            mbar_arrive(&sm.ds_ready[b]);
+        }
+        // ---- epilogue: dK (times scale) and dV of this key tile
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_done, 0, err, abort));
+        if (ok) {
+            tc_fence_after();
+            const int t = kt * kBT + kr;
+            const size_t grow = (size_t)bh * T + t;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t src = which == 0 ? tdK : tdV;
+                const float mul = which == 0 ? scale : 1.f;
+                __nv_bfloat16 *out = which == 0 ? dk : dv;
+#pragma unroll
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(src + lane_off + c, r);
+                    tmem_wait_ld();
+                    reg_fence32(r);
+                    if (t < T) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(out + grow * D + c);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            uint4 w4;
+                            w4.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * mul, __uint_as_float(r[8 * x + 1]) * mul);
+                            w4.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * mul, __uint_as_float(r[8 * x + 3]) * mul);
+                            w4.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * mul, __uint_as_float(r[8 * x + 5]) * mul);
+                            w4.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * mul, __uint_as_float(r[8 * x + 7]) * mul);
+                            dst[x] = w4;
+                        }
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ dQ drain
+        const int quad = warp & 3;
+        const int qr = quad * 32 + lane;                // query row within the tile
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const bool leader = (warp == 6 && lane == 0);
+        const uint32_t sw = (uint32_t)(qr & 7);
+        for (int idx = 0; idx < n_q; ++idx) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, (uint32_t)idx & 1u, err, abort));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t r[D / 32][32];
+#pragma unroll
+            for (int h = 0; h < D / 32; ++h) tmem_ld32(tdQ + lane_off + 32 * h, r[h]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < D / 32; ++h) reg_fence32(r[h]);
+            tc_fence_before();
+            mbar_arrive(&sm.dq_free);
+            if (leader) bulk_wait_read_all();   // previous reduce has read the staging
+            named_bar_sync(1, 128);
+#pragma unroll
+            for (int h = 0; h < D / 32; ++h) {
+                const uint32_t row = smem_u32(sm.stage[h]) + (uint32_t)qr * 128;
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    st_shared_v4(row + ((u ^ sw) << 4), r[h][4 * u], r[h][4 * u + 1], r[h][4 * u + 2],
+                                 r[h][4 * u + 3]);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (leader) {
+#pragma unroll
+                for (int h = 0; h < D / 32; ++h)
+                    tma_reduce_add_3d(&tdq, sm.stage[h], 32 * h, (kt + idx) * kBT, bh);
+                bulk_commit();
+            }
+        }
+        if (leader) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Encodes a [BH, T, D] tensor (bf16 or float32) as a 3-D TMA map.
+cudaError_t make_map(CUtensorMap *map, const void *ptr, int BH, int T, int D, bool f32, int box_x) {
+    auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+    if (!enc) return cudaErrorInitializationError;
+    const int es = f32 ? 4 : 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)T * D * es};
+    const cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)kBT, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle swz = (box_x * es == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                           const_cast<void *>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                       const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
+                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
+                       float *lse2, float *delta, Shape s, int *err, cudaStream_t st,
+                       LaunchInfo &li) {
+    const int BH = s.B * s.H;
+    const int nt = (s.T + kBT - 1) / kBT;
+    const int Tpad = nt * kBT;
+    const long long blocks = (long long)nt * BH;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    CUtensorMap mq, mk, mv, mdo, mdq;
+    cudaError_t e;
+    if ((e = make_map(&mq, q, BH, s.T, D, false, D)) != cudaSuccess) return e;
+    if ((e = make_map(&mk, k, BH, s.T, D, false, D)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, v, BH, s.T, D, false, D)) != cudaSuccess) return e;
+    if ((e = make_map(&mdo, dO, BH, s.T, D, false, D)) != cudaSuccess) return e;
+    if ((e = make_map(&mdq, dq_acc, BH, s.T, D, true, 32)) != cudaSuccess) return e;
+
+    bwd_prep_kernel<D><<<(unsigned)blocks, 128, 0, st>>>(o, dO, lse, lse2, delta, dq_acc, s.T, Tpad);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    li.kernels += 1;
+
+    const size_t smem = sizeof(BwdSmem<D>) + 1024;
+    if ((e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+        return e;
+    if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
+    bwd_main_kernel<D><<<(unsigned)blocks, kThreads, smem, st>>>(
+        mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, s.T, Tpad, BH, nt, s.scale * kLog2e, s.scale, err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    li.kernels += 1;
+    if ((e = mark_main_end(li, st)) != cudaSuccess) return e;
+
+    const long long n4 = (long long)BH * s.T * D / 4;
+    const int post_blocks = (int)((n4 + 255) / 256 < 148 * 16 ? (n4 + 255) / 256 : 148 * 16);
+    bwd_post_kernel<<<post_blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc),
+                                                  reinterpret_cast<uint2 *>(dq), n4, s.scale);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    li.kernels += 1;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                      const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
+                      __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
+                      float *lse2, float *delta, Shape s, int *err, cudaStream_t st,
+                      LaunchInfo &li) {
+    if (s.D == 64)
+        return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, err, st, li);
+    if (s.D == 32)
+        return launch_bwd<32>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, err, st, li);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace attn

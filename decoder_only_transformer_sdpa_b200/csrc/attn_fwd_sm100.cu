@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t r[32];
                 tmem_ld32(tS[b] + lane_off + c, r);
                 tmem_wait_ld();
+                reg_fence32(r);
 #pragma unroll
                 for (int x = 0; x < 32; ++x) s[c + x] = __uint_as_float(r[x]);
             }
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint32_t r[32];
                         tmem_ld32(tO + lane_off + c, r);
                         tmem_wait_ld();
+                        reg_fence32(r);
 #pragma unroll
                         for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
                         tmem_st32(tO + lane_off + c, r);
@@ -254,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t r[32];
                 tmem_ld32(tO + lane_off + c, r);
                 tmem_wait_ld();
+                reg_fence32(r);
                 if (t < T) {
                     uint4 *dst = reinterpret_cast<uint4 *>(o + grow * D + c);
 #pragma unroll

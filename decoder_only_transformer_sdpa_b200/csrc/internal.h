@@ -54,8 +54,26 @@ cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
 cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv,
-                      float *dq_acc, float *delta, Shape s, int *err, cudaStream_t st,
+                      float *dq_acc, float *lse2, float *delta, Shape s, int *err, cudaStream_t st,
                       LaunchInfo &li);
+
+// Workspace layout of the bf16 backward (offsets in bytes, each 256-aligned):
+// float32 dQ accumulator [B*H*T*D], then log2-scaled lse and Delta, each
+// [B*H][T padded to a multiple of 128].
+struct BwdWorkspace {
+    size_t dq_acc, lse2, delta, total;
+};
+inline BwdWorkspace bwd_workspace_layout(int B, int H, int T, int D) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t rows = (size_t)B * H * T;
+    const size_t prows = (size_t)B * H * (size_t)((T + 127) / 128 * 128);
+    BwdWorkspace w;
+    w.dq_acc = 0;
+    w.lse2 = up(rows * D * sizeof(float));
+    w.delta = w.lse2 + up(prows * sizeof(float));
+    w.total = w.delta + up(prows * sizeof(float));
+    return w;
+}
 
 // Launches one thread that waits on an mbarrier nobody arrives at, polling at
 // most `polls` times, so the timeout path can be exercised without a fault.

@@ -52,8 +52,10 @@ def test_workspace_sizes():
     B, H, T, D = 12, 12, 1024, 64
     rows = B * H * T
     rnd = lambda x: (x + 255) // 256 * 256
-    assert lib_mod.attn_bwd_workspace_bytes(B, H, T, D) == rnd(rows * D * 4) + rnd(rows * 4)
-    assert lib_mod.attn_bwd_workspace_bytes(1, 1, 1, 32) == 256 + 256
+    tpad = lambda t: (t + 127) // 128 * 128
+    assert lib_mod.attn_bwd_workspace_bytes(B, H, T, D) == rnd(rows * D * 4) + 2 * rnd(B * H * tpad(T) * 4)
+    assert lib_mod.attn_bwd_workspace_bytes(1, 1, 1, 32) == 256 + 2 * 512
+    assert lib_mod.attn_bwd_workspace_bytes(2, 3, 129, 64) == rnd(2 * 3 * 129 * 64 * 4) + 2 * rnd(6 * 256 * 4)
     assert lib_mod.attn_bwd_workspace_bytes(1, 1, 1, 48) == 0       # unsupported D
     assert lib_mod.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0       # bad shape
     assert lib_mod.attn_bwd_f32_workspace_bytes(4, 4, 8, 8) == rnd(4 * 4 * 8 * 4)
