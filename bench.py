@@ -49,6 +49,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=5, help="steps of the host-buffer end-to-end leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--layers", type=int, default=None,
+                   help="layer instances per step (default: the workload's 12); fewer only for profiling")
     return p.parse_args()
 
 
@@ -258,7 +260,7 @@ def run_ours(args, w):
     import decoder_only_transformer_sdpa_b200 as A
     from workloads import make_inputs
 
-    L = w.layers
+    L = w.layers if args.layers is None else max(1, args.layers)
     peaks, peak_kind = load_peaks()
     # ---- inputs, outputs and workspaces of every layer, resident in HBM
     layers = []
