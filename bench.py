@@ -172,6 +172,21 @@ def measured_traffic(kernel: str):
     return ent.get("bytes_per_launch")
 
 
+def reduce_max(value: float, world: int, device) -> float:
+    """The maximum of a per-rank value over all ranks (identity at world 1)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, steps: int, ms_max: float) -> float:
+    """Aggregate throughput: the work of every rank over the slowest rank's time."""
+    return flops_per_rank_step * world * steps / (ms_max * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------ CPU oracle leg
 
 def oracle_sample(w, seed, n_heads):
@@ -328,12 +343,9 @@ def run_ours(args, w):
 
     fwd_ms = [a.elapsed_time(b) for e in ev for a, b in e[0]]
     bwd_ms = [a.elapsed_time(b) for e in ev for a, b in e[1]]
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = reduce_max(ms, world, dev)
     flops_step = w.flops() * L
-    value = flops_step * world * args.steps / (ms_max * 1e-3) / 1e12
+    value = whole_job_tflops(flops_step, world, args.steps, ms_max)
 
     # ---- roofline of the dominant kernel (the one with the larger total time)
     pairs = w.causal_pairs()
@@ -382,11 +394,8 @@ def run_ours(args, w):
             e2e_step()
         s1.record(stream)
         barrier()
-        te = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item())
-        e2e = {"value": flops_step * world * args.e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e_ms = reduce_max(s0.elapsed_time(s1), world, dev)
+        e2e = {"value": whole_job_tflops(flops_step, world, args.e2e_steps, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps}
 
