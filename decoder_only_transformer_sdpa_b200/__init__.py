@@ -38,6 +38,8 @@ _lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
 _lib.attn_bwd_workspace_bytes.restype = _sz
 _lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]
 _lib.attn_bwd.restype = _i
+_lib.attn_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+_lib.attn_bwd_noalloc.restype = _i
 _lib.attn_fwd_f32.argtypes = [_fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _vp]
 _lib.attn_fwd_f32.restype = _i
 _lib.attn_bwd_f32_workspace_bytes.argtypes = [_i, _i, _i, _i]
@@ -54,7 +56,7 @@ _lib.attn_profile_next_call.restype = _i
 EXPORTED = ("attn_status_string", "attn_version", "attn_last_launch_count", "attn_fwd",
             "attn_bwd_workspace_bytes", "attn_bwd", "attn_fwd_f32", "attn_bwd_f32_workspace_bytes",
             "attn_bwd_f32", "attn_device_error", "attn_profile_next_call",
-            "attn_selftest_wait_timeout")
+            "attn_selftest_wait_timeout", "attn_bwd_noalloc")
 
 
 class AttnError(RuntimeError):
@@ -171,6 +173,28 @@ def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[flo
     """bf16 backward: returns (dQ, dK, dV) bf16."""
     return _bwd(_lib.attn_bwd, _lib.attn_bwd_workspace_bytes, _torch().bfloat16, q, k, v, o, lse,
                 dO, dq, dk, dv, scale, workspace, stream)
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, dO, dq=None, dk=None, dv=None,
+                     scale: Optional[float] = None, stream=None):
+    """bf16 backward whose scratch is a fixed array inside the library (for
+    callers that cannot allocate device memory; see include/attn.h for the
+    size limit and the sharing rules).  Returns (dQ, dK, dV)."""
+    torch = _torch()
+    B, H, T, D = _shape4(q)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    bf = torch.bfloat16
+    ptrs = [_check(q, "q", bf), _check(k, "k", bf, q.shape), _check(v, "v", bf, q.shape),
+            _check(o, "o", bf, q.shape), _check(lse, "lse", torch.float32, (B, H, T)),
+            _check(dO, "dO", bf, q.shape), _check(dq, "dq", bf, q.shape),
+            _check(dk, "dk", bf, q.shape), _check(dv, "dv", bf, q.shape)]
+    with torch.cuda.device(q.device):
+        _raise(_lib.attn_bwd_noalloc(*ptrs, B, H, T, D, scale, _stream_handle(stream)),
+               "attn_bwd_noalloc")
+    return dq, dk, dv
 
 
 def attn_fwd_f32(q, k, v, o=None, lse=None, scale: Optional[float] = None, stream=None):

@@ -92,6 +92,29 @@ int attn_bwd(const void *q, const void *k, const void *v, const void *o, const f
              int B, int H, int T, int D, float scale,
              void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Backward without caller-supplied workspace (no counterpart in the pages:
+ * it exists for the library's users, not for the method).
+ *
+ * For callers that cannot allocate device memory: C hosts without a device
+ * allocator, plug-ins in a framework that owns all device memory through its
+ * own pool and forbids cudaMalloc, and latency-critical loops where a
+ * cudaMalloc (which may synchronise the device) is not acceptable.  Same
+ * arguments, result and errors as attn_bwd minus the workspace: the scratch
+ * comes from a fixed array of ATTN_NOALLOC_SCRATCH_BYTES built into the
+ * library, which every GPU that loads the library holds until exit.  The call
+ * allocates nothing.
+ *  - Shapes whose attn_bwd_workspace_bytes() exceeds the array (e.g. more than
+ *    about 16 M (B*H*T*D) elements at D=64) return ATTN_ERR_WORKSPACE.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls on a device share the array; calls that overlap on the GPU
+ *    (other streams or host threads on the same device) race and must be
+ *    serialised by the caller.  Each call clears what must start at zero. */
+#define ATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                     const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                     int B, int H, int T, int D, float scale, cudaStream_t stream);
+
 /* ---------------- float32 path: CUDA cores, IEEE expf -------------------- */
 
 /* Forward in float32 (all tensors float32).  1 <= D <= 128. */
