@@ -21,15 +21,17 @@
 //          reduce-add;
 //   post   dQ = scale * accumulator, rounded to bf16.
 //
-// Main kernel, ten warps:
+// Main kernel, fourteen warps:
 //   warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, Delta_i per tile
-//               into a 2-stage ring
+//               into a 3-stage ring (a stage is released after dK_i, since
+//               dQ_i reads neither Q nor dO)
 //   warp 1      tcgen05 issuer, TMEM owner
-//   warps 2..5  softmax gradient: one key row per thread (TMEM lane) over the
-//               128 query columns: P^T = exp2(S^T - lse), dS^T = P^T (dP^T -
-//               Delta); P^T to TMEM (bf16), dS^T to shared memory (bf16,
-//               double buffered); final dK, dV epilogue
-//   warps 6..9  dQ drain: TMEM -> swizzled shared staging -> TMA reduce-add
+//   warps 2..9  softmax gradient, two warps per TMEM lane quadrant (one per
+//               64-query half): per key row (TMEM lane) P^T = exp2(S^T - lse),
+//               dS^T = P^T (dP^T - Delta); P^T to TMEM (bf16), dS^T to shared
+//               memory (bf16, double buffered); final dK (first half) and dV
+//               (second half) epilogue
+//   warps 10..13 dQ drain: TMEM -> swizzled shared staging -> TMA reduce-add
 //
 // Per query tile the issuer runs S^T = K Q^T and dP^T = V dO^T (M = key rows),
 // then, once the softmax gradient of that tile is ready, dV += P^T dO (A from
@@ -50,24 +52,26 @@ namespace {
 using namespace sm100;
 
 constexpr int kBT = 128;          // rows per tile (keys and queries)
-constexpr int kThreads = 320;     // 10 warps
+constexpr int kThreads = 448;     // 14 warps
+constexpr int kEwThreads = 256;   // softmax-gradient threads (warps 2..9)
+constexpr int kQStages = 3;       // Q / dO / lse / Delta ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct BwdSmem {
     static constexpr int kTileBytes = kBT * D * 2;
-    alignas(1024) __nv_bfloat16 q[2][kBT * D];
-    alignas(1024) __nv_bfloat16 dO[2][kBT * D];
+    alignas(1024) __nv_bfloat16 q[kQStages][kBT * D];
+    alignas(1024) __nv_bfloat16 dO[kQStages][kBT * D];
     alignas(1024) __nv_bfloat16 k[kBT * D];
     alignas(1024) __nv_bfloat16 v[kBT * D];
     // dS^T, [buffer][query half][key row][64 queries], 128-byte swizzled rows
     alignas(1024) __nv_bfloat16 ds[2][2][kBT * 64];
-    // dQ staging for the TMA reduce: [32-column box][row][32 floats], swizzled
-    alignas(1024) float stage[D / 32][kBT * 32];
-    alignas(16) float lse2[2][kBT];
-    alignas(16) float delta[2][kBT];
-    uint64_t kv_full, qdo_full[2], qdo_empty[2];
+    // dQ staging for the TMA reduce: one 32-column box [row][32 floats], swizzled
+    alignas(1024) float stage[kBT * 32];
+    alignas(16) float lse2[kQStages][kBT];
+    alignas(16) float delta[kQStages][kBT];
+    uint64_t kv_full, qdo_full[kQStages], qdo_empty[kQStages];
     uint64_t sdp_full, sdp_free, p_ready[2], ds_ready[2], p_free, ds_free[2];
     uint64_t dq_full, dq_free, acc_done, drain;
     uint32_t tmem_slot;
@@ -157,15 +161,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.kv_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kQStages; ++s) {
             mbar_init(&sm.qdo_full[s], 1);
             mbar_init(&sm.qdo_empty[s], 1);
-            mbar_init(&sm.p_ready[s], kBT);
-            mbar_init(&sm.ds_ready[s], kBT);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.p_ready[s], kEwThreads);
+            mbar_init(&sm.ds_ready[s], kEwThreads);
             mbar_init(&sm.ds_free[s], 1);
         }
         mbar_init(&sm.sdp_full, 1);
-        mbar_init(&sm.sdp_free, kBT);
+        mbar_init(&sm.sdp_free, kEwThreads);
         mbar_init(&sm.p_free, 1);
         mbar_init(&sm.dq_full, 1);
         mbar_init(&sm.dq_free, kBT);
@@ -184,133 +190,136 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tP = tmem + 256 + 3 * D;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (whole warp,
+        // one elected lane issues)
         if (lane == 0) {
             prefetch_tensormap(&tq);
             prefetch_tensormap(&tk);
             prefetch_tensormap(&tv);
             prefetch_tensormap(&tdo);
-            mbar_arrive_expect_tx(&sm.kv_full, 2 * Smem::kTileBytes);
-            tma_load_3d(sm.k, &tk, &sm.kv_full, 0, kt * kBT, bh);
-            tma_load_3d(sm.v, &tv, &sm.kv_full, 0, kt * kBT, bh);
-            int issued = 0;
-            for (int idx = 0; idx < n_q; ++idx) {
-                const int st = idx & 1;
-                const int i = kt + idx;
-                if (!mbar_wait(&sm.qdo_empty[st], (uint32_t)((idx >> 1) & 1) ^ 1u, err, abort)) break;
-                mbar_arrive_expect_tx(&sm.qdo_full[st], 2 * Smem::kTileBytes + 2 * kBT * 4);
-                tma_load_3d(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, bh);
-                tma_load_3d(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, bh);
-                const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
-                bulk_load(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
-                bulk_load(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
-                issued = idx + 1;
-            }
-            for (int idx = (issued > 2 ? issued - 2 : 0); idx < issued; ++idx)
-                for (uint32_t n = 0; n < kWaitLimit && !mbar_try_wait(&sm.qdo_full[idx & 1], (uint32_t)(idx >> 1) & 1u); ++n) {}
-            mbar_wait(&sm.kv_full, 0, err, abort);
         }
+        __syncwarp();
+        mbar_arrive_expect_tx_e(&sm.kv_full, 2 * Smem::kTileBytes);
+        tma_load_3d_e(sm.k, &tk, &sm.kv_full, 0, kt * kBT, bh);
+        tma_load_3d_e(sm.v, &tv, &sm.kv_full, 0, kt * kBT, bh);
+        int issued = 0;
+        for (int idx = 0; idx < n_q; ++idx) {
+            const int st = idx % kQStages;
+            const int i = kt + idx;
+            if (!mbar_wait_warp(&sm.qdo_empty[st], (uint32_t)((idx / kQStages) & 1) ^ 1u, err, abort)) break;
+            mbar_arrive_expect_tx_e(&sm.qdo_full[st], 2 * Smem::kTileBytes + 2 * kBT * 4);
+            tma_load_3d_e(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, bh);
+            tma_load_3d_e(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, bh);
+            const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
+            bulk_load_e(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
+            bulk_load_e(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
+            issued = idx + 1;
+        }
+        for (int idx = (issued > kQStages ? issued - kQStages : 0); idx < issued; ++idx)
+            for (uint32_t n = 0; n < kWaitLimit && !mbar_try_wait(&sm.qdo_full[idx % kQStages], (uint32_t)(idx / kQStages) & 1u); ++n) {}
+        mbar_wait_warp(&sm.kv_full, 0, err, abort);
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16(kBT, kBT, 0, 0);  // S^T, dP^T: both K-major
-            constexpr uint32_t idKV = idesc_bf16(kBT, D, 0, 1);   // dV, dK: A K-major/TMEM, B MN-major
-            constexpr uint32_t idQ = idesc_bf16(kBT, D, 1, 1);    // dQ: A (dS) and B (K) MN-major
-            const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
-            bool ok = mbar_wait(&sm.kv_full, 0, err, abort);
-            for (int idx = 0; ok && idx <= n_q; ++idx) {
-                if (idx < n_q) {
-                    const int st = idx & 1;
-                    if (!(ok = mbar_wait(&sm.qdo_full[st], (uint32_t)(idx >> 1) & 1u, err, abort))) break;
-                    if (idx >= 1 && !(ok = mbar_wait(&sm.sdp_free, (uint32_t)(idx - 1) & 1u, err, abort))) break;
-                    tc_fence_after();
-                    const uint32_t q_addr = smem_u32(sm.q[st]), do_addr = smem_u32(sm.dO[st]);
+        // ------------------------------------------------ MMA issuer (whole warp,
+        // one elected lane issues)
+        constexpr uint32_t idS = idesc_bf16(kBT, kBT, 0, 0);  // S^T, dP^T: both K-major
+        constexpr uint32_t idKV = idesc_bf16(kBT, D, 0, 1);   // dV, dK: A K-major/TMEM, B MN-major
+        constexpr uint32_t idQ = idesc_bf16(kBT, D, 1, 1);    // dQ: A (dS) and B (K) MN-major
+        const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+        bool ok = mbar_wait_warp(&sm.kv_full, 0, err, abort);
+        for (int idx = 0; ok && idx <= n_q; ++idx) {
+            if (idx < n_q) {
+                const int st = idx % kQStages;
+                if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(idx / kQStages) & 1u, err, abort))) break;
+                if (idx >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(idx - 1) & 1u, err, abort))) break;
+                tc_fence_after();
+                const uint32_t q_addr = smem_u32(sm.q[st]), do_addr = smem_u32(sm.dO[st]);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tS, smem_desc(k_addr + kk * 32, 16, kAtom, kSwz),
-                               smem_desc(q_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss_e(tS, smem_desc(k_addr + kk * 32, 16, kAtom, kSwz),
+                             smem_desc(q_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tdP, smem_desc(v_addr + kk * 32, 16, kAtom, kSwz),
-                               smem_desc(do_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
-                    mma_commit(&sm.sdp_full);
-                }
-                if (idx >= 1) {
-                    const int p = idx - 1;  // the tile whose gradients are now issued
-                    const int st = p & 1, b = p & 1;
-                    const uint32_t q_addr = smem_u32(sm.q[st]), do_addr = smem_u32(sm.dO[st]);
-                    const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
-                    if (!(ok = mbar_wait(&sm.p_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int s = 0; s < kBT / 16; ++s)  // dV += P^T dO, K = 16 queries per step
-                        mma_ts(tdV, tP + s * 8,
-                               smem_desc(do_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
-                               idKV, (p > 0 || s > 0) ? 1u : 0u);
-                    mma_commit(&sm.p_free);
-                    if (!(ok = mbar_wait(&sm.ds_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int s = 0; s < kBT / 16; ++s)  // dK += dS^T Q
-                        mma_ss(tdK,
-                               smem_desc(ds_addr + (s >> 2) * kHalf + (s & 3) * 32, 16, 1024, kSwizzle128B),
-                               smem_desc(q_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
-                               idKV, (p > 0 || s > 0) ? 1u : 0u);
-                    if (p >= 1 && !(ok = mbar_wait(&sm.dq_free, (uint32_t)(p - 1) & 1u, err, abort))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int s = 0; s < kBT / 16; ++s)  // dQ_i = dS K, K = 16 keys per step
-                        mma_ss(tdQ, smem_desc(ds_addr + s * 16 * 128, kHalf, 1024, kSwizzle128B),
-                               smem_desc(k_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
-                               idQ, s > 0 ? 1u : 0u);
-                    mma_commit(&sm.dq_full);
-                    mma_commit(&sm.qdo_empty[st]);
-                    mma_commit(&sm.ds_free[b]);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss_e(tdP, smem_desc(v_addr + kk * 32, 16, kAtom, kSwz),
+                             smem_desc(do_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
+                mma_commit_e(&sm.sdp_full);
             }
-            mma_commit(&sm.acc_done);
-            mma_commit(&sm.drain);
-            mbar_wait(&sm.drain, 0, err, abort);
+            if (idx >= 1) {
+                const int p = idx - 1;  // the tile whose gradients are now issued
+                const int st = p % kQStages, b = p & 1;
+                const uint32_t q_addr = smem_u32(sm.q[st]), do_addr = smem_u32(sm.dO[st]);
+                const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
+                if (!(ok = mbar_wait_warp(&sm.p_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < kBT / 16; ++s)  // dV += P^T dO, K = 16 queries per step
+                    mma_ts_e(tdV, tP + s * 8,
+                             smem_desc(do_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
+                             idKV, (p > 0 || s > 0) ? 1u : 0u);
+                mma_commit_e(&sm.p_free);
+                if (!(ok = mbar_wait_warp(&sm.ds_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < kBT / 16; ++s)  // dK += dS^T Q
+                    mma_ss_e(tdK,
+                             smem_desc(ds_addr + (s >> 2) * kHalf + (s & 3) * 32, 16, 1024, kSwizzle128B),
+                             smem_desc(q_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
+                             idKV, (p > 0 || s > 0) ? 1u : 0u);
+                mma_commit_e(&sm.qdo_empty[st]);  // Q, dO, lse, Delta of this tile are consumed
+                if (p >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(p - 1) & 1u, err, abort))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < kBT / 16; ++s)  // dQ_i = dS K, K = 16 keys per step
+                    mma_ss_e(tdQ, smem_desc(ds_addr + s * 16 * 128, kHalf, 1024, kSwizzle128B),
+                             smem_desc(k_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
+                             idQ, s > 0 ? 1u : 0u);
+                mma_commit_e(&sm.dq_full);
+                mma_commit_e(&sm.ds_free[b]);
+            }
         }
-    } else if (warp < 6) {
+        mma_commit_e(&sm.acc_done);
+        mma_commit_e(&sm.drain);
+        mbar_wait_warp(&sm.drain, 0, err, abort);
+    } else if (warp < 10) {
         // ------------------------------------------------ softmax gradient
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;               // query columns [64 half, 64 half + 64)
         const int kr = quad * 32 + lane;                // key row within the tile (TMEM lane)
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t sw = (uint32_t)(kr & 7);
         bool ok = true;
         for (int idx = 0; idx < n_q; ++idx) {
-            const int st = idx & 1, b = idx & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&sm.sdp_full, (uint32_t)idx & 1u, err, abort));
+            const int st = idx % kQStages, b = idx & 1;
+            ok = mbar_wait_warp(&sm.sdp_full, (uint32_t)idx & 1u, err, abort);
             if (!ok) break;
             tc_fence_after();
             const bool diag = (idx == 0);
             const uint32_t lse_addr = smem_u32(sm.lse2[st]), dl_addr = smem_u32(sm.delta[st]);
-            const uint32_t ds_row = smem_u32(sm.ds[b][0]) + (uint32_t)kr * 128;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {  // 32 query columns per chunk
+            const uint32_t ds_row = smem_u32(sm.ds[b][half]) + (uint32_t)kr * 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {  // 32 query columns per chunk
+                const int q0 = 64 * half + 32 * c;
                 uint32_t rs[32], rp[32];
-                tmem_ld32(tS + lane_off + 32 * c, rs);
-                tmem_ld32(tdP + lane_off + 32 * c, rp);
+                tmem_ld32(tS + lane_off + q0, rs);
+                tmem_ld32(tdP + lane_off + q0, rp);
                 tmem_wait_ld();
                 reg_fence32(rs);
                 reg_fence32(rp);
-                if (c == 3) {  // S^T and dP^T fully read: the next tile may overwrite them
+                if (c == 1) {  // this warp's S^T and dP^T columns are read: the next tile may overwrite them
                     tc_fence_before();
                     mbar_arrive(&sm.sdp_free);
                 }
                 uint32_t pw[16], dw[16];
 #pragma unroll
                 for (int x = 0; x < 32; x += 4) {
-                    const float4 l4 = ld_shared_f4(lse_addr + (32 * c + x) * 4);
-                    const float4 d4 = ld_shared_f4(dl_addr + (32 * c + x) * 4);
+                    const float4 l4 = ld_shared_f4(lse_addr + (q0 + x) * 4);
+                    const float4 d4 = ld_shared_f4(dl_addr + (q0 + x) * 4);
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
                     const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
                     float pp[4], dd[4];
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
                         float pv = ex2(fmaf(__uint_as_float(rs[x + y]), scale_log2, -lv[y]));
-                        if (diag && (32 * c + x + y) < kr) pv = 0.f;  // query before key: masked
+                        if (diag && (q0 + x + y) < kr) pv = 0.f;  // query before key: masked
                         pp[y] = pv;
                         dd[y] = pv * (__uint_as_float(rp[x + y]) - dvv[y]);
                     }
@@ -329,12 +338,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
                 }
-                tmem_st16(tP + lane_off + 16 * c, pw);
+                tmem_st16(tP + lane_off + q0 / 2, pw);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {  // four 16-byte chunks = 32 queries
-                    const uint32_t g = 4 * c + u;          // 8-query group 0..15
-                    const uint32_t addr = ds_row + (g >> 3) * kHalf + (((g & 7) ^ sw) << 4);
-                    st_shared_v4(addr, dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
+                    const uint32_t g = 4 * c + u;          // 8-query group within this half
+                    st_shared_v4(ds_row + ((g ^ sw) << 4), dw[4 * u], dw[4 * u + 1], dw[4 * u + 2],
+                                 dw[4 * u + 3]);
                 }
             }
             if (!ok) break;
@@ -344,34 +353,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&sm.p_ready[b]);
             mbar_arrive(&sm.ds_ready[b]);
         }
-        // ---- epilogue: dK (times scale) and dV of this key tile
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_done, 0, err, abort));
+        // ---- epilogue: dK (times scale) from the first half's warps, dV from the second's
+        if (ok) ok = mbar_wait_warp(&sm.acc_done, 0, err, abort);
         if (ok) {
             tc_fence_after();
             const int t = kt * kBT + kr;
             const size_t grow = (size_t)bh * T + t;
+            const uint32_t src = half == 0 ? tdK : tdV;
+            const float mul = half == 0 ? scale : 1.f;
+            __nv_bfloat16 *out = half == 0 ? dk : dv;
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t src = which == 0 ? tdK : tdV;
-                const float mul = which == 0 ? scale : 1.f;
-                __nv_bfloat16 *out = which == 0 ? dk : dv;
+            for (int c = 0; c < D; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(src + lane_off + c, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+                if (t < T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + grow * D + c);
 #pragma unroll
-                for (int c = 0; c < D; c += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(src + lane_off + c, r);
-                    tmem_wait_ld();
-                    reg_fence32(r);
-                    if (t < T) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(out + grow * D + c);
-#pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            uint4 w4;
-                            w4.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * mul, __uint_as_float(r[8 * x + 1]) * mul);
-                            w4.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * mul, __uint_as_float(r[8 * x + 3]) * mul);
-                            w4.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * mul, __uint_as_float(r[8 * x + 5]) * mul);
-                            w4.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * mul, __uint_as_float(r[8 * x + 7]) * mul);
-                            dst[x] = w4;
-                        }
+                    for (int x = 0; x < 4; ++x) {
+                        uint4 w4;
+                        w4.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * mul, __uint_as_float(r[8 * x + 1]) * mul);
+                        w4.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * mul, __uint_as_float(r[8 * x + 3]) * mul);
+                        w4.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * mul, __uint_as_float(r[8 * x + 5]) * mul);
+                        w4.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * mul, __uint_as_float(r[8 * x + 7]) * mul);
+                        dst[x] = w4;
                     }
                 }
             }
@@ -381,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;
         const int qr = quad * 32 + lane;                // query row within the tile
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const bool leader = (warp == 6 && lane == 0);
+        const bool leader = (warp == 10 && lane == 0);
         const uint32_t sw = (uint32_t)(qr & 7);
         for (int idx = 0; idx < n_q; ++idx) {
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, (uint32_t)idx & 1u, err, abort));
@@ -395,23 +401,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int h = 0; h < D / 32; ++h) reg_fence32(r[h]);
             tc_fence_before();
             mbar_arrive(&sm.dq_free);
-            if (leader) bulk_wait_read_all();   // previous reduce has read the staging
-            named_bar_sync(1, 128);
 #pragma unroll
             for (int h = 0; h < D / 32; ++h) {
-                const uint32_t row = smem_u32(sm.stage[h]) + (uint32_t)qr * 128;
+                if (leader) bulk_wait_read_all();  // the previous reduce has read the staging box
+                named_bar_sync(1, 128);
+                const uint32_t row = smem_u32(sm.stage) + (uint32_t)qr * 128;
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
                     st_shared_v4(row + ((u ^ sw) << 4), r[h][4 * u], r[h][4 * u + 1], r[h][4 * u + 2],
                                  r[h][4 * u + 3]);
-            }
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (leader) {
-#pragma unroll
-                for (int h = 0; h < D / 32; ++h)
-                    tma_reduce_add_3d(&tdq, sm.stage[h], 32 * h, (kt + idx) * kBT, bh);
-                bulk_commit();
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (leader) {
+                    tma_reduce_add_3d(&tdq, sm.stage, 32 * h, (kt + idx) * kBT, bh);
+                    bulk_commit();
+                }
             }
         }
         if (leader) bulk_wait_all();

@@ -8,17 +8,19 @@
 // [55:20] for the -inf upper triangle and the softmax).
 //
 // One CTA per (128-row query tile, head); heaviest tiles (most key tiles
-// under the causal mask) are launched first.  Six warps:
-//   warp 0      TMA producer: Q once, then K_j / V_j tiles into a 3-stage ring
-//   warp 1      tcgen05 issuer: S_j = Q K_j^T into TMEM (double buffered),
-//               O += P_j V_j with P_j read from TMEM; owns the TMEM allocation
+// under the causal mask) are launched first.  Two CTAs share an SM (256 TMEM
+// columns, ~81 KB shared memory and <= 168 registers each), so one CTA's
+// softmax overlaps the other's MMAs and both keep the exp unit busy.  Six warps:
+//   warp 0      TMA producer: Q once, then K_j / V_j tiles into a 2-stage ring
+//   warp 1      tcgen05 issuer: S_j = Q K_j^T into TMEM, O += P_j V_j with P_j
+//               read from TMEM; owns the TMEM allocation
 //   warps 2..5  softmax: one query row per thread (TMEM lane), online max and
 //               sum in registers, P_j written back to TMEM as bf16 over S_j,
 //               lazy rescale of the O accumulator, final O / l and lse.
 // Key tiles wholly above the diagonal are never loaded; only the diagonal
 // tile applies the element mask.  The score matrix never leaves the SM.
 //
-// TMEM columns: S_0 [0,128), S_1 [128,256), O [256, 256+D).
+// TMEM columns: S (then P) [0,128), O [128, 128+D).
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -31,9 +33,9 @@ using namespace sm100;
 
 constexpr int kBM = 128;          // query rows per CTA (= TMEM lanes)
 constexpr int kBN = 128;          // key rows per tile
-constexpr int kStages = 3;        // K/V ring depth
+constexpr int kStages = 2;        // K/V ring depth
 constexpr int kThreads = 192;     // 6 warps
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
 
 template <int D>
@@ -44,14 +46,14 @@ struct FwdSmem {
     alignas(1024) __nv_bfloat16 v[kStages][kBN * D];
     uint64_t q_full;
     uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
-    uint64_t s_full[2], p_full[2];
+    uint64_t s_full, p_full;
     uint64_t o_done, o_final, drain;
     uint32_t tmem_slot;
     int abort;
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16 *__restrict__ o,
                float *__restrict__ lse, int T, int BH, int ntiles, float scale_log2, int *err) {
@@ -77,10 +79,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.k_empty[s], 1);
             mbar_init(&sm.v_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.p_full[b], kBM);
-        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.p_full, kBM);
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.o_final, 1);
         mbar_init(&sm.drain, 1);
@@ -92,84 +92,87 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_slot;
-    const uint32_t tS[2] = {tmem, tmem + 128};
-    const uint32_t tO = tmem + 256;
+    const uint32_t tS = tmem;
+    const uint32_t tO = tmem + 128;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (whole warp,
+        // one elected lane issues)
         if (lane == 0) {
             prefetch_tensormap(&tq);
             prefetch_tensormap(&tk);
             prefetch_tensormap(&tv);
-            mbar_arrive_expect_tx(&sm.q_full, Smem::kTileBytes);
-            tma_load_3d(sm.q, &tq, &sm.q_full, 0, qt * kBM, bh);
-            int issued = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j % kStages;
-                const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-                if (!mbar_wait(&sm.k_empty[s], ph ^ 1u, err, abort)) break;
-                mbar_arrive_expect_tx(&sm.k_full[s], Smem::kTileBytes);
-                tma_load_3d(sm.k[s], &tk, &sm.k_full[s], 0, j * kBN, bh);
-                if (!mbar_wait(&sm.v_empty[s], ph ^ 1u, err, abort)) {
-                    issued = j + 1;  // K_j is in flight
-                    mbar_wait(&sm.k_full[s], ph, err, abort);
-                    break;
-                }
-                mbar_arrive_expect_tx(&sm.v_full[s], Smem::kTileBytes);
-                tma_load_3d(sm.v[s], &tv, &sm.v_full[s], 0, j * kBN, bh);
-                issued = j + 1;
-            }
-            // Drain: every load this thread issued has landed before exit.
-            for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
-                const int s = j % kStages;
-                const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
-                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.v_full[s], ph); ++i) {}
-            }
-            mbar_wait(&sm.q_full, 0, err, abort);
         }
+        __syncwarp();
+        mbar_arrive_expect_tx_e(&sm.q_full, Smem::kTileBytes);
+        tma_load_3d_e(sm.q, &tq, &sm.q_full, 0, qt * kBM, bh);
+        int issued = 0;
+        for (int j = 0; j < n_kv; ++j) {
+            const int s = j % kStages;
+            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+            if (!mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort)) break;
+            mbar_arrive_expect_tx_e(&sm.k_full[s], Smem::kTileBytes);
+            tma_load_3d_e(sm.k[s], &tk, &sm.k_full[s], 0, j * kBN, bh);
+            if (!mbar_wait_warp(&sm.v_empty[s], ph ^ 1u, err, abort)) {
+                issued = j + 1;  // K_j is in flight
+                mbar_wait_warp(&sm.k_full[s], ph, err, abort);
+                break;
+            }
+            mbar_arrive_expect_tx_e(&sm.v_full[s], Smem::kTileBytes);
+            tma_load_3d_e(sm.v[s], &tv, &sm.v_full[s], 0, j * kBN, bh);
+            issued = j + 1;
+        }
+        // Drain: every load this warp issued has landed before exit.
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
+            const int s = j % kStages;
+            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+            for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
+            for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.v_full[s], ph); ++i) {}
+        }
+        mbar_wait_warp(&sm.q_full, 0, err, abort);
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);  // Q, K both K-major
-            constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);    // P from TMEM, V MN-major
-            const uint32_t q_addr = smem_u32(sm.q);
-            bool ok = mbar_wait(&sm.q_full, 0, err, abort);
-            for (int j = 0; ok && j <= n_kv; ++j) {
-                if (j < n_kv) {
-                    const int s = j % kStages;
-                    if (!(ok = mbar_wait(&sm.k_full[s], (uint32_t)(j / kStages) & 1u, err, abort))) break;
-                    if (j >= 2 && !(ok = mbar_wait(&sm.o_done, (uint32_t)(j - 2) & 1u, err, abort))) break;
-                    tc_fence_after();
-                    const uint32_t k_addr = smem_u32(sm.k[s]);
+        // ------------------------------------------------ MMA issuer (whole warp,
+        // one elected lane issues)
+        constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);  // Q, K both K-major
+        constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);    // P from TMEM, V MN-major
+        const uint32_t q_addr = smem_u32(sm.q);
+        bool ok = mbar_wait_warp(&sm.q_full, 0, err, abort);
+        for (int j = 0; ok && j <= n_kv; ++j) {
+            if (j >= 1) {
+                // O += P_{j-1} V_{j-1}, P read from TMEM over S.
+                const int jj = j - 1;
+                const int s = jj % kStages;
+                if (!(ok = mbar_wait_warp(&sm.p_full, (uint32_t)jj & 1u, err, abort))) break;
+                if (!(ok = mbar_wait_warp(&sm.v_full[s], (uint32_t)(jj / kStages) & 1u, err, abort))) break;
+                tc_fence_after();
+                const uint32_t v_addr = smem_u32(sm.v[s]);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tS[j & 1], smem_desc(q_addr + kk * 32, 16, kAtom, kSwz),
-                               smem_desc(k_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
-                    mma_commit(&sm.s_full[j & 1]);
-                    mma_commit(&sm.k_empty[s]);
-                }
-                if (j >= 1) {
-                    const int jj = j - 1;
-                    const int s = jj % kStages;
-                    if (!(ok = mbar_wait(&sm.p_full[jj & 1], (uint32_t)(jj >> 1) & 1u, err, abort))) break;
-                    if (!(ok = mbar_wait(&sm.v_full[s], (uint32_t)(jj / kStages) & 1u, err, abort))) break;
-                    tc_fence_after();
-                    const uint32_t v_addr = smem_u32(sm.v[s]);
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_ts(tO, tS[jj & 1] + kk * 8,
-                               smem_desc(v_addr + kk * 16 * kRowBytes, kBN * kRowBytes, kAtom, kSwz),
-                               idO, (jj > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(&sm.o_done);
-                    mma_commit(&sm.v_empty[s]);
-                }
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_ts_e(tO, tS + kk * 8,
+                             smem_desc(v_addr + kk * 16 * kRowBytes, kBN * kRowBytes, kAtom, kSwz),
+                             idO, (jj > 0 || kk > 0) ? 1u : 0u);
+                mma_commit_e(&sm.o_done);
+                mma_commit_e(&sm.v_empty[s]);
             }
-            // All MMAs this thread issued are complete once `drain` fires.
-            mma_commit(&sm.o_final);
-            mma_commit(&sm.drain);
-            mbar_wait(&sm.drain, 0, err, abort);
+            if (j < n_kv) {
+                // S_j = Q K_j^T overwrites P_{j-1}: PV_{j-1} must have completed.
+                const int s = j % kStages;
+                if (!(ok = mbar_wait_warp(&sm.k_full[s], (uint32_t)(j / kStages) & 1u, err, abort))) break;
+                if (j >= 1 && !(ok = mbar_wait_warp(&sm.o_done, (uint32_t)(j - 1) & 1u, err, abort))) break;
+                tc_fence_after();
+                const uint32_t k_addr = smem_u32(sm.k[s]);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss_e(tS, smem_desc(q_addr + kk * 32, 16, kAtom, kSwz),
+                             smem_desc(k_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
+                mma_commit_e(&sm.s_full);
+                mma_commit_e(&sm.k_empty[s]);
+            }
         }
+        // All MMAs this warp issued are complete once `drain` fires.
+        mma_commit_e(&sm.o_final);
+        mma_commit_e(&sm.drain);
+        mbar_wait_warp(&sm.drain, 0, err, abort);
     } else {
         // ------------------------------------------------ softmax warps
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
@@ -178,28 +181,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
-            const int b = j & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (uint32_t)(j >> 1) & 1u, err, abort));
+            ok = mbar_wait_warp(&sm.s_full, (uint32_t)j & 1u, err, abort);
             if (!ok) break;
             tc_fence_after();
             float s[kBN];
-#pragma unroll
-            for (int c = 0; c < kBN; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tS[b] + lane_off + c, r);
+            {
+                // All four 32-column loads in flight before one wait.
+                uint32_t r0[32], r1[32], r2[32], r3[32];
+                tmem_ld32(tS + lane_off + 0, r0);
+                tmem_ld32(tS + lane_off + 32, r1);
+                tmem_ld32(tS + lane_off + 64, r2);
+                tmem_ld32(tS + lane_off + 96, r3);
                 tmem_wait_ld();
-                reg_fence32(r);
+                reg_fence32(r0);
+                reg_fence32(r1);
+                reg_fence32(r2);
+                reg_fence32(r3);
 #pragma unroll
-                for (int x = 0; x < 32; ++x) s[c + x] = __uint_as_float(r[x]);
+                for (int x = 0; x < 32; ++x) {
+                    s[x] = __uint_as_float(r0[x]);
+                    s[32 + x] = __uint_as_float(r1[x]);
+                    s[64 + x] = __uint_as_float(r2[x]);
+                    s[96 + x] = __uint_as_float(r3[x]);
+                }
             }
             if (j == n_kv - 1) {  // diagonal tile: key column c is visible to row r iff c <= r
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
                     if (c > row) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // Row max as eight independent chains (short dependency depth).
+            float mc[8];
 #pragma unroll
-            for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+            for (int x = 0; x < 8; ++x) mc[x] = s[x];
+#pragma unroll
+            for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+                for (int x = 0; x < 8; ++x) mc[x] = fmaxf(mc[x], s[c + x]);
+            const float mx = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
+                                   fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
             const float mxs = mx * scale_log2;
             // Each row moves its own running max only when its scores exceed
             // it by more than the threshold; the warp merely decides whether
@@ -215,14 +235,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < D; c += 32) {
-                        uint32_t r[32];
-                        tmem_ld32(tO + lane_off + c, r);
+                    for (int c = 0; c < D; c += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(tO + lane_off + c, r);
                         tmem_wait_ld();
-                        reg_fence32(r);
+                        reg_fence16(r);
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-                        tmem_st32(tO + lane_off + c, r);
+                        for (int x = 0; x < 16; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+                        tmem_st16(tO + lane_off + c, r);
                     }
                 }
                 l *= alpha;
@@ -230,20 +250,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float neg_m = -m_used;
 #pragma unroll
-            for (int c = 0; c < kBN; c += 64) {
-                uint32_t pk[32];
+            for (int c = 0; c < kBN; c += 32) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
+                for (int x = 0; x < 16; ++x) {
                     const float p0 = ex2(fmaf(s[c + 2 * x], scale_log2, neg_m));
                     const float p1 = ex2(fmaf(s[c + 2 * x + 1], scale_log2, neg_m));
                     l += p0 + p1;
                     pk[x] = pack_bf16x2(p0, p1);
                 }
-                tmem_st32(tS[b] + lane_off + c / 2, pk);
+                tmem_st16(tS + lane_off + c / 2, pk);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sm.p_full[b]);
+            mbar_arrive(&sm.p_full);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, 0, err, abort));
         if (ok) {
