@@ -80,56 +80,65 @@ struct BwdSmem {
 
 // ------------------------------------------------------------------ prep
 
+// One thread per (tile-padded row, 16-byte chunk of the row): D/8 threads per
+// row read O and dO with coalesced 16-byte loads, Delta_i is reduced across
+// them with shuffles, and the same threads zero their part of the dQ
+// accumulator row.
 template <int D>
-__global__ void __launch_bounds__(128) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
                                                        const __nv_bfloat16 *__restrict__ dO,
                                                        const float *__restrict__ lse,
                                                        float *__restrict__ lse2,
                                                        float *__restrict__ delta,
-                                                       float *__restrict__ dq_acc, int T, int Tpad) {
-    const int nt = Tpad / 128;
-    const long long bh = blockIdx.x / nt;
-    const int t = (int)(blockIdx.x - bh * nt) * 128 + threadIdx.x;
-    if (t >= Tpad) return;
-    const size_t prow = (size_t)bh * Tpad + t;
-    if (t < T) {
-        const size_t row = (size_t)bh * T + t;
-        const uint4 *po = reinterpret_cast<const uint4 *>(o + row * D);
-        const uint4 *pg = reinterpret_cast<const uint4 *>(dO + row * D);
-        float acc = 0.f;
+                                                       float *__restrict__ dq_acc, int T, int Tpad,
+                                                       long long prows) {
+    constexpr int kTpr = D / 8;  // threads per row (a power of two dividing 32)
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long prow = gid / kTpr;
+    const int c = (int)(gid - prow * kTpr);
+    const bool valid = prow < prows;
+    const long long bh = valid ? prow / Tpad : 0;
+    const int t = valid ? (int)(prow - bh * Tpad) : 0;
+    const bool live = valid && t < T;
+    const size_t row = (size_t)bh * T + t;
+    float acc = 0.f;
+    if (live) {
+        const uint4 a = reinterpret_cast<const uint4 *>(o + row * D)[c];
+        const uint4 g = reinterpret_cast<const uint4 *>(dO + row * D)[c];
+        const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&g);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            const uint4 a = po[c], b = pg[c];
-            const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
-            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&b);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const float2 fa = __bfloat1622float2(a2[x]), fb = __bfloat1622float2(b2[x]);
-                acc = fmaf(fa.x, fb.x, acc);
-                acc = fmaf(fa.y, fb.y, acc);
-            }
+        for (int x = 0; x < 4; ++x) {
+            const float2 fa = __bfloat1622float2(a2[x]), fg = __bfloat1622float2(g2[x]);
+            acc = fmaf(fa.x, fg.x, acc);
+            acc = fmaf(fa.y, fg.y, acc);
         }
-        delta[prow] = acc;
-        lse2[prow] = lse[row] * kLog2e;
-        float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D);
+        float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D + 8 * c);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
-        for (int c = 0; c < D / 4; ++c) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-        delta[prow] = 0.f;
-        lse2[prow] = INFINITY;
+    for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (valid && c == 0) {
+        delta[prow] = live ? acc : 0.f;
+        lse2[prow] = live ? lse[row] * kLog2e : INFINITY;
     }
 }
 
 // ------------------------------------------------------------------ post
 
-__global__ void bwd_post_kernel(const float4 *__restrict__ acc, uint2 *__restrict__ dq, long long n4,
+// dQ = scale * accumulator, 8 elements per thread (two 16-byte loads, one
+// 16-byte store).
+__global__ void bwd_post_kernel(const float4 *__restrict__ acc, uint4 *__restrict__ dq, long long n8,
                                 float scale) {
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
          i += (long long)gridDim.x * blockDim.x) {
-        const float4 a = acc[i];
-        uint2 r;
+        const float4 a = acc[2 * i], b = acc[2 * i + 1];
+        uint4 r;
         r.x = pack_bf16x2(a.x * scale, a.y * scale);
         r.y = pack_bf16x2(a.z * scale, a.w * scale);
+        r.z = pack_bf16x2(b.x * scale, b.y * scale);
+        r.w = pack_bf16x2(b.z * scale, b.w * scale);
         dq[i] = r;
     }
 }
@@ -466,7 +475,10 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if ((e = make_map(&mdo, dO, BH, s.T, D, false, D)) != cudaSuccess) return e;
     if ((e = make_map(&mdq, dq_acc, BH, s.T, D, true, 32)) != cudaSuccess) return e;
 
-    bwd_prep_kernel<D><<<(unsigned)blocks, 128, 0, st>>>(o, dO, lse, lse2, delta, dq_acc, s.T, Tpad);
+    const long long prows = (long long)BH * Tpad;
+    const long long prep_threads = prows * (D / 8);
+    bwd_prep_kernel<D><<<(unsigned)((prep_threads + 255) / 256), 256, 0, st>>>(
+        o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
 
@@ -481,10 +493,11 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     li.kernels += 1;
     if ((e = mark_main_end(li, st)) != cudaSuccess) return e;
 
-    const long long n4 = (long long)BH * s.T * D / 4;
-    const int post_blocks = (int)((n4 + 255) / 256 < 148 * 16 ? (n4 + 255) / 256 : 148 * 16);
+    const long long n8 = (long long)BH * s.T * D / 8;
+    const long long want = (n8 + 255) / 256;
+    const int post_blocks = (int)(want < 148 * 16 ? want : 148 * 16);
     bwd_post_kernel<<<post_blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc),
-                                                  reinterpret_cast<uint2 *>(dq), n4, s.scale);
+                                                  reinterpret_cast<uint4 *>(dq), n8, s.scale);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
     return cudaSuccess;

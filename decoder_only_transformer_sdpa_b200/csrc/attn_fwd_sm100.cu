@@ -13,14 +13,15 @@
 // softmax overlaps the other's MMAs and both keep the exp unit busy.  Six warps:
 //   warp 0      TMA producer: Q once, then K_j / V_j tiles into a 2-stage ring
 //   warp 1      tcgen05 issuer: S_j = Q K_j^T into TMEM, O += P_j V_j with P_j
-//               read from TMEM; owns the TMEM allocation
+//               read from TMEM; owns the TMEM allocation.  S_{j+1} is issued as
+//               soon as the softmax has read S_j, so it overlaps softmax j.
 //   warps 2..5  softmax: one query row per thread (TMEM lane), online max and
-//               sum in registers, P_j written back to TMEM as bf16 over S_j,
-//               lazy rescale of the O accumulator, final O / l and lse.
+//               sum in registers, P_j written to TMEM as bf16, lazy rescale of
+//               the O accumulator, final O / l and lse.
 // Key tiles wholly above the diagonal are never loaded; only the diagonal
 // tile applies the element mask.  The score matrix never leaves the SM.
 //
-// TMEM columns: S (then P) [0,128), O [128, 128+D).
+// TMEM columns: S [0,128), P (bf16 pairs) [128,192), O [192, 192+D).
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -46,7 +47,7 @@ struct FwdSmem {
     alignas(1024) __nv_bfloat16 v[kStages][kBN * D];
     uint64_t q_full;
     uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
-    uint64_t s_full, p_full;
+    uint64_t s_full, s_free, p_full;
     uint64_t o_done, o_final, drain;
     uint32_t tmem_slot;
     int abort;
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(&sm.v_empty[s], 1);
         }
         mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.s_free, kBM);
         mbar_init(&sm.p_full, kBM);
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.o_final, 1);
@@ -93,7 +95,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_slot;
     const uint32_t tS = tmem;
-    const uint32_t tO = tmem + 128;
+    const uint32_t tP = tmem + 128;
+    const uint32_t tO = tmem + 192;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (whole warp,
@@ -138,27 +141,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t q_addr = smem_u32(sm.q);
         bool ok = mbar_wait_warp(&sm.q_full, 0, err, abort);
         for (int j = 0; ok && j <= n_kv; ++j) {
-            if (j >= 1) {
-                // O += P_{j-1} V_{j-1}, P read from TMEM over S.
-                const int jj = j - 1;
-                const int s = jj % kStages;
-                if (!(ok = mbar_wait_warp(&sm.p_full, (uint32_t)jj & 1u, err, abort))) break;
-                if (!(ok = mbar_wait_warp(&sm.v_full[s], (uint32_t)(jj / kStages) & 1u, err, abort))) break;
-                tc_fence_after();
-                const uint32_t v_addr = smem_u32(sm.v[s]);
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts_e(tO, tS + kk * 8,
-                             smem_desc(v_addr + kk * 16 * kRowBytes, kBN * kRowBytes, kAtom, kSwz),
-                             idO, (jj > 0 || kk > 0) ? 1u : 0u);
-                mma_commit_e(&sm.o_done);
-                mma_commit_e(&sm.v_empty[s]);
-            }
             if (j < n_kv) {
-                // S_j = Q K_j^T overwrites P_{j-1}: PV_{j-1} must have completed.
+                // S_j = Q K_j^T, once the softmax has read S_{j-1} out of TMEM.
                 const int s = j % kStages;
                 if (!(ok = mbar_wait_warp(&sm.k_full[s], (uint32_t)(j / kStages) & 1u, err, abort))) break;
-                if (j >= 1 && !(ok = mbar_wait_warp(&sm.o_done, (uint32_t)(j - 1) & 1u, err, abort))) break;
+                if (j >= 1 && !(ok = mbar_wait_warp(&sm.s_free, (uint32_t)(j - 1) & 1u, err, abort))) break;
                 tc_fence_after();
                 const uint32_t k_addr = smem_u32(sm.k[s]);
 #pragma unroll
@@ -167,6 +154,22 @@ __global__ void __launch_bounds__(kThreads, 2)
                              smem_desc(k_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
                 mma_commit_e(&sm.s_full);
                 mma_commit_e(&sm.k_empty[s]);
+            }
+            if (j >= 1) {
+                // O += P_{j-1} V_{j-1}, P read from TMEM.
+                const int jj = j - 1;
+                const int s = jj % kStages;
+                if (!(ok = mbar_wait_warp(&sm.p_full, (uint32_t)jj & 1u, err, abort))) break;
+                if (!(ok = mbar_wait_warp(&sm.v_full[s], (uint32_t)(jj / kStages) & 1u, err, abort))) break;
+                tc_fence_after();
+                const uint32_t v_addr = smem_u32(sm.v[s]);
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_ts_e(tO, tP + kk * 8,
+                             smem_desc(v_addr + kk * 16 * kRowBytes, kBN * kRowBytes, kAtom, kSwz),
+                             idO, (jj > 0 || kk > 0) ? 1u : 0u);
+                mma_commit_e(&sm.o_done);  // PV_{j-1} complete: O stable, P region free
+                mma_commit_e(&sm.v_empty[s]);
             }
         }
         // All MMAs this warp issued are complete once `drain` fires.
@@ -197,6 +200,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 reg_fence32(r1);
                 reg_fence32(r2);
                 reg_fence32(r3);
+                tc_fence_before();
+                mbar_arrive(&sm.s_free);  // S_j is in registers: S_{j+1} may overwrite it
 #pragma unroll
                 for (int x = 0; x < 32; ++x) {
                     s[x] = __uint_as_float(r0[x]);
@@ -227,12 +232,14 @@ __global__ void __launch_bounds__(kThreads, 2)
             // scale by exactly 1).  A row's arithmetic thus depends on its own
             // scores alone.
             const bool need = mxs > m_used + kRescaleThreshold;
+            bool pv_done = (j == 0);  // PV_{j-1} complete: O stable and the P region free
             if (__any_sync(0xffffffffu, need)) {
                 const float m_new = need ? mxs : m_used;
                 const float alpha = ex2(m_used - m_new);
                 if (j > 0) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done, (uint32_t)(j - 1) & 1u, err, abort));
+                    ok = mbar_wait_warp(&sm.o_done, (uint32_t)(j - 1) & 1u, err, abort);
                     if (!ok) break;
+                    pv_done = true;
                     tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < D; c += 16) {
@@ -259,8 +266,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                     l += p0 + p1;
                     pk[x] = pack_bf16x2(p0, p1);
                 }
-                tmem_st16(tS + lane_off + c / 2, pk);
+                if (c == 0 && !pv_done) {  // P_{j-1} must be consumed before P_j lands
+                    ok = mbar_wait_warp(&sm.o_done, (uint32_t)(j - 1) & 1u, err, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                tmem_st16(tP + lane_off + c / 2, pk);
             }
+            if (!ok) break;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full);
