@@ -233,7 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idS = idesc_bf16(kBT, kBT, 0, 0);  // S^T, dP^T: both K-major
         constexpr uint32_t idKV = idesc_bf16(kBT, D, 0, 1);   // dV, dK: A K-major/TMEM, B MN-major
         constexpr uint32_t idQ = idesc_bf16(kBT, D, 1, 1);    // dQ: A (dS) and B (K) MN-major
-        const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+        // K and V as K-major operands (S^T, dP^T) and K as the MN-major B of dQ.
+        const uint64_t kd_k = smem_desc(smem_u32(sm.k), 16, kAtom, kSwz);
+        const uint64_t vd_k = smem_desc(smem_u32(sm.v), 16, kAtom, kSwz);
+        const uint64_t kd_mn = smem_desc(smem_u32(sm.k), kBT * kRowBytes, kAtom, kSwz);
         bool ok = mbar_wait_warp(&sm.kv_full, 0, err, abort);
         for (int idx = 0; ok && idx <= n_q; ++idx) {
             if (idx < n_q) {
@@ -241,46 +244,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(idx / kQStages) & 1u, err, abort))) break;
                 if (idx >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(idx - 1) & 1u, err, abort))) break;
                 tc_fence_after();
-                const uint32_t q_addr = smem_u32(sm.q[st]), do_addr = smem_u32(sm.dO[st]);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss_e(tS, smem_desc(k_addr + kk * 32, 16, kAtom, kSwz),
-                             smem_desc(q_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss_e(tdP, smem_desc(v_addr + kk * 32, 16, kAtom, kSwz),
-                             smem_desc(do_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
+                // S^T = K Q^T and dP^T = V dO^T: D / 16 MMAs each, all operands
+                // K-major (32 bytes per step).
+                const uint64_t qd = smem_desc(smem_u32(sm.q[st]), 16, kAtom, kSwz);
+                const uint64_t dod = smem_desc(smem_u32(sm.dO[st]), 16, kAtom, kSwz);
+                if constexpr (D == 64) {
+                    mma_ss_x4<2, 2>(tS, kd_k, qd, idS, 0u);
+                    mma_ss_x4<2, 2>(tdP, vd_k, dod, idS, 0u);
+                } else {
+                    mma_ss_x2<2, 2>(tS, kd_k, qd, idS, 0u);
+                    mma_ss_x2<2, 2>(tdP, vd_k, dod, idS, 0u);
+                }
                 mma_commit_e(&sm.sdp_full);
             }
             if (idx >= 1) {
                 const int p = idx - 1;  // the tile whose gradients are now issued
                 const int st = p % kQStages, b = p & 1;
-                const uint32_t q_addr = smem_u32(sm.q[st]), do_addr = smem_u32(sm.dO[st]);
+                // MN-major views (16 rows = kRowBytes 16-byte units per K step).
+                const uint64_t qd_mn = smem_desc(smem_u32(sm.q[st]), kBT * kRowBytes, kAtom, kSwz);
+                const uint64_t dod_mn = smem_desc(smem_u32(sm.dO[st]), kBT * kRowBytes, kAtom, kSwz);
                 const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
+                // dS^T read K-major for dK (32 bytes per step within a 64-query
+                // half, the second half kHalf further) and MN-major for dQ (16 key
+                // rows of 128 bytes per step, the two query halves kHalf apart).
+                const uint64_t dsd_k = smem_desc(ds_addr, 16, 1024, kSwizzle128B);
+                const uint64_t dsd_mn = smem_desc(ds_addr, kHalf, 1024, kSwizzle128B);
                 if (!(ok = mbar_wait_warp(&sm.p_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < kBT / 16; ++s)  // dV += P^T dO, K = 16 queries per step
-                    mma_ts_e(tdV, tP + s * 8,
-                             smem_desc(do_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
-                             idKV, (p > 0 || s > 0) ? 1u : 0u);
+                // dV += P^T dO: 8 MMAs of K = 16 queries, A from TMEM.
+                mma_ts_x4<kRowBytes>(tdV, tP, dod_mn, idKV, p > 0 ? 1u : 0u);
+                mma_ts_x4<kRowBytes>(tdV, tP + 32, dod_mn + 4 * kRowBytes, idKV, 1u);
                 mma_commit_e(&sm.p_free);
                 if (!(ok = mbar_wait_warp(&sm.ds_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < kBT / 16; ++s)  // dK += dS^T Q
-                    mma_ss_e(tdK,
-                             smem_desc(ds_addr + (s >> 2) * kHalf + (s & 3) * 32, 16, 1024, kSwizzle128B),
-                             smem_desc(q_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
-                             idKV, (p > 0 || s > 0) ? 1u : 0u);
+                // dK += dS^T Q: 8 MMAs of K = 16 queries.
+                mma_ss_x4<2, kRowBytes>(tdK, dsd_k, qd_mn, idKV, p > 0 ? 1u : 0u);
+                mma_ss_x4<2, kRowBytes>(tdK, dsd_k + (kHalf >> 4), qd_mn + 4 * kRowBytes, idKV, 1u);
                 mma_commit_e(&sm.qdo_empty[st]);  // Q, dO, lse, Delta of this tile are consumed
                 if (p >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(p - 1) & 1u, err, abort))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < kBT / 16; ++s)  // dQ_i = dS K, K = 16 keys per step
-                    mma_ss_e(tdQ, smem_desc(ds_addr + s * 16 * 128, kHalf, 1024, kSwizzle128B),
-                             smem_desc(k_addr + s * 16 * kRowBytes, kBT * kRowBytes, kAtom, kSwz),
-                             idQ, s > 0 ? 1u : 0u);
+                // dQ_i = dS K: 8 MMAs of K = 16 keys, both operands MN-major.
+                mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn, kd_mn, idQ, 0u);
+                mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn + 4 * 128, kd_mn + 4 * kRowBytes, idQ, 1u);
                 mma_commit_e(&sm.dq_full);
                 mma_commit_e(&sm.ds_free[b]);
             }

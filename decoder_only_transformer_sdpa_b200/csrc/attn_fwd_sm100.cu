@@ -7,17 +7,23 @@
 // the value aggregation; section "Self-Attention: the mathematical trick"
 // [55:20] for the -inf upper triangle and the softmax).
 //
-// One CTA per (128-row query tile, head); heaviest tiles (most key tiles
-// under the causal mask) are launched first.  Two CTAs share an SM (256 TMEM
-// columns, ~81 KB shared memory and <= 168 registers each), so one CTA's
-// softmax overlaps the other's MMAs and both keep the exp unit busy.  Six warps:
-//   warp 0      TMA producer: Q once, then K_j / V_j tiles into a 2-stage ring
-//   warp 1      tcgen05 issuer: S_j = Q K_j^T into TMEM, O += P_j V_j with P_j
-//               read from TMEM; owns the TMEM allocation.  S_{j+1} is issued as
-//               soon as the softmax has read S_j, so it overlaps softmax j.
+// Persistent kernel: two CTAs per SM (256 TMEM columns, ~97 KB shared
+// memory and <= 168 registers each), so one CTA's softmax overlaps the other's
+// MMAs and both keep the exp unit busy.  Work items are (128-row query tile,
+// head) pairs ordered heaviest first (most key tiles under the causal mask);
+// CTA c takes items c, 2G-1-c, 2G+c, ... (a snake over rounds of G = grid size
+// items), which balances the causal work as well as greedy longest-first.
+// Barrier phases run on across items, so the next item's Q and K/V tiles
+// stream in and its first S MMA issues while the current item drains.
+// Six warps:
+//   warp 0      TMA producer: Q of each item into a 2-buffer ring, K_j / V_j
+//               tiles into a 2-stage ring
+//   warp 1      tcgen05 issuer: S = Q K_j^T into TMEM, O += P_j V_j with P_j
+//               read from TMEM; owns the TMEM allocation.  S of the next tile
+//               is issued as soon as the softmax has read the current one.
 //   warps 2..5  softmax: one query row per thread (TMEM lane), online max and
 //               sum in registers, P_j written to TMEM as bf16, lazy rescale of
-//               the O accumulator, final O / l and lse.
+//               the O accumulator, final O / l and lse per item.
 // Key tiles wholly above the diagonal are never loaded; only the diagonal
 // tile applies the element mask.  The score matrix never leaves the SM.
 //
@@ -42,16 +48,23 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max gro
 template <int D>
 struct FwdSmem {
     static constexpr int kTileBytes = kBN * D * 2;
-    alignas(1024) __nv_bfloat16 q[kBM * D];
+    alignas(1024) __nv_bfloat16 q[2][kBM * D];
     alignas(1024) __nv_bfloat16 k[kStages][kBN * D];
     alignas(1024) __nv_bfloat16 v[kStages][kBN * D];
-    uint64_t q_full;
+    uint64_t q_full[2], q_empty[2];
     uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
     uint64_t s_full, s_free, p_full;
-    uint64_t o_done, o_final, drain;
+    uint64_t o_done, o_final, o_free, drain;
     uint32_t tmem_slot;
     int abort;
 };
+
+// The n-th work item of CTA c in a grid of G CTAs over W items (snake order),
+// or -1 when the CTA has no n-th item.
+__device__ __forceinline__ int item_of(int c, int n, int G, int W) {
+    const long long w = (long long)n * G + ((n & 1) ? (G - 1 - c) : c);
+    return w < W ? (int)w : -1;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -68,12 +81,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     volatile int *abort = &sm.abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = ntiles - 1 - (int)(blockIdx.x / BH);  // heaviest first
-    const int bh = (int)(blockIdx.x % BH);
-    const int n_kv = qt + 1;
+    const int G = (int)gridDim.x, cta = (int)blockIdx.x;
+    const int W = ntiles * BH;  // work items; item w is query tile ntiles-1-w/BH of head w%BH
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.q_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.q_full[b], 1);
+            mbar_init(&sm.q_empty[b], 1);
+        }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
             mbar_init(&sm.v_full[s], 1);
@@ -85,6 +100,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(&sm.p_full, kBM);
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.o_final, 1);
+        mbar_init(&sm.o_free, kBM);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -107,73 +123,107 @@ __global__ void __launch_bounds__(kThreads, 2)
             prefetch_tensormap(&tv);
         }
         __syncwarp();
-        mbar_arrive_expect_tx_e(&sm.q_full, Smem::kTileBytes);
-        tma_load_3d_e(sm.q, &tq, &sm.q_full, 0, qt * kBM, bh);
-        int issued = 0;
-        for (int j = 0; j < n_kv; ++j) {
-            const int s = j % kStages;
-            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-            if (!mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort)) break;
-            mbar_arrive_expect_tx_e(&sm.k_full[s], Smem::kTileBytes);
-            tma_load_3d_e(sm.k[s], &tk, &sm.k_full[s], 0, j * kBN, bh);
-            if (!mbar_wait_warp(&sm.v_empty[s], ph ^ 1u, err, abort)) {
-                issued = j + 1;  // K_j is in flight
-                mbar_wait_warp(&sm.k_full[s], ph, err, abort);
-                break;
+        int gt = 0;  // key tiles loaded so far (the K/V ring position)
+        int nq = 0;  // Q tiles loaded so far
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            const int w = item_of(cta, n, G, W);
+            if (w < 0) break;
+            const int qt = ntiles - 1 - w / BH, bh = w % BH;
+            const int qb = n & 1;
+            if (!(ok = mbar_wait_warp(&sm.q_empty[qb], (uint32_t)((n >> 1) & 1) ^ 1u, err, abort))) break;
+            mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
+            tma_load_3d_e(sm.q[qb], &tq, &sm.q_full[qb], 0, qt * kBM, bh);
+            nq = n + 1;
+            for (int j = 0; j <= qt; ++j, ++gt) {
+                const int s = gt % kStages;
+                const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
+                if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
+                mbar_arrive_expect_tx_e(&sm.k_full[s], Smem::kTileBytes);
+                tma_load_3d_e(sm.k[s], &tk, &sm.k_full[s], 0, j * kBN, bh);
+                if (!(ok = mbar_wait_warp(&sm.v_empty[s], ph ^ 1u, err, abort))) {
+                    // K of this tile is in flight: let it land before leaving.
+                    for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
+                    break;
+                }
+                mbar_arrive_expect_tx_e(&sm.v_full[s], Smem::kTileBytes);
+                tma_load_3d_e(sm.v[s], &tv, &sm.v_full[s], 0, j * kBN, bh);
             }
-            mbar_arrive_expect_tx_e(&sm.v_full[s], Smem::kTileBytes);
-            tma_load_3d_e(sm.v[s], &tv, &sm.v_full[s], 0, j * kBN, bh);
-            issued = j + 1;
         }
-        // Drain: every load this warp issued has landed before exit.
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
-            const int s = j % kStages;
-            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+        // Drain: the last loads this warp issued have landed before exit (on the
+        // normal path the consumers waited on all of them already).
+        for (int g = (gt > kStages ? gt - kStages : 0); g < gt; ++g) {
+            const int s = g % kStages;
+            const uint32_t ph = (uint32_t)(g / kStages) & 1u;
             for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
             for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.v_full[s], ph); ++i) {}
         }
-        mbar_wait_warp(&sm.q_full, 0, err, abort);
+        for (int n = (nq > 2 ? nq - 2 : 0); n < nq; ++n)
+            for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.q_full[n & 1], (uint32_t)(n >> 1) & 1u); ++i) {}
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (whole warp,
-        // one elected lane issues)
+        // one elected lane issues).  Global tile g runs S_g, then PV_{g-1}: the
+        // S of a tile is in flight while the softmax of the previous one runs,
+        // also across item boundaries.
         constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);  // Q, K both K-major
         constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);    // P from TMEM, V MN-major
-        const uint32_t q_addr = smem_u32(sm.q);
-        bool ok = mbar_wait_warp(&sm.q_full, 0, err, abort);
-        for (int j = 0; ok && j <= n_kv; ++j) {
-            if (j < n_kv) {
-                // S_j = Q K_j^T, once the softmax has read S_{j-1} out of TMEM.
-                const int s = j % kStages;
-                if (!(ok = mbar_wait_warp(&sm.k_full[s], (uint32_t)(j / kStages) & 1u, err, abort))) break;
-                if (j >= 1 && !(ok = mbar_wait_warp(&sm.s_free, (uint32_t)(j - 1) & 1u, err, abort))) break;
+        // The pending PV (of the previous tile): its global index, item, key
+        // tile index within the item and whether it is the item's last.
+        int pv_g = -1, pv_n = 0, pv_j = 0;
+        bool pv_last = false;
+        bool ok = true;
+        auto issue_pv = [&]() -> bool {
+            const int s = pv_g % kStages;
+            if (!mbar_wait_warp(&sm.p_full, (uint32_t)pv_g & 1u, err, abort)) return false;
+            if (!mbar_wait_warp(&sm.v_full[s], (uint32_t)(pv_g / kStages) & 1u, err, abort)) return false;
+            // The first PV of an item overwrites O: the previous item's O must
+            // have been read out by the softmax warps.
+            if (pv_j == 0 && pv_n >= 1 &&
+                !mbar_wait_warp(&sm.o_free, (uint32_t)(pv_n - 1) & 1u, err, abort))
+                return false;
+            tc_fence_after();
+            // 8 MMAs of K = 16 keys: P from TMEM (8 columns per step), V MN-major
+            // (16 rows = kRowBytes 16-byte units per step).
+            const uint64_t vd = smem_desc(smem_u32(sm.v[s]), kBN * kRowBytes, kAtom, kSwz);
+            mma_ts_x4<kRowBytes>(tO, tP, vd, idO, pv_j > 0 ? 1u : 0u);
+            mma_ts_x4<kRowBytes>(tO, tP + 32, vd + 4 * kRowBytes, idO, 1u);
+            mma_commit_e(&sm.o_done);  // PV complete: O stable, P region free
+            mma_commit_e(&sm.v_empty[s]);
+            if (pv_last) mma_commit_e(&sm.o_final);
+            return true;
+        };
+        int gt = 0;
+        for (int n = 0; ok; ++n) {
+            const int w = item_of(cta, n, G, W);
+            if (w < 0) break;
+            const int qt = ntiles - 1 - w / BH;
+            const int qb = n & 1;
+            if (!(ok = mbar_wait_warp(&sm.q_full[qb], (uint32_t)(n >> 1) & 1u, err, abort))) break;
+            const uint64_t qd = smem_desc(smem_u32(sm.q[qb]), 16, kAtom, kSwz);
+            for (int j = 0; j <= qt; ++j, ++gt) {
+                // S_g = Q K_j^T, once the softmax has read S_{g-1} out of TMEM.
+                const int s = gt % kStages;
+                if (!(ok = mbar_wait_warp(&sm.k_full[s], (uint32_t)(gt / kStages) & 1u, err, abort))) break;
+                if (gt >= 1 && !(ok = mbar_wait_warp(&sm.s_free, (uint32_t)(gt - 1) & 1u, err, abort))) break;
                 tc_fence_after();
-                const uint32_t k_addr = smem_u32(sm.k[s]);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss_e(tS, smem_desc(q_addr + kk * 32, 16, kAtom, kSwz),
-                             smem_desc(k_addr + kk * 32, 16, kAtom, kSwz), idS, kk > 0);
+                // D / 16 MMAs of K = 16: Q and K both K-major (32 bytes per step).
+                const uint64_t kd = smem_desc(smem_u32(sm.k[s]), 16, kAtom, kSwz);
+                if constexpr (D == 64)
+                    mma_ss_x4<2, 2>(tS, qd, kd, idS, 0u);
+                else
+                    mma_ss_x2<2, 2>(tS, qd, kd, idS, 0u);
                 mma_commit_e(&sm.s_full);
                 mma_commit_e(&sm.k_empty[s]);
-            }
-            if (j >= 1) {
-                // O += P_{j-1} V_{j-1}, P read from TMEM.
-                const int jj = j - 1;
-                const int s = jj % kStages;
-                if (!(ok = mbar_wait_warp(&sm.p_full, (uint32_t)jj & 1u, err, abort))) break;
-                if (!(ok = mbar_wait_warp(&sm.v_full[s], (uint32_t)(jj / kStages) & 1u, err, abort))) break;
-                tc_fence_after();
-                const uint32_t v_addr = smem_u32(sm.v[s]);
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts_e(tO, tP + kk * 8,
-                             smem_desc(v_addr + kk * 16 * kRowBytes, kBN * kRowBytes, kAtom, kSwz),
-                             idO, (jj > 0 || kk > 0) ? 1u : 0u);
-                mma_commit_e(&sm.o_done);  // PV_{j-1} complete: O stable, P region free
-                mma_commit_e(&sm.v_empty[s]);
+                if (j == qt) mma_commit_e(&sm.q_empty[qb]);  // this item's Q no longer read
+                if (pv_g >= 0 && !(ok = issue_pv())) break;
+                pv_g = gt;
+                pv_n = n;
+                pv_j = j;
+                pv_last = (j == qt);
             }
         }
+        if (ok && pv_g >= 0) ok = issue_pv();
         // All MMAs this warp issued are complete once `drain` fires.
-        mma_commit_e(&sm.o_final);
         mma_commit_e(&sm.drain);
         mbar_wait_warp(&sm.drain, 0, err, abort);
     } else {
@@ -181,129 +231,141 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
         const int row = quad * 32 + lane;          // row within the query tile
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        float m_used = -INFINITY, l = 0.f;
+        int gt = 0;  // global key-tile counter (barrier phases)
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            ok = mbar_wait_warp(&sm.s_full, (uint32_t)j & 1u, err, abort);
-            if (!ok) break;
-            tc_fence_after();
-            float s[kBN];
-            {
-                // All four 32-column loads in flight before one wait.
-                uint32_t r0[32], r1[32], r2[32], r3[32];
-                tmem_ld32(tS + lane_off + 0, r0);
-                tmem_ld32(tS + lane_off + 32, r1);
-                tmem_ld32(tS + lane_off + 64, r2);
-                tmem_ld32(tS + lane_off + 96, r3);
-                tmem_wait_ld();
-                reg_fence32(r0);
-                reg_fence32(r1);
-                reg_fence32(r2);
-                reg_fence32(r3);
-                tc_fence_before();
-                mbar_arrive(&sm.s_free);  // S_j is in registers: S_{j+1} may overwrite it
+        for (int n = 0; ok; ++n) {
+            const int w = item_of(cta, n, G, W);
+            if (w < 0) break;
+            const int qt = ntiles - 1 - w / BH, bh = w % BH;
+            float m_used = -INFINITY, l = 0.f;
+            for (int j = 0; j <= qt; ++j, ++gt) {
+                ok = mbar_wait_warp(&sm.s_full, (uint32_t)gt & 1u, err, abort);
+                if (!ok) break;
+                tc_fence_after();
+                float s[kBN];
+                {
+                    // All four 32-column loads in flight before one wait.
+                    uint32_t r0[32], r1[32], r2[32], r3[32];
+                    tmem_ld32(tS + lane_off + 0, r0);
+                    tmem_ld32(tS + lane_off + 32, r1);
+                    tmem_ld32(tS + lane_off + 64, r2);
+                    tmem_ld32(tS + lane_off + 96, r3);
+                    tmem_wait_ld();
+                    reg_fence32(r0);
+                    reg_fence32(r1);
+                    reg_fence32(r2);
+                    reg_fence32(r3);
+                    tc_fence_before();
+                    mbar_arrive(&sm.s_free);  // S is in registers: the next S may overwrite it
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    s[x] = __uint_as_float(r0[x]);
-                    s[32 + x] = __uint_as_float(r1[x]);
-                    s[64 + x] = __uint_as_float(r2[x]);
-                    s[96 + x] = __uint_as_float(r3[x]);
-                }
-            }
-            if (j == n_kv - 1) {  // diagonal tile: key column c is visible to row r iff c <= r
-#pragma unroll
-                for (int c = 0; c < kBN; ++c)
-                    if (c > row) s[c] = -INFINITY;
-            }
-            // Row max as eight independent chains (short dependency depth).
-            float mc[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) mc[x] = s[x];
-#pragma unroll
-            for (int c = 8; c < kBN; c += 8)
-#pragma unroll
-                for (int x = 0; x < 8; ++x) mc[x] = fmaxf(mc[x], s[c + x]);
-            const float mx = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
-                                   fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
-            const float mxs = mx * scale_log2;
-            // Each row moves its own running max only when its scores exceed
-            // it by more than the threshold; the warp merely decides whether
-            // the TMEM round trip of O is needed (rows that keep their max
-            // scale by exactly 1).  A row's arithmetic thus depends on its own
-            // scores alone.
-            const bool need = mxs > m_used + kRescaleThreshold;
-            bool pv_done = (j == 0);  // PV_{j-1} complete: O stable and the P region free
-            if (__any_sync(0xffffffffu, need)) {
-                const float m_new = need ? mxs : m_used;
-                const float alpha = ex2(m_used - m_new);
-                if (j > 0) {
-                    ok = mbar_wait_warp(&sm.o_done, (uint32_t)(j - 1) & 1u, err, abort);
-                    if (!ok) break;
-                    pv_done = true;
-                    tc_fence_after();
-#pragma unroll
-                    for (int c = 0; c < D; c += 16) {
-                        uint32_t r[16];
-                        tmem_ld16(tO + lane_off + c, r);
-                        tmem_wait_ld();
-                        reg_fence16(r);
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-                        tmem_st16(tO + lane_off + c, r);
+                    for (int x = 0; x < 32; ++x) {
+                        s[x] = __uint_as_float(r0[x]);
+                        s[32 + x] = __uint_as_float(r1[x]);
+                        s[64 + x] = __uint_as_float(r2[x]);
+                        s[96 + x] = __uint_as_float(r3[x]);
                     }
                 }
-                l *= alpha;
-                m_used = m_new;
-            }
-            const float neg_m = -m_used;
+                if (j == qt) {  // diagonal tile: key column c is visible to row r iff c <= r
 #pragma unroll
-            for (int c = 0; c < kBN; c += 32) {
-                uint32_t pk[16];
+                    for (int c = 0; c < kBN; ++c)
+                        if (c > row) s[c] = -INFINITY;
+                }
+                // Row max as eight independent chains (short dependency depth).
+                float mc[8];
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const float p0 = ex2(fmaf(s[c + 2 * x], scale_log2, neg_m));
-                    const float p1 = ex2(fmaf(s[c + 2 * x + 1], scale_log2, neg_m));
-                    l += p0 + p1;
-                    pk[x] = pack_bf16x2(p0, p1);
+                for (int x = 0; x < 8; ++x) mc[x] = s[x];
+#pragma unroll
+                for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) mc[x] = fmaxf(mc[x], s[c + x]);
+                const float mx = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
+                                       fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
+                const float mxs = mx * scale_log2;
+                // Each row moves its own running max only when its scores exceed
+                // it by more than the threshold; the warp merely decides whether
+                // the TMEM round trip of O is needed (rows that keep their max
+                // scale by exactly 1).  A row's arithmetic thus depends on its
+                // own scores alone.
+                const bool need = mxs > m_used + kRescaleThreshold;
+                bool pv_done = (gt == 0);  // the previous PV is complete: O stable, P free
+                if (__any_sync(0xffffffffu, need)) {
+                    const float m_new = need ? mxs : m_used;
+                    const float alpha = ex2(m_used - m_new);
+                    if (j > 0) {
+                        ok = mbar_wait_warp(&sm.o_done, (uint32_t)(gt - 1) & 1u, err, abort);
+                        if (!ok) break;
+                        pv_done = true;
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < D; c += 16) {
+                            uint32_t r[16];
+                            tmem_ld16(tO + lane_off + c, r);
+                            tmem_wait_ld();
+                            reg_fence16(r);
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+                            tmem_st16(tO + lane_off + c, r);
+                        }
+                    }
+                    l *= alpha;
+                    m_used = m_new;
                 }
-                if (c == 0 && !pv_done) {  // P_{j-1} must be consumed before P_j lands
-                    ok = mbar_wait_warp(&sm.o_done, (uint32_t)(j - 1) & 1u, err, abort);
-                    if (!ok) break;
-                    tc_fence_after();
+                const float neg_m = -m_used;
+#pragma unroll
+                for (int c = 0; c < kBN; c += 32) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        const float p0 = ex2(fmaf(s[c + 2 * x], scale_log2, neg_m));
+                        const float p1 = ex2(fmaf(s[c + 2 * x + 1], scale_log2, neg_m));
+                        l += p0 + p1;
+                        pk[x] = pack_bf16x2(p0, p1);
+                    }
+                    if (c == 0 && !pv_done) {  // the previous P must be consumed first
+                        ok = mbar_wait_warp(&sm.o_done, (uint32_t)(gt - 1) & 1u, err, abort);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    tmem_st16(tP + lane_off + c / 2, pk);
                 }
-                tmem_st16(tP + lane_off + c / 2, pk);
+                if (!ok) break;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.p_full);
             }
             if (!ok) break;
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.p_full);
-        }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, 0, err, abort));
-        if (ok) {
+            // ---- epilogue of the item: O / l and lse; O's TMEM is released as
+            // soon as it is in registers so the next item's PV can start.
+            ok = mbar_wait_warp(&sm.o_final, (uint32_t)n & 1u, err, abort);
+            if (!ok) break;
             tc_fence_after();
-            const int t = qt * kBM + row;
-            const float inv = 1.f / l;
-            const size_t grow = (size_t)bh * T + t;
+            uint32_t r[D / 32][32];
 #pragma unroll
-            for (int c = 0; c < D; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tO + lane_off + c, r);
-                tmem_wait_ld();
-                reg_fence32(r);
-                if (t < T) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(o + grow * D + c);
+            for (int h = 0; h < D / 32; ++h) tmem_ld32(tO + lane_off + 32 * h, r[h]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < D / 32; ++h) reg_fence32(r[h]);
+            tc_fence_before();
+            mbar_arrive(&sm.o_free);
+            const int t = qt * kBM + row;
+            if (t < T) {
+                const float inv = 1.f / l;
+                const size_t grow = (size_t)bh * T + t;
+#pragma unroll
+                for (int h = 0; h < D / 32; ++h) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(o + grow * D + 32 * h);
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * inv, __uint_as_float(r[8 * x + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv, __uint_as_float(r[8 * x + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv, __uint_as_float(r[8 * x + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv, __uint_as_float(r[8 * x + 7]) * inv);
-                        dst[x] = w;
+                        uint4 w4;
+                        w4.x = pack_bf16x2(__uint_as_float(r[h][8 * x + 0]) * inv, __uint_as_float(r[h][8 * x + 1]) * inv);
+                        w4.y = pack_bf16x2(__uint_as_float(r[h][8 * x + 2]) * inv, __uint_as_float(r[h][8 * x + 3]) * inv);
+                        w4.z = pack_bf16x2(__uint_as_float(r[h][8 * x + 4]) * inv, __uint_as_float(r[h][8 * x + 5]) * inv);
+                        w4.w = pack_bf16x2(__uint_as_float(r[h][8 * x + 6]) * inv, __uint_as_float(r[h][8 * x + 7]) * inv);
+                        dst[x] = w4;
                     }
                 }
+                lse[grow] = (m_used + log2f(l)) * 0.69314718055994531f;
             }
-            if (t < T) lse[grow] = (m_used + log2f(l)) * 0.69314718055994531f;
         }
     }
 
@@ -337,8 +399,14 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
                        LaunchInfo &li) {
     const int BH = s.B * s.H;
     const int ntiles = (s.T + kBM - 1) / kBM;
-    const long long blocks = (long long)ntiles * BH;
-    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const long long items = (long long)ntiles * BH;
+    if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    int dev = 0, sms = 0;
+    cudaError_t e0;
+    if ((e0 = cudaGetDevice(&dev)) != cudaSuccess) return e0;
+    if ((e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e0;
+    // Persistent grid: two CTAs per SM, never more CTAs than work items.
+    const long long grid = items < 2LL * sms ? items : 2LL * sms;
     CUtensorMap mq, mk, mv;
     cudaError_t e;
     if ((e = make_map(&mq, q, BH, s.T, D)) != cudaSuccess) return e;
@@ -350,7 +418,7 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
         return e;
     const float scale_log2 = s.scale * 1.4426950408889634f;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    fwd_kernel<D><<<(unsigned)blocks, kThreads, smem, st>>>(mq, mk, mv, o, lse, s.T, BH, ntiles,
+    fwd_kernel<D><<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, o, lse, s.T, BH, ntiles,
                                                             scale_log2, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;

@@ -292,6 +292,66 @@ __device__ __forceinline__ void mma_ts_e(uint32_t d_tmem, uint32_t a_tmem, uint6
         : "memory");
 }
 
+// Four (or two) MMAs from one asm block with one elect: descriptors advance by
+// compile-time steps (in 16-byte units of the start-address field), the TMEM
+// A operand by 8 columns (16 bf16) per MMA.  Keeping the issuing warp's
+// instruction stream this short is what lets the tensor core run at its
+// measured rate (~32 cycles per 128x64x16 MMA with A in TMEM, ~65 per
+// 128x128x16 with both operands in shared memory); building descriptors per
+// MMA costs more than the MMA itself.  The first MMA accumulates iff `acc`;
+// the rest always accumulate.
+template <int AS, int BS>
+__device__ __forceinline__ void mma_ss_x4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, q, e;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 q, 0, 0;\n\t"
+        "add.s64 a1, %1, %5;\n\tadd.s64 a2, %1, %6;\n\tadd.s64 a3, %1, %7;\n\t"
+        "add.s64 b1, %2, %8;\n\tadd.s64 b2, %2, %9;\n\tadd.s64 b3, %2, %10;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, q;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "n"(AS), "n"(2 * AS), "n"(3 * AS), "n"(BS),
+        "n"(2 * BS), "n"(3 * BS)
+        : "memory");
+}
+
+template <int AS, int BS>
+__device__ __forceinline__ void mma_ss_x2(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, q, e;\n\t.reg .b64 a1, b1;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 q, 0, 0;\n\t"
+        "add.s64 a1, %1, %5;\n\tadd.s64 b1, %2, %6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, q;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "n"(AS), "n"(BS)
+        : "memory");
+}
+
+template <int BS>
+__device__ __forceinline__ void mma_ts_x4(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                          uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, q, e;\n\t.reg .b32 a1, a2, a3;\n\t.reg .b64 b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 q, 0, 0;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+        "add.s64 b1, %2, %5;\n\tadd.s64 b2, %2, %6;\n\tadd.s64 b3, %2, %7;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, q;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "n"(BS), "n"(2 * BS), "n"(3 * BS)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_commit_e(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
