@@ -311,24 +311,28 @@ __global__ void __launch_bounds__(kThreads, 2)
                     m_used = m_new;
                 }
                 const float neg_m = -m_used;
+                // All exponentials first (packed bf16 pairs), then wait for the
+                // previous PV to release the P region: the wait sits at the end
+                // of the tile, where the previous PV has had the most time.
+                uint32_t pk[kBN / 2];
+                float la = 0.f, lb = 0.f;
 #pragma unroll
-                for (int c = 0; c < kBN; c += 32) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const float p0 = ex2(fmaf(s[c + 2 * x], scale_log2, neg_m));
-                        const float p1 = ex2(fmaf(s[c + 2 * x + 1], scale_log2, neg_m));
-                        l += p0 + p1;
-                        pk[x] = pack_bf16x2(p0, p1);
-                    }
-                    if (c == 0 && !pv_done) {  // the previous P must be consumed first
-                        ok = mbar_wait_warp(&sm.o_done, (uint32_t)(gt - 1) & 1u, err, abort);
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
-                    tmem_st16(tP + lane_off + c / 2, pk);
+                for (int x = 0; x < kBN / 2; ++x) {
+                    const float p0 = ex2(fmaf(s[2 * x], scale_log2, neg_m));
+                    const float p1 = ex2(fmaf(s[2 * x + 1], scale_log2, neg_m));
+                    la += p0;
+                    lb += p1;
+                    pk[x] = pack_bf16x2(p0, p1);
                 }
-                if (!ok) break;
+                l += la + lb;
+                if (!pv_done) {
+                    ok = mbar_wait_warp(&sm.o_done, (uint32_t)(gt - 1) & 1u, err, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int c = 0; c < kBN / 2; c += 16)
+                    tmem_st16(tP + lane_off + c, *reinterpret_cast<uint32_t (*)[16]>(&pk[c]));
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_full);
