@@ -49,6 +49,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=5, help="steps of the host-buffer end-to-end leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-strided", action="store_true",
+                   help="skip the secondary measurement on c_attn-layout (strided) buffers")
     p.add_argument("--layers", type=int, default=None,
                    help="layer instances per step (default: the workload's 12); fewer only for profiling")
     return p.parse_args()
@@ -403,6 +405,44 @@ def run_ours(args, w):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps}
 
+    # ---- secondary: the same step on the layouts nanoGPT's attention sees
+    # (q, k, v slices of a [B, T, 3C] c_attn output; O, dO as [B, T, C];
+    # dq | dk | dv into one [B, T, 3C] buffer), through the strided entry points
+    strided = None
+    if not args.no_strided:
+        H, D = w.H, w.D
+        tm = lambda t: t.permute(0, 2, 1, 3).reshape(w.B, w.T, H * D)
+        pk = []
+        for b in layers:
+            qkv = torch.cat([tm(b["q"]), tm(b["k"]), tm(b["v"])], dim=2).contiguous()
+            dqkv = torch.empty_like(qkv)
+            views = lambda x: [x[:, :, i * H * D:(i + 1) * H * D].view(w.B, w.T, H, D).permute(0, 2, 1, 3)
+                               for i in range(3)]
+            do_p = tm(b["do"]).contiguous().view(w.B, w.T, H, D).permute(0, 2, 1, 3)
+            o_p = A.empty_token_major(w.B, H, w.T, D, dev)
+            pk.append((views(qkv), views(dqkv), do_p, o_p, qkv, dqkv))
+
+        def strided_step():
+            for l, (qv, _, _, o_p, _, _) in enumerate(pk):
+                A.attn_fwd_strided(*qv, o=o_p, lse=layers[l]["lse"])
+            for l in range(L - 1, -1, -1):
+                qv, dv3, do_p, o_p, _, _ = pk[l]
+                A.attn_bwd_strided(*qv, o_p, layers[l]["lse"], do_p, *dv3, workspace=layers[l]["ws"])
+        n_s = max(3, min(args.steps, 50))
+        strided_step()
+        barrier()
+        s0, s1 = mk(), mk()
+        s0.record(stream)
+        for _ in range(n_s):
+            strided_step()
+        s1.record(stream)
+        barrier()
+        st_ms = reduce_max(s0.elapsed_time(s1), world, dev)
+        strided = {"value": whole_job_tflops(flops_step, world, n_s, st_ms), "unit": "TFLOP/s",
+                   "ms_per_step": st_ms / n_s, "steps": n_s,
+                   "layout": "q,k,v slices of [B,T,3C]; O, dO [B,T,C]; dq|dk|dv into [B,T,3C]"}
+        del pk
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.seed)
@@ -417,7 +457,7 @@ def run_ours(args, w):
             "pct_of_peak": {"measured_burst": value / world / peak,
                             "measured_sustained": value / world / float(peaks.get("bf16_tflops_sustained", peak)),
                             "datasheet_2250": value / world / 2250.0},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "strided_io": strided,
             "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

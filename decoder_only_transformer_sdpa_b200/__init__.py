@@ -40,6 +40,16 @@ _lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _
 _lib.attn_bwd.restype = _i
 _lib.attn_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
 _lib.attn_bwd_noalloc.restype = _i
+class attn_strides(ctypes.Structure):
+    """Element strides (batch, head, token) of one [B, H, T, D] operand."""
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("t", ctypes.c_int64)]
+
+
+_sp = ctypes.POINTER(attn_strides)
+_lib.attn_fwd_strided.argtypes = [_vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _f, _sp, _vp]
+_lib.attn_fwd_strided.restype = _i
+_lib.attn_bwd_strided.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _sp, _vp, _sz, _vp]
+_lib.attn_bwd_strided.restype = _i
 _lib.attn_fwd_f32.argtypes = [_fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _vp]
 _lib.attn_fwd_f32.restype = _i
 _lib.attn_bwd_f32_workspace_bytes.argtypes = [_i, _i, _i, _i]
@@ -56,7 +66,8 @@ _lib.attn_profile_next_call.restype = _i
 EXPORTED = ("attn_status_string", "attn_version", "attn_last_launch_count", "attn_fwd",
             "attn_bwd_workspace_bytes", "attn_bwd", "attn_fwd_f32", "attn_bwd_f32_workspace_bytes",
             "attn_bwd_f32", "attn_device_error", "attn_profile_next_call",
-            "attn_selftest_wait_timeout", "attn_bwd_noalloc")
+            "attn_selftest_wait_timeout", "attn_bwd_noalloc", "attn_fwd_strided",
+            "attn_bwd_strided")
 
 
 class AttnError(RuntimeError):
@@ -236,3 +247,75 @@ def attn_selftest_wait_timeout(polls: int = 1024, stream=None) -> None:
     """Enqueue the bounded-wait failure self test (see include/attn.h)."""
     _raise(_lib.attn_selftest_wait_timeout(int(polls), _stream_handle(stream)),
            "attn_selftest_wait_timeout")
+
+
+def _check_view(t, name, shape):
+    """A bf16 CUDA [B, H, T, D] view with unit D stride; returns its pointer."""
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.stride(3) != 1:
+        raise ValueError(f"{name} must have unit stride along D")
+    return t.data_ptr()
+
+
+def _strides_of(*tensors):
+    arr = (attn_strides * len(tensors))()
+    for i, t in enumerate(tensors):
+        arr[i] = attn_strides(t.stride(0), t.stride(1), t.stride(2))
+    return arr
+
+
+def empty_token_major(B: int, H: int, T: int, D: int, device):
+    """A bf16 [B, H, T, D] view of a fresh [B, T, H*D] tensor (the layout the
+    output projection consumes)."""
+    torch = _torch()
+    return torch.empty(B, T, H, D, dtype=torch.bfloat16, device=device).permute(0, 2, 1, 3)
+
+
+def attn_fwd_strided(q, k, v, o=None, lse=None, scale: Optional[float] = None, stream=None):
+    """Forward on strided [B, H, T, D] views (e.g. slices of the c_attn output
+    [B, T, 3C]).  O defaults to a [B, T, C] buffer viewed as [B, H, T, D]."""
+    torch = _torch()
+    B, H, T, D = _shape4(q)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    o = empty_token_major(B, H, T, D, q.device) if o is None else o
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    ptrs = [_check_view(q, "q", q.shape), _check_view(k, "k", q.shape),
+            _check_view(v, "v", q.shape), _check_view(o, "o", q.shape),
+            _check(lse, "lse", torch.float32, (B, H, T))]
+    st = _strides_of(q, k, v, o)
+    with torch.cuda.device(q.device):
+        _raise(_lib.attn_fwd_strided(*ptrs, B, H, T, D, scale, st, _stream_handle(stream)),
+               "attn_fwd_strided")
+    return o, lse
+
+
+def attn_bwd_strided(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[float] = None,
+                     workspace=None, stream=None):
+    """Backward on strided views; dq/dk/dv default to [B, T, C] buffers viewed
+    as [B, H, T, D].  Returns (dQ, dK, dV)."""
+    torch = _torch()
+    B, H, T, D = _shape4(q)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq = empty_token_major(B, H, T, D, q.device) if dq is None else dq
+    dk = empty_token_major(B, H, T, D, q.device) if dk is None else dk
+    dv = empty_token_major(B, H, T, D, q.device) if dv is None else dv
+    need = attn_bwd_workspace_bytes(B, H, T, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ptrs = [_check_view(q, "q", q.shape), _check_view(k, "k", q.shape),
+            _check_view(v, "v", q.shape), _check_view(o, "o", q.shape),
+            _check(lse, "lse", torch.float32, (B, H, T)), _check_view(dO, "dO", q.shape),
+            _check_view(dq, "dq", q.shape), _check_view(dk, "dk", q.shape),
+            _check_view(dv, "dv", q.shape)]
+    st = _strides_of(q, k, v, o, dO, dq, dk, dv)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        _raise(_lib.attn_bwd_strided(*ptrs, B, H, T, D, scale, st, workspace.data_ptr(), ws_bytes,
+                                     _stream_handle(stream)), "attn_bwd_strided")
+    return dq, dk, dv

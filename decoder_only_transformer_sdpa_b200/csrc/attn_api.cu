@@ -124,9 +124,19 @@ ATTN_API int attn_profile_next_call(cudaEvent_t start, cudaEvent_t end) {
 
 ATTN_API int attn_last_launch_count(void) { return t_last_launches; }
 
-ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
-                      int H, int T, int D, float scale, cudaStream_t stream) {
-    LaunchInfo li = take_launch_info();
+namespace {
+
+// A [B,H,T,D] bf16 view is usable by TMA when its batch, head and token
+// strides are positive multiples of 8 elements (16 bytes) below 2^39.
+bool strides_ok(const attn_strides &x) {
+    auto ok = [](int64_t v) { return v > 0 && v % 8 == 0 && v < (1ll << 39); };
+    return ok(x.b) && ok(x.h) && ok(x.t);
+}
+
+TStrides to_tstrides(const attn_strides &x) { return TStrides{x.b, x.h, x.t}; }
+
+int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int T,
+             int D, float scale, const FwdStrides &str, cudaStream_t stream, LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 64);
     if (st != ATTN_OK) return st;
@@ -138,20 +148,14 @@ ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, floa
     if ((st = device_setup(&err)) != ATTN_OK) return st;
     cudaError_t e = sm100_fwd(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
                               static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), lse,
-                              Shape{B, H, T, D, scale}, err, stream, li);
+                              Shape{B, H, T, D, scale}, str, err, stream, li);
     return finish(e, li);
 }
 
-// Workspace of the bf16 backward: dQ float32 accumulator, padded lse, Delta.
-ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
-    if (check_shape(B, H, T, D, 64) != ATTN_OK || !bf16_d_supported(D)) return 0;
-    return bwd_workspace_layout(B, H, T, D).total;
-}
-
-ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
-                      const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D,
-                      float scale, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    LaunchInfo li = take_launch_info();
+int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D, float scale,
+             const BwdStrides &str, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+             LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 64);
     if (st != ATTN_OK) return st;
@@ -175,8 +179,59 @@ ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o
         static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(o), lse,
         static_cast<const __nv_bfloat16 *>(dO), static_cast<__nv_bfloat16 *>(dq),
         static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv), dq_acc, lse2, delta,
-        Shape{B, H, T, D, scale}, err, stream, li);
+        Shape{B, H, T, D, scale}, str, err, stream, li);
     return finish(e, li);
+}
+
+}  // namespace
+
+ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                      int H, int T, int D, float scale, cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    const TStrides c = contiguous_strides(Shape{B, H, T, D, scale});
+    return fwd_impl(q, k, v, o, lse, B, H, T, D, scale, FwdStrides{c, c, c, c}, stream, li);
+}
+
+ATTN_API int attn_fwd_strided(const void *q, const void *k, const void *v, void *o, float *lse,
+                              int B, int H, int T, int D, float scale, const attn_strides *strides,
+                              cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    if (!strides) return ATTN_ERR_NULL;
+    for (int i = 0; i < 4; ++i)
+        if (!strides_ok(strides[i])) return ATTN_ERR_ALIGN;
+    const FwdStrides str{to_tstrides(strides[0]), to_tstrides(strides[1]), to_tstrides(strides[2]),
+                         to_tstrides(strides[3])};
+    return fwd_impl(q, k, v, o, lse, B, H, T, D, scale, str, stream, li);
+}
+
+// Workspace of the bf16 backward: dQ float32 accumulator, padded lse, Delta.
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
+    if (check_shape(B, H, T, D, 64) != ATTN_OK || !bf16_d_supported(D)) return 0;
+    return bwd_workspace_layout(B, H, T, D).total;
+}
+
+ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                      const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D,
+                      float scale, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    const TStrides c = contiguous_strides(Shape{B, H, T, D, scale});
+    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale,
+                    BwdStrides{c, c, c, c, c, c, c, c}, workspace, workspace_bytes, stream, li);
+}
+
+ATTN_API int attn_bwd_strided(const void *q, const void *k, const void *v, const void *o,
+                              const float *lse, const void *dO, void *dq, void *dk, void *dv, int B,
+                              int H, int T, int D, float scale, const attn_strides *strides,
+                              void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    if (!strides) return ATTN_ERR_NULL;
+    for (int i = 0; i < 8; ++i)
+        if (!strides_ok(strides[i])) return ATTN_ERR_ALIGN;
+    BwdStrides str;
+    TStrides *dst[8] = {&str.q, &str.k, &str.v, &str.o, &str.dO, &str.dq, &str.dk, &str.dv};
+    for (int i = 0; i < 8; ++i) *dst[i] = to_tstrides(strides[i]);
+    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, str, workspace,
+                    workspace_bytes, stream, li);
 }
 
 ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,

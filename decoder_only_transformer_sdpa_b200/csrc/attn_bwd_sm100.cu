@@ -91,7 +91,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
                                                        float *__restrict__ lse2,
                                                        float *__restrict__ delta,
                                                        float *__restrict__ dq_acc, int T, int Tpad,
-                                                       long long prows) {
+                                                       long long prows, int H, TStrides so,
+                                                       TStrides sdo) {
     constexpr int kTpr = D / 8;  // threads per row (a power of two dividing 32)
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long prow = gid / kTpr;
@@ -103,8 +104,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
     const size_t row = (size_t)bh * T + t;
     float acc = 0.f;
     if (live) {
-        const uint4 a = reinterpret_cast<const uint4 *>(o + row * D)[c];
-        const uint4 g = reinterpret_cast<const uint4 *>(dO + row * D)[c];
+        const long long hb = bh / H, hh = bh % H;
+        const uint4 a = reinterpret_cast<const uint4 *>(o + hb * so.b + hh * so.h + (long long)t * so.t)[c];
+        const uint4 g = reinterpret_cast<const uint4 *>(dO + hb * sdo.b + hh * sdo.h + (long long)t * sdo.t)[c];
         const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
         const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&g);
 #pragma unroll
@@ -128,18 +130,23 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
 // ------------------------------------------------------------------ post
 
 // dQ = scale * accumulator, 8 elements per thread (two 16-byte loads, one
-// 16-byte store).
-__global__ void bwd_post_kernel(const float4 *__restrict__ acc, uint4 *__restrict__ dq, long long n8,
-                                float scale) {
+// 16-byte store into the strided dQ view).
+__global__ void bwd_post_kernel(const float4 *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
+                                long long n8, float scale, int T, int H, int D, TStrides sdq) {
+    const int cpr = D / 8;  // 8-element chunks per row
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
          i += (long long)gridDim.x * blockDim.x) {
+        const long long row = i / cpr;
+        const int c = (int)(i - row * cpr);
+        const long long bh = row / T;
+        const long long t = row - bh * T;
         const float4 a = acc[2 * i], b = acc[2 * i + 1];
         uint4 r;
         r.x = pack_bf16x2(a.x * scale, a.y * scale);
         r.y = pack_bf16x2(a.z * scale, a.w * scale);
         r.z = pack_bf16x2(b.x * scale, b.y * scale);
         r.w = pack_bf16x2(b.z * scale, b.w * scale);
-        dq[i] = r;
+        *reinterpret_cast<uint4 *>(dq + (bh / H) * sdq.b + (bh % H) * sdq.h + t * sdq.t + 8 * c) = r;
     }
 }
 
@@ -151,8 +158,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                     const __grid_constant__ CUtensorMap tdq, const float *__restrict__ lse2,
                     const float *__restrict__ delta, __nv_bfloat16 *__restrict__ dk,
-                    __nv_bfloat16 *__restrict__ dv, int T, int Tpad, int BH, int nt,
-                    float scale_log2, float scale, int *err) {
+                    __nv_bfloat16 *__restrict__ dv, const TStrides sdk, const TStrides sdv,
+                    int T, int Tpad, int H, int BH, int nt, float scale_log2, float scale,
+                    int *err) {
     using Smem = BwdSmem<D>;
     constexpr int kRowBytes = D * 2;
     constexpr uint32_t kSwz = (D == 64) ? kSwizzle128B : kSwizzle64B;
@@ -166,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kt = (int)(blockIdx.x / BH);  // key tile; tile 0 sees the most query tiles
     const int bh = (int)(blockIdx.x % BH);
+    const int hh = bh % H, bb = bh / H;
     const int n_q = nt - kt;                // query tiles kt .. nt-1
 
     if (threadIdx.x == 0) {
@@ -209,16 +218,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         mbar_arrive_expect_tx_e(&sm.kv_full, 2 * Smem::kTileBytes);
-        tma_load_3d_e(sm.k, &tk, &sm.kv_full, 0, kt * kBT, bh);
-        tma_load_3d_e(sm.v, &tv, &sm.kv_full, 0, kt * kBT, bh);
+        tma_load_4d_e(sm.k, &tk, &sm.kv_full, 0, kt * kBT, hh, bb);
+        tma_load_4d_e(sm.v, &tv, &sm.kv_full, 0, kt * kBT, hh, bb);
         int issued = 0;
         for (int idx = 0; idx < n_q; ++idx) {
             const int st = idx % kQStages;
             const int i = kt + idx;
             if (!mbar_wait_warp(&sm.qdo_empty[st], (uint32_t)((idx / kQStages) & 1) ^ 1u, err, abort)) break;
             mbar_arrive_expect_tx_e(&sm.qdo_full[st], 2 * Smem::kTileBytes + 2 * kBT * 4);
-            tma_load_3d_e(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, bh);
-            tma_load_3d_e(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, bh);
+            tma_load_4d_e(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, hh, bb);
+            tma_load_4d_e(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, hh, bb);
             const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
             bulk_load_e(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
             bulk_load_e(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
@@ -372,10 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             tc_fence_after();
             const int t = kt * kBT + kr;
-            const size_t grow = (size_t)bh * T + t;
             const uint32_t src = half == 0 ? tdK : tdV;
             const float mul = half == 0 ? scale : 1.f;
-            __nv_bfloat16 *out = half == 0 ? dk : dv;
+            const TStrides so = half == 0 ? sdk : sdv;
+            __nv_bfloat16 *out = (half == 0 ? dk : dv) + (long long)bb * so.b + (long long)hh * so.h +
+                                 (long long)t * so.t;
 #pragma unroll
             for (int c = 0; c < D; c += 32) {
                 uint32_t r[32];
@@ -383,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
                 reg_fence32(r);
                 if (t < T) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + grow * D + c);
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + c);
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
                         uint4 w4;
@@ -465,8 +475,8 @@ template <int D>
 cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                        const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                        __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
-                       float *lse2, float *delta, Shape s, int *err, cudaStream_t st,
-                       LaunchInfo &li) {
+                       float *lse2, float *delta, Shape s, const BwdStrides &str, int *err,
+                       cudaStream_t st, LaunchInfo &li) {
     const int BH = s.B * s.H;
     const int nt = (s.T + kBT - 1) / kBT;
     const int Tpad = nt * kBT;
@@ -474,16 +484,16 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     CUtensorMap mq, mk, mv, mdo, mdq;
     cudaError_t e;
-    if ((e = make_map(&mq, q, BH, s.T, D, false, D)) != cudaSuccess) return e;
-    if ((e = make_map(&mk, k, BH, s.T, D, false, D)) != cudaSuccess) return e;
-    if ((e = make_map(&mv, v, BH, s.T, D, false, D)) != cudaSuccess) return e;
-    if ((e = make_map(&mdo, dO, BH, s.T, D, false, D)) != cudaSuccess) return e;
+    if ((e = make_map_bf16(&mq, q, s, str.q)) != cudaSuccess) return e;
+    if ((e = make_map_bf16(&mk, k, s, str.k)) != cudaSuccess) return e;
+    if ((e = make_map_bf16(&mv, v, s, str.v)) != cudaSuccess) return e;
+    if ((e = make_map_bf16(&mdo, dO, s, str.dO)) != cudaSuccess) return e;
     if ((e = make_map(&mdq, dq_acc, BH, s.T, D, true, 32)) != cudaSuccess) return e;
 
     const long long prows = (long long)BH * Tpad;
     const long long prep_threads = prows * (D / 8);
     bwd_prep_kernel<D><<<(unsigned)((prep_threads + 255) / 256), 256, 0, st>>>(
-        o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows);
+        o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows, s.H, str.o, str.dO);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
 
@@ -493,7 +503,8 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
         return e;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     bwd_main_kernel<D><<<(unsigned)blocks, kThreads, smem, st>>>(
-        mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, s.T, Tpad, BH, nt, s.scale * kLog2e, s.scale, err);
+        mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, str.dk, str.dv, s.T, Tpad, s.H, BH, nt,
+        s.scale * kLog2e, s.scale, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
     if ((e = mark_main_end(li, st)) != cudaSuccess) return e;
@@ -501,8 +512,8 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     const long long n8 = (long long)BH * s.T * D / 8;
     const long long want = (n8 + 255) / 256;
     const int post_blocks = (int)(want < 148 * 16 ? want : 148 * 16);
-    bwd_post_kernel<<<post_blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc),
-                                                  reinterpret_cast<uint4 *>(dq), n8, s.scale);
+    bwd_post_kernel<<<post_blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc), dq, n8,
+                                                  s.scale, s.T, s.H, D, str.dq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
     return cudaSuccess;
@@ -513,12 +524,12 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
 cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
-                      float *lse2, float *delta, Shape s, int *err, cudaStream_t st,
-                      LaunchInfo &li) {
+                      float *lse2, float *delta, Shape s, const BwdStrides &str, int *err,
+                      cudaStream_t st, LaunchInfo &li) {
     if (s.D == 64)
-        return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, err, st, li);
+        return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, str, err, st, li);
     if (s.D == 32)
-        return launch_bwd<32>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, err, st, li);
+        return launch_bwd<32>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, str, err, st, li);
     return cudaErrorInvalidValue;
 }
 

@@ -70,7 +70,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16 *__restrict__ o,
-               float *__restrict__ lse, int T, int BH, int ntiles, float scale_log2, int *err) {
+               const TStrides so, float *__restrict__ lse, int T, int H, int BH, int ntiles,
+               float scale_log2, int *err) {
     using Smem = FwdSmem<D>;
     constexpr int kRowBytes = D * 2;                      // 128 (D=64) or 64 (D=32)
     constexpr uint32_t kSwz = (D == 64) ? kSwizzle128B : kSwizzle64B;
@@ -130,24 +131,25 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int w = item_of(cta, n, G, W);
             if (w < 0) break;
             const int qt = ntiles - 1 - w / BH, bh = w % BH;
+            const int hh = bh % H, bb = bh / H;
             const int qb = n & 1;
             if (!(ok = mbar_wait_warp(&sm.q_empty[qb], (uint32_t)((n >> 1) & 1) ^ 1u, err, abort))) break;
             mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
-            tma_load_3d_e(sm.q[qb], &tq, &sm.q_full[qb], 0, qt * kBM, bh);
+            tma_load_4d_e(sm.q[qb], &tq, &sm.q_full[qb], 0, qt * kBM, hh, bb);
             nq = n + 1;
             for (int j = 0; j <= qt; ++j, ++gt) {
                 const int s = gt % kStages;
                 const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
                 if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
                 mbar_arrive_expect_tx_e(&sm.k_full[s], Smem::kTileBytes);
-                tma_load_3d_e(sm.k[s], &tk, &sm.k_full[s], 0, j * kBN, bh);
+                tma_load_4d_e(sm.k[s], &tk, &sm.k_full[s], 0, j * kBN, hh, bb);
                 if (!(ok = mbar_wait_warp(&sm.v_empty[s], ph ^ 1u, err, abort))) {
                     // K of this tile is in flight: let it land before leaving.
                     for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
                     break;
                 }
                 mbar_arrive_expect_tx_e(&sm.v_full[s], Smem::kTileBytes);
-                tma_load_3d_e(sm.v[s], &tv, &sm.v_full[s], 0, j * kBN, bh);
+                tma_load_4d_e(sm.v[s], &tv, &sm.v_full[s], 0, j * kBN, hh, bb);
             }
         }
         // Drain: the last loads this warp issued have landed before exit (on the
@@ -355,9 +357,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (t < T) {
                 const float inv = 1.f / l;
                 const size_t grow = (size_t)bh * T + t;
+                __nv_bfloat16 *orow = o + (long long)(bh / H) * so.b + (long long)(bh % H) * so.h +
+                                      (long long)t * so.t;
 #pragma unroll
                 for (int h = 0; h < D / 32; ++h) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(o + grow * D + 32 * h);
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * h);
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
                         uint4 w4;
@@ -382,25 +386,29 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-// Encodes a [BH, T, D] bf16 tensor as a 3-D TMA map with 128-row boxes.
-cudaError_t make_map(CUtensorMap *map, const void *ptr, int BH, int T, int D) {
+}  // namespace
+
+cudaError_t make_map_bf16(void *map, const void *ptr, const Shape &s, const TStrides &st) {
     auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
     if (!enc) return cudaErrorInitializationError;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)D, 128, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
-                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+    const cuuint64_t dims[4] = {(cuuint64_t)s.D, (cuuint64_t)s.T, (cuuint64_t)s.H, (cuuint64_t)s.B};
+    const cuuint64_t strides[3] = {(cuuint64_t)st.t * 2, (cuuint64_t)st.h * 2, (cuuint64_t)st.b * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)s.D, 128, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = enc(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                           const_cast<void *>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           s.D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+namespace {
+
 template <int D>
 cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                       __nv_bfloat16 *o, float *lse, Shape s, int *err, cudaStream_t st,
-                       LaunchInfo &li) {
+                       __nv_bfloat16 *o, float *lse, Shape s, const FwdStrides &str, int *err,
+                       cudaStream_t st, LaunchInfo &li) {
     const int BH = s.B * s.H;
     const int ntiles = (s.T + kBM - 1) / kBM;
     const long long items = (long long)ntiles * BH;
@@ -413,16 +421,16 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     const long long grid = items < 2LL * sms ? items : 2LL * sms;
     CUtensorMap mq, mk, mv;
     cudaError_t e;
-    if ((e = make_map(&mq, q, BH, s.T, D)) != cudaSuccess) return e;
-    if ((e = make_map(&mk, k, BH, s.T, D)) != cudaSuccess) return e;
-    if ((e = make_map(&mv, v, BH, s.T, D)) != cudaSuccess) return e;
+    if ((e = make_map_bf16(&mq, q, s, str.q)) != cudaSuccess) return e;
+    if ((e = make_map_bf16(&mk, k, s, str.k)) != cudaSuccess) return e;
+    if ((e = make_map_bf16(&mv, v, s, str.v)) != cudaSuccess) return e;
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
     if ((e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
     const float scale_log2 = s.scale * 1.4426950408889634f;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    fwd_kernel<D><<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, o, lse, s.T, BH, ntiles,
+    fwd_kernel<D><<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, o, str.o, lse, s.T, s.H, BH, ntiles,
                                                             scale_log2, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
@@ -432,10 +440,10 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
 }  // namespace
 
 cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                      __nv_bfloat16 *o, float *lse, Shape s, int *err, cudaStream_t st,
-                      LaunchInfo &li) {
-    if (s.D == 64) return launch_fwd<64>(q, k, v, o, lse, s, err, st, li);
-    if (s.D == 32) return launch_fwd<32>(q, k, v, o, lse, s, err, st, li);
+                      __nv_bfloat16 *o, float *lse, Shape s, const FwdStrides &str, int *err,
+                      cudaStream_t st, LaunchInfo &li) {
+    if (s.D == 64) return launch_fwd<64>(q, k, v, o, lse, s, str, err, st, li);
+    if (s.D == 32) return launch_fwd<32>(q, k, v, o, lse, s, str, err, st, li);
     return cudaErrorInvalidValue;
 }
 

@@ -22,6 +22,27 @@ struct Shape {
     float scale;
 };
 
+// Element strides of a [B, H, T, D] view (the d stride is 1).  Contiguous
+// tensors have {H*T*D, T*D, D}; q/k/v viewed inside a [B, T, 3*H*D] c_attn
+// output have {T*3*H*D, D, 3*H*D}.
+struct TStrides {
+    long long b, h, t;
+};
+inline TStrides contiguous_strides(const Shape &s) {
+    return TStrides{(long long)s.H * s.T * s.D, (long long)s.T * s.D, (long long)s.D};
+}
+struct FwdStrides {
+    TStrides q, k, v, o;
+};
+struct BwdStrides {
+    TStrides q, k, v, o, dO, dq, dk, dv;
+};
+
+// Builds a 4-D TMA map over a bf16 [B, H, T, D] view with the given element
+// strides: dimensions (D, T, H, B), box (D, 128, 1, 1), swizzle matching a
+// D * 2-byte row (128 B at D = 64, 64 B at D = 32).
+cudaError_t make_map_bf16(void *map, const void *ptr, const Shape &s, const TStrides &st);
+
 // Per-call bookkeeping: kernels enqueued, and the optional event pair to
 // record around the call's main kernel (see attn_profile_next_call).
 struct LaunchInfo {
@@ -49,13 +70,13 @@ cudaError_t simt_bwd(const T *q, const T *k, const T *v, const T *o, const float
 
 // ---- tcgen05 / TMA kernels for bf16, D in {32, 64}
 cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                      __nv_bfloat16 *o, float *lse, Shape s, int *err, cudaStream_t st,
-                      LaunchInfo &li);
+                      __nv_bfloat16 *o, float *lse, Shape s, const FwdStrides &str, int *err,
+                      cudaStream_t st, LaunchInfo &li);
 cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv,
-                      float *dq_acc, float *lse2, float *delta, Shape s, int *err, cudaStream_t st,
-                      LaunchInfo &li);
+                      float *dq_acc, float *lse2, float *delta, Shape s, const BwdStrides &str,
+                      int *err, cudaStream_t st, LaunchInfo &li);
 
 // Workspace layout of the bf16 backward (offsets in bytes, each 256-aligned):
 // float32 dQ accumulator [B*H*T*D], then log2-scaled lse and Delta, each

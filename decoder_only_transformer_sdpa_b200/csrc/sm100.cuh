@@ -381,6 +381,18 @@ __device__ __forceinline__ void tma_load_3d_e(void *dst, const CUtensorMap *map,
         : "memory");
 }
 
+// 4-D tile load (d, token, head, batch coordinates) issued by one elected lane.
+__device__ __forceinline__ void tma_load_4d_e(void *dst, const CUtensorMap *map, uint64_t *bar, int c0,
+                                              int c1, int c2, int c3) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];\n\t}" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_load_e(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"

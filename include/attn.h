@@ -115,6 +115,38 @@ int attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
                      const float *lse, const void *dO, void *dq, void *dk, void *dv,
                      int B, int H, int T, int D, float scale, cudaStream_t stream);
 
+/* ---------------- bf16 path on strided views --------------------------- */
+
+/* Element strides of one [B, H, T, D] operand: from one batch to the next, one
+ * head to the next and one token to the next; the D stride is 1.  A
+ * contiguous tensor has {H*T*D, T*D, D}.  In nanoGPT's CausalSelfAttention
+ * ("nanoGPT — 架构与原理", section 7 code map, and the component table of
+ * section 2.2) q, k and v are slices of one c_attn projection [B, T, 3*H*D]
+ * and the attention output feeds c_proj as [B, T, H*D]; with strides the
+ * kernels read and write those layouts directly, with no transposes:
+ *   q: {T*3*H*D, D, 3*H*D} at offset 0, k: the same at offset H*D, v at 2*H*D;
+ *   o: {T*H*D, D, H*D}. */
+typedef struct {
+    int64_t b, h, t;
+} attn_strides;
+
+/* attn_fwd on strided views.  strides[0..3] describe q, k, v, o.  Every
+ * stride must be a positive multiple of 8 elements (16 bytes), else
+ * ATTN_ERR_ALIGN; NULL strides give ATTN_ERR_NULL.  lse stays [B, H, T]
+ * contiguous.  Output rows must not overlap one another.  Other rules as
+ * attn_fwd. */
+int attn_fwd_strided(const void *q, const void *k, const void *v, void *o, float *lse,
+                     int B, int H, int T, int D, float scale, const attn_strides *strides,
+                     cudaStream_t stream);
+
+/* attn_bwd on strided views.  strides[0..7] describe q, k, v, o, dO, dq, dk,
+ * dv (dq/dk/dv may be slices of one [B, T, 3*H*D] buffer for the c_attn
+ * backward).  Same stride rules as attn_fwd_strided; workspace as attn_bwd. */
+int attn_bwd_strided(const void *q, const void *k, const void *v, const void *o,
+                     const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                     int B, int H, int T, int D, float scale, const attn_strides *strides,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* ---------------- float32 path: CUDA cores, IEEE expf -------------------- */
 
 /* Forward in float32 (all tensors float32).  1 <= D <= 128. */

@@ -120,3 +120,29 @@ def test_bwd_f32_workspace_error():
 def test_selftest_argument_errors():
     assert lib_mod.lib().attn_selftest_wait_timeout(0, None) == E_SHAPE
     assert lib_mod.lib().attn_selftest_wait_timeout((1 << 22) + 1, None) == E_SHAPE
+
+
+def _strides(n, b=1 << 16, h=64, t=1 << 10):
+    import ctypes
+    arr = (lib_mod.attn_strides * n)()
+    for i in range(n):
+        arr[i] = lib_mod.attn_strides(b, h, t)
+    return arr
+
+
+@pytest.mark.parametrize("bad", [dict(t=0), dict(h=-8), dict(b=12), dict(t=3), dict(t=1 << 40)])
+def test_strided_argument_errors(bad):
+    lib = lib_mod.lib()
+    good = _strides(8)
+    assert lib.attn_fwd_strided(P, P, P, P, P, 1, 1, 8, 64, 0.125, None, None) == E_NULL
+    assert lib.attn_bwd_strided(*([P] * 9), 1, 1, 8, 64, 0.125, None, P, 1 << 30, None) == E_NULL
+    for i in range(4):
+        st = _strides(4)
+        st[i] = lib_mod.attn_strides(**{**dict(b=1 << 16, h=64, t=1 << 10), **bad})
+        assert lib.attn_fwd_strided(P, P, P, P, P, 1, 1, 8, 64, 0.125, st, None) == E_ALIGN
+    for i in range(8):
+        st = _strides(8)
+        st[i] = lib_mod.attn_strides(**{**dict(b=1 << 16, h=64, t=1 << 10), **bad})
+        assert lib.attn_bwd_strided(*([P] * 9), 1, 1, 8, 64, 0.125, st, P, 1 << 30, None) == E_ALIGN
+    # valid strides still hit the ordinary checks first-class (unsupported D)
+    assert lib.attn_fwd_strided(P, P, P, P, P, 1, 1, 8, 48, 0.125, good, None) == E_D

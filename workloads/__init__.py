@@ -137,6 +137,25 @@ def make_inputs(w: Workload, seed: int = 0, layer: int = 0,
             (("q", q), ("k", k), ("v", v), ("do", do))}
 
 
+def make_inputs_packed(w: Workload, seed: int = 0, layer: int = 0) -> Dict[str, torch.Tensor]:
+    """The same values as make_inputs, laid out the way nanoGPT's attention
+    sees them: "qkv" [B, T, 3C] (the c_attn output, q | k | v along the last
+    dim) and "do_packed" [B, T, C] (the gradient arriving from c_proj), next to
+    make_inputs' contiguous [B, H, T, D] "q", "k", "v", "do"."""
+    inp = make_inputs(w, seed=seed, layer=layer)
+    tm = lambda t: t.permute(0, 2, 1, 3).reshape(t.shape[0], t.shape[2], -1)
+    qkv = torch.cat([tm(inp["q"]), tm(inp["k"]), tm(inp["v"])], dim=2).contiguous()
+    return {**inp, "qkv": qkv, "do_packed": tm(inp["do"]).contiguous()}
+
+
+def packed_views(qkv: torch.Tensor, H: int):
+    """[B, H, T, D] views of q, k, v inside a [B, T, 3C] tensor."""
+    B, T, C3 = qkv.shape
+    C = C3 // 3
+    D = C // H
+    return [qkv[:, :, i * C:(i + 1) * C].view(B, T, H, D).permute(0, 2, 1, 3) for i in range(3)]
+
+
 def random_qkv(seed: int, B: int, H: int, T: int, D: int, dtype=torch.float32,
                std: float = 1.0, do_std: float = 1.0) -> Dict[str, torch.Tensor]:
     """Plain i.i.d. normal inputs of any shape (edge cases, ragged tails)."""
