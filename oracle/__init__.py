@@ -1,4 +1,5 @@
-"""Double-precision CPU oracle of causal multi-head attention (fwd + bwd).
+"""Double-precision CPU oracle of causal multi-head attention (fwd + bwd), and
+of the same attention without the mask (``causal=False``).
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
 bench's CPU-baseline leg may import this package.  The product path (the CUDA
@@ -42,43 +43,51 @@ class OracleLib:
         lib = ctypes.CDLL(path)
         dp = ctypes.POINTER(ctypes.c_double)
         i = ctypes.c_int
-        lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double]
-        lib.oracle_attn_fwd.restype = None
-        lib.oracle_attn_probs.argtypes = [dp, dp, dp, i, i, i, i, ctypes.c_double]
-        lib.oracle_attn_probs.restype = None
-        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double]
-        lib.oracle_attn_bwd.restype = None
+        for suffix in ("", "_nc"):
+            f = getattr(lib, "oracle_attn_fwd" + suffix)
+            f.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double]
+            f.restype = None
+            f = getattr(lib, "oracle_attn_probs" + suffix)
+            f.argtypes = [dp, dp, dp, i, i, i, i, ctypes.c_double]
+            f.restype = None
+            f = getattr(lib, "oracle_attn_bwd" + suffix)
+            f.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double]
+            f.restype = None
         lib.oracle_threads.argtypes = []
         lib.oracle_threads.restype = i
         self.lib = lib
 
-    def attn_fwd(self, q, k, v, scale=None):
+    def _fn(self, name: str, causal: bool):
+        return getattr(self.lib, name if causal else name + "_nc")
+
+    def attn_fwd(self, q, k, v, scale=None, causal=True):
         """Returns (O [B,H,T,D], lse [B,H,T]) in float64."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, H, T, D = _shape(q)
         scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
         o = np.empty_like(q)
         lse = np.empty((B, H, T), dtype=np.float64)
-        self.lib.oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D, scale)
+        self._fn("oracle_attn_fwd", causal)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                            B, H, T, D, scale)
         return o, lse
 
-    def attn_probs(self, q, k, scale=None):
-        """The causal softmax matrices P [B,H,T,T] (zero above the diagonal)."""
+    def attn_probs(self, q, k, scale=None, causal=True):
+        """The softmax matrices P [B,H,T,T] (zero above the diagonal if causal)."""
         q, k = _f64(q), _f64(k)
         B, H, T, D = _shape(q)
         scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
         p = np.empty((B, H, T, T), dtype=np.float64)
-        self.lib.oracle_attn_probs(_ptr(q), _ptr(k), _ptr(p), B, H, T, D, scale)
+        self._fn("oracle_attn_probs", causal)(_ptr(q), _ptr(k), _ptr(p), B, H, T, D, scale)
         return p
 
-    def attn_bwd(self, q, k, v, do, scale=None):
+    def attn_bwd(self, q, k, v, do, scale=None, causal=True):
         """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
         q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
         B, H, T, D = _shape(q)
         scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
         dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
-        self.lib.oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
-                                 B, H, T, D, scale)
+        self._fn("oracle_attn_bwd", causal)(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq),
+                                            _ptr(dk), _ptr(dv), B, H, T, D, scale)
         return dq, dk, dv
 
     def threads_used(self) -> int:
@@ -111,19 +120,19 @@ def _shape(q: np.ndarray):
     return tuple(int(s) for s in q.shape)
 
 
-def attn_fwd(q, k, v, scale=None):
+def attn_fwd(q, k, v, scale=None, causal=True):
     """Returns (O [B,H,T,D], lse [B,H,T]) in float64."""
-    return _load().attn_fwd(q, k, v, scale)
+    return _load().attn_fwd(q, k, v, scale, causal)
 
 
-def attn_probs(q, k, scale=None):
-    """The causal softmax matrices P [B,H,T,T] (zero above the diagonal)."""
-    return _load().attn_probs(q, k, scale)
+def attn_probs(q, k, scale=None, causal=True):
+    """The softmax matrices P [B,H,T,T] (zero above the diagonal if causal)."""
+    return _load().attn_probs(q, k, scale, causal)
 
 
-def attn_bwd(q, k, v, do, scale=None):
+def attn_bwd(q, k, v, do, scale=None, causal=True):
     """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
-    return _load().attn_bwd(q, k, v, do, scale)
+    return _load().attn_bwd(q, k, v, do, scale, causal)
 
 
 def threads_used() -> int:

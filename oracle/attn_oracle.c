@@ -36,6 +36,12 @@
  *   dQ_i  = scale * sum_{j<=i} dS_ij k_j
  *   dK_j  = scale * sum_{i>=j} dS_ij q_i
  *
+ * Non-causal variant (the "_nc" entry points): the same computation with no
+ * mask, every query attending to all T keys -- the encoder-style attention the
+ * pages contrast with the decoder's masked one when they introduce the -inf
+ * upper triangle ([55:20]); the backward is the same derivative with sums over
+ * all i and j.
+ *
  * Layout: every tensor is [B, H, T, D] contiguous float64; lse is [B, H, T].
  * No blocking, no fusion, no reordering beyond the definition.  The softmax
  * subtracts the row maximum before exponentiating, which changes nothing in
@@ -49,11 +55,13 @@
 #include <omp.h>
 #endif
 
-/* Row i of the causal softmax of one head: fills p[0..i] (p[j>i] untouched),
- * returns lse_i.  q_i is one query row, kh the head's keys. */
-static double causal_softmax_row(const double *qi, const double *kh, int i, int D,
-                                 double scale, double *p)
+/* Row i of the softmax of one head over keys 0..last (last = i when causal,
+ * T - 1 otherwise): fills p[0..last] (later entries untouched), returns lse_i.
+ * q_i is one query row, kh the head's keys. */
+static double softmax_row(const double *qi, const double *kh, int last, int D, double scale,
+                          double *p)
 {
+    const int i = last;
     double m = -INFINITY;
     for (int j = 0; j <= i; ++j) {
         double s = 0.0;
@@ -76,9 +84,16 @@ static int num_threads_used = 1;
 /* Number of OpenMP threads the last call ran on. */
 int oracle_threads(void) { return num_threads_used; }
 
+/* Last key row i attends to: itself when causal, the final token otherwise. */
+static int last_key(int i, int T, int causal) { return causal ? i : T - 1; }
+
+/* First query row that attends to key j: j itself when causal, else row 0. */
+static int first_query(int j, int causal) { return causal ? j : 0; }
+
 /* Forward: o [B,H,T,D], lse [B,H,T] (lse may be NULL). */
-void oracle_attn_fwd(const double *q, const double *k, const double *v,
-                     double *o, double *lse, int B, int H, int T, int D, double scale)
+static void attn_fwd(const double *q, const double *k, const double *v,
+                     double *o, double *lse, int B, int H, int T, int D, double scale,
+                     int causal)
 {
     const int64_t heads = (int64_t)B * H;
     const int64_t hs = (int64_t)T * D;
@@ -94,11 +109,12 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v,
             const double *qh = q + bh * hs, *kh = k + bh * hs, *vh = v + bh * hs;
             double *oh = o + bh * hs;
             for (int i = 0; i < T; ++i) {
-                double li = causal_softmax_row(qh + (int64_t)i * D, kh, i, D, scale, p);
+                const int last = last_key(i, T, causal);
+                double li = softmax_row(qh + (int64_t)i * D, kh, last, D, scale, p);
                 if (lse) lse[bh * T + i] = li;
                 for (int d = 0; d < D; ++d) {
                     double acc = 0.0;
-                    for (int j = 0; j <= i; ++j) acc += p[j] * vh[(int64_t)j * D + d];
+                    for (int j = 0; j <= last; ++j) acc += p[j] * vh[(int64_t)j * D + d];
                     oh[(int64_t)i * D + d] = acc;
                 }
             }
@@ -107,9 +123,10 @@ void oracle_attn_fwd(const double *q, const double *k, const double *v,
     }
 }
 
-/* The full probability matrices P [B,H,T,T] (zeros above the diagonal). */
-void oracle_attn_probs(const double *q, const double *k, double *p,
-                       int B, int H, int T, int D, double scale)
+/* The full probability matrices P [B,H,T,T] (zeros above the diagonal when
+ * causal). */
+static void attn_probs(const double *q, const double *k, double *p,
+                       int B, int H, int T, int D, double scale, int causal)
 {
     const int64_t heads = (int64_t)B * H;
     const int64_t hs = (int64_t)T * D;
@@ -118,16 +135,16 @@ void oracle_attn_probs(const double *q, const double *k, double *p,
         double *ph = p + bh * (int64_t)T * T;
         memset(ph, 0, sizeof(double) * (size_t)T * (size_t)T);
         for (int i = 0; i < T; ++i)
-            causal_softmax_row(q + bh * hs + (int64_t)i * D, k + bh * hs, i, D, scale,
-                               ph + (int64_t)i * T);
+            softmax_row(q + bh * hs + (int64_t)i * D, k + bh * hs, last_key(i, T, causal), D,
+                        scale, ph + (int64_t)i * T);
     }
 }
 
 /* Backward: dq, dk, dv [B,H,T,D] from q, k, v and the upstream gradient dO.
  * The forward (P, O) is recomputed here from q, k, v in double. */
-void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
+static void attn_bwd(const double *q, const double *k, const double *v, const double *dO,
                      double *dq, double *dk, double *dv,
-                     int B, int H, int T, int D, double scale)
+                     int B, int H, int T, int D, double scale, int causal)
 {
     const int64_t heads = (int64_t)B * H;
     const int64_t hs = (int64_t)T * D;
@@ -150,42 +167,43 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
             memset(dS, 0, sizeof(double) * tt);
             /* forward recompute: P and O */
             for (int i = 0; i < T; ++i) {
-                causal_softmax_row(qh + (int64_t)i * D, kh, i, D, scale, P + (int64_t)i * T);
+                const int last = last_key(i, T, causal);
+                softmax_row(qh + (int64_t)i * D, kh, last, D, scale, P + (int64_t)i * T);
                 for (int d = 0; d < D; ++d) {
                     double acc = 0.0;
-                    for (int j = 0; j <= i; ++j) acc += P[(int64_t)i * T + j] * vh[(int64_t)j * D + d];
+                    for (int j = 0; j <= last; ++j) acc += P[(int64_t)i * T + j] * vh[(int64_t)j * D + d];
                     O[(int64_t)i * D + d] = acc;
                 }
             }
-            /* dV_j = sum_{i>=j} P_ij dO_i */
+            /* dV_j = sum_{i>=j} P_ij dO_i (all i when not causal) */
             for (int j = 0; j < T; ++j)
                 for (int d = 0; d < D; ++d) {
                     double acc = 0.0;
-                    for (int i = j; i < T; ++i) acc += P[(int64_t)i * T + j] * gh[(int64_t)i * D + d];
+                    for (int i = first_query(j, causal); i < T; ++i) acc += P[(int64_t)i * T + j] * gh[(int64_t)i * D + d];
                     dvh[(int64_t)j * D + d] = acc;
                 }
             /* dS_ij = P_ij (dP_ij - Delta_i), dP_ij = <dO_i, v_j>, Delta_i = <dO_i, O_i> */
             for (int i = 0; i < T; ++i) {
                 double delta = 0.0;
                 for (int d = 0; d < D; ++d) delta += gh[(int64_t)i * D + d] * O[(int64_t)i * D + d];
-                for (int j = 0; j <= i; ++j) {
+                for (int j = 0; j <= last_key(i, T, causal); ++j) {
                     double dp = 0.0;
                     for (int d = 0; d < D; ++d) dp += gh[(int64_t)i * D + d] * vh[(int64_t)j * D + d];
                     dS[(int64_t)i * T + j] = P[(int64_t)i * T + j] * (dp - delta);
                 }
             }
-            /* dQ_i = scale * sum_{j<=i} dS_ij k_j */
+            /* dQ_i = scale * sum_{j<=i} dS_ij k_j (all j when not causal) */
             for (int i = 0; i < T; ++i)
                 for (int d = 0; d < D; ++d) {
                     double acc = 0.0;
-                    for (int j = 0; j <= i; ++j) acc += dS[(int64_t)i * T + j] * kh[(int64_t)j * D + d];
+                    for (int j = 0; j <= last_key(i, T, causal); ++j) acc += dS[(int64_t)i * T + j] * kh[(int64_t)j * D + d];
                     dqh[(int64_t)i * D + d] = scale * acc;
                 }
-            /* dK_j = scale * sum_{i>=j} dS_ij q_i */
+            /* dK_j = scale * sum_{i>=j} dS_ij q_i (all i when not causal) */
             for (int j = 0; j < T; ++j)
                 for (int d = 0; d < D; ++d) {
                     double acc = 0.0;
-                    for (int i = j; i < T; ++i) acc += dS[(int64_t)i * T + j] * qh[(int64_t)i * D + d];
+                    for (int i = first_query(j, causal); i < T; ++i) acc += dS[(int64_t)i * T + j] * qh[(int64_t)i * D + d];
                     dkh[(int64_t)j * D + d] = scale * acc;
                 }
         }
@@ -193,4 +211,43 @@ void oracle_attn_bwd(const double *q, const double *k, const double *v, const do
         free(dS);
         free(O);
     }
+}
+
+/* Exported entry points: the causal attention of the decoder, and the same
+ * computation without the mask ("_nc"). */
+void oracle_attn_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
+                     int B, int H, int T, int D, double scale)
+{
+    attn_fwd(q, k, v, o, lse, B, H, T, D, scale, 1);
+}
+
+void oracle_attn_fwd_nc(const double *q, const double *k, const double *v, double *o,
+                        double *lse, int B, int H, int T, int D, double scale)
+{
+    attn_fwd(q, k, v, o, lse, B, H, T, D, scale, 0);
+}
+
+void oracle_attn_probs(const double *q, const double *k, double *p, int B, int H, int T, int D,
+                       double scale)
+{
+    attn_probs(q, k, p, B, H, T, D, scale, 1);
+}
+
+void oracle_attn_probs_nc(const double *q, const double *k, double *p, int B, int H, int T,
+                          int D, double scale)
+{
+    attn_probs(q, k, p, B, H, T, D, scale, 0);
+}
+
+void oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
+                     double *dq, double *dk, double *dv, int B, int H, int T, int D, double scale)
+{
+    attn_bwd(q, k, v, dO, dq, dk, dv, B, H, T, D, scale, 1);
+}
+
+void oracle_attn_bwd_nc(const double *q, const double *k, const double *v, const double *dO,
+                        double *dq, double *dk, double *dv, int B, int H, int T, int D,
+                        double scale)
+{
+    attn_bwd(q, k, v, dO, dq, dk, dv, B, H, T, D, scale, 0);
 }

@@ -23,6 +23,14 @@ What pins what:
 * torch's float64 CPU ``scaled_dot_product_attention(is_causal=True)`` and its
   autograd, a library routine used as an independent witness;
 * small hand-derived golden examples under tests/golden/.
+
+The non-causal variant (``causal=False``: no -inf triangle, every token sees
+every token) has pins of its own: rows of P sum to 1 with every entry positive;
+Q = 0 gives the mean of all values and lse = ln T; relabelling the tokens by a
+permutation relabels every output the same way (nothing depends on position);
+its last row equals the causal last row (both see all T keys); shift
+invariance, finite differences, torch's ``is_causal=False`` witness and a
+hand-derived golden example.
 """
 from __future__ import annotations
 
@@ -186,15 +194,149 @@ def check_golden(impl):
             g = json.load(f)
         arr = lambda key: np.asarray(g[key], dtype=np.float64)[None, None]
         q, k, v = arr("q"), arr("k"), arr("v")
-        o, lse = impl.attn_fwd(q, k, v, g.get("scale"))
+        causal = g.get("causal", True)
+        o, lse = impl.attn_fwd(q, k, v, g.get("scale"), causal=causal)
         np.testing.assert_allclose(o[0, 0], np.asarray(g["o"]), rtol=0, atol=g["atol"], err_msg=name)
         np.testing.assert_allclose(lse[0, 0], np.asarray(g["lse"]), rtol=0, atol=g["atol"], err_msg=name)
         if "do" in g:
-            dq, dk, dv = impl.attn_bwd(q, k, v, arr("do"), g.get("scale"))
+            dq, dk, dv = impl.attn_bwd(q, k, v, arr("do"), g.get("scale"), causal=causal)
             for key, got in (("dq", dq), ("dk", dk), ("dv", dv)):
                 np.testing.assert_allclose(got[0, 0], np.asarray(g[key]), rtol=0, atol=g["atol"],
                                            err_msg=f"{name}:{key}")
 
 
+def check_nc_probs_rows(impl, seed=11):
+    r = _rng(seed)
+    B, H, T, D = 2, 3, 17, 5
+    q, k = r.standard_normal((B, H, T, D)), r.standard_normal((B, H, T, D)) * 3.0
+    p = impl.attn_probs(q, k, causal=False)
+    assert np.all(np.abs(p.sum(-1) - 1.0) <= 1e-14), "rows of P must sum to 1"
+    assert np.all(p > 0.0), "without the mask every key gets a positive weight"
+
+
+def check_nc_averaging(impl, seed=12):
+    """Q = 0 (then K = 0) without the mask: uniform weights 1/T over all keys."""
+    r = _rng(seed)
+    B, H, T, D = 2, 2, 11, 6
+    k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(3))
+    scale = 1.0 / math.sqrt(D)
+    mean = np.broadcast_to(v.mean(axis=2, keepdims=True), v.shape)
+    zero = np.zeros_like(k)
+    o, lse = impl.attn_fwd(zero, k, v, causal=False)
+    np.testing.assert_allclose(o, mean, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, np.full(lse.shape, math.log(T)), rtol=0, atol=1e-14)
+    dq, dk, dv = impl.attn_bwd(zero, k, v, do, causal=False)
+    dv_ref = np.broadcast_to(do.sum(axis=2, keepdims=True) / T, dv.shape)
+    np.testing.assert_allclose(dv, dv_ref, rtol=0, atol=1e-13)
+    assert np.all(dk == 0.0), "Q = 0 must give dK = 0 exactly"
+    g = np.einsum("bhid,bhjd->bhij", do, v)
+    delta = np.einsum("bhid,bhid->bhi", do, mean)
+    ds = (g - delta[..., None]) / T
+    np.testing.assert_allclose(dq, scale * np.einsum("bhij,bhjd->bhid", ds, k), rtol=0, atol=1e-13)
+    q = r.standard_normal((B, H, T, D))
+    o2, lse2 = impl.attn_fwd(q, zero, v, causal=False)
+    np.testing.assert_allclose(o2, mean, rtol=0, atol=1e-13)
+    dq2, dk2, dv2 = impl.attn_bwd(q, zero, v, do, causal=False)
+    assert np.all(dq2 == 0.0), "K = 0 must give dQ = 0 exactly"
+    np.testing.assert_allclose(dv2, dv_ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk2, scale * np.einsum("bhij,bhid->bhjd", ds, q), rtol=0, atol=1e-13)
+
+
+def check_nc_permutation(impl, seed=13):
+    """Without the mask nothing depends on position: relabelling the tokens by
+    a permutation relabels O, lse, dQ, dK and dV the same way, and permuting
+    only the key/value pairs changes nothing."""
+    r = _rng(seed)
+    B, H, T, D = 1, 2, 10, 4
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    perm = r.permutation(T)
+    o, lse = impl.attn_fwd(q, k, v, causal=False)
+    grads = impl.attn_bwd(q, k, v, do, causal=False)
+    pq, pk, pv, pdo = (a[:, :, perm] for a in (q, k, v, do))
+    o2, lse2 = impl.attn_fwd(pq, pk, pv, causal=False)
+    np.testing.assert_allclose(o2, o[:, :, perm], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse2, lse[:, :, perm], rtol=0, atol=1e-13)
+    for a, b in zip(grads, impl.attn_bwd(pq, pk, pv, pdo, causal=False)):
+        np.testing.assert_allclose(b, a[:, :, perm], rtol=0, atol=1e-13)
+    o3, lse3 = impl.attn_fwd(q, pk, pv, causal=False)
+    np.testing.assert_allclose(o3, o, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse3, lse, rtol=0, atol=1e-13)
+
+
+def check_nc_last_row_and_single_token(impl, seed=14):
+    """The causal last row already sees every key, so both variants agree
+    there; at T = 1 they agree everywhere."""
+    r = _rng(seed)
+    B, H, T, D = 2, 2, 9, 5
+    q, k, v = (r.standard_normal((B, H, T, D)) for _ in range(3))
+    o, lse = impl.attn_fwd(q, k, v)
+    onc, lsenc = impl.attn_fwd(q, k, v, causal=False)
+    np.testing.assert_allclose(onc[:, :, -1], o[:, :, -1], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lsenc[:, :, -1], lse[:, :, -1], rtol=0, atol=1e-14)
+    assert not np.allclose(onc[:, :, 0], o[:, :, 0]), "row 0 must see the later keys"
+    q1, k1, v1, do1 = (r.standard_normal((B, H, 1, D)) for _ in range(4))
+    o1, _ = impl.attn_fwd(q1, k1, v1, causal=False)
+    assert np.array_equal(o1, v1), "T = 1 must return V exactly"
+    assert np.array_equal(impl.attn_bwd(q1, k1, v1, do1, causal=False)[2], do1)
+
+
+def check_nc_shift_invariance(impl, seed=15):
+    r = _rng(seed)
+    B, H, T, D = 2, 2, 9, 5
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    u = 4.0 * r.standard_normal((B, H, 1, D))
+    scale = 1.0 / math.sqrt(D)
+    o, lse = impl.attn_fwd(q, k, v, causal=False)
+    o2, lse2 = impl.attn_fwd(q, k + u, v, causal=False)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse2, lse + scale * np.sum(q * u, -1), rtol=0, atol=1e-12)
+    g, g2 = impl.attn_bwd(q, k, v, do, causal=False), impl.attn_bwd(q, k + u, v, do, causal=False)
+    for a, b in zip(g, g2):
+        np.testing.assert_allclose(b, a, rtol=0, atol=1e-12)
+
+
+def check_nc_finite_differences(impl, seed=16):
+    r = _rng(seed)
+    B, H, T, D = 1, 2, 5, 3
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    dq, dk, dv = impl.attn_bwd(q, k, v, do, causal=False)
+
+    def loss(q_, k_, v_):
+        return float(np.sum(impl.attn_fwd(q_, k_, v_, causal=False)[0] * do))
+
+    h = 1e-6
+    for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+        fd = np.zeros_like(grad)
+        for idx in np.ndindex(*grad.shape):
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[which][idx] += h
+            lp = loss(args["q"], args["k"], args["v"])
+            args[which][idx] -= 2 * h
+            lm = loss(args["q"], args["k"], args["v"])
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.linalg.norm(fd - grad) / max(np.linalg.norm(grad), 1e-300)
+        assert err <= 1e-7, f"d{which}: finite differences disagree (rel {err:.2e})"
+
+
+def check_nc_torch_witness(impl, seed=17):
+    import torch
+    r = _rng(seed)
+    B, H, T, D = 2, 3, 33, 16
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=False)
+    to.backward(torch.tensor(do))
+    o, lse = impl.attn_fwd(q, k, v, causal=False)
+    dq, dk, dv = impl.attn_bwd(q, k, v, do, causal=False)
+    np.testing.assert_allclose(o, to.detach().numpy(), rtol=0, atol=1e-12)
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-12)
+    s = torch.tensor(q) @ torch.tensor(k).transpose(-1, -2) / math.sqrt(D)
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [check_probs_rows, check_averaging_trick, check_causality, check_single_token,
-            check_shift_invariance, check_finite_differences, check_torch_witness, check_golden]
+            check_shift_invariance, check_finite_differences, check_torch_witness, check_golden,
+            check_nc_probs_rows, check_nc_averaging, check_nc_permutation,
+            check_nc_last_row_and_single_token, check_nc_shift_invariance,
+            check_nc_finite_differences, check_nc_torch_witness]

@@ -22,6 +22,9 @@ MUTATIONS = {
     "dq_scale_dropped": ("dqh[(int64_t)i * D + d] = scale * acc;", "dqh[(int64_t)i * D + d] = acc;"),
     "dq_transposed_ds": ("acc += dS[(int64_t)i * T + j] * kh[(int64_t)j * D + d];",
                          "acc += dS[(int64_t)j * T + i] * kh[(int64_t)j * D + d];"),
+    "nc_keeps_mask": ("return causal ? i : T - 1;", "return i;"),
+    "nc_bwd_sums_keep_mask": ("return causal ? j : 0;", "return j;"),
+    "nc_misses_last_key": ("return causal ? i : T - 1;", "return causal ? i : T - 2;"),
 }
 
 
