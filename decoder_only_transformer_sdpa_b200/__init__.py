@@ -50,6 +50,22 @@ _lib.attn_fwd_strided.argtypes = [_vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _f, _
 _lib.attn_fwd_strided.restype = _i
 _lib.attn_bwd_strided.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _sp, _vp, _sz, _vp]
 _lib.attn_bwd_strided.restype = _i
+class attn_options(ctypes.Structure):
+    """Options of the _ex entry points (include/attn.h): the mask."""
+    _fields_ = [("causal", ctypes.c_int32)]
+
+
+_op = ctypes.POINTER(attn_options)
+_lib.attn_fwd_ex.argtypes = [_vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _f, _sp, _op, _vp]
+_lib.attn_fwd_ex.restype = _i
+_lib.attn_bwd_ex.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _sp, _op,
+                             _vp, _sz, _vp]
+_lib.attn_bwd_ex.restype = _i
+_lib.attn_fwd_f32_ex.argtypes = [_fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _op, _vp]
+_lib.attn_fwd_f32_ex.restype = _i
+_lib.attn_bwd_f32_ex.argtypes = [_fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _op,
+                                 _vp, _sz, _vp]
+_lib.attn_bwd_f32_ex.restype = _i
 _lib.attn_fwd_f32.argtypes = [_fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _vp]
 _lib.attn_fwd_f32.restype = _i
 _lib.attn_bwd_f32_workspace_bytes.argtypes = [_i, _i, _i, _i]
@@ -67,7 +83,7 @@ EXPORTED = ("attn_status_string", "attn_version", "attn_last_launch_count", "att
             "attn_bwd_workspace_bytes", "attn_bwd", "attn_fwd_f32", "attn_bwd_f32_workspace_bytes",
             "attn_bwd_f32", "attn_device_error", "attn_profile_next_call",
             "attn_selftest_wait_timeout", "attn_bwd_noalloc", "attn_fwd_strided",
-            "attn_bwd_strided")
+            "attn_bwd_strided", "attn_fwd_ex", "attn_bwd_ex", "attn_fwd_f32_ex", "attn_bwd_f32_ex")
 
 
 class AttnError(RuntimeError):
@@ -319,3 +335,84 @@ def attn_bwd_strided(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Opti
         _raise(_lib.attn_bwd_strided(*ptrs, B, H, T, D, scale, st, workspace.data_ptr(), ws_bytes,
                                      _stream_handle(stream)), "attn_bwd_strided")
     return dq, dk, dv
+
+
+def _options(causal: bool):
+    opts = attn_options(1 if causal else 0)
+    return opts
+
+
+def _all_contiguous(*tensors) -> bool:
+    return all(t.is_contiguous() for t in tensors)
+
+
+def attn_fwd_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = True,
+                stream=None):
+    """bf16 forward with options: ``causal=False`` drops the mask (every query
+    sees all T keys).  Contiguous or strided [B, H, T, D] views; O defaults to
+    the layout of q (contiguous, else a [B, T, C] buffer).  Returns (O, lse)."""
+    torch = _torch()
+    B, H, T, D = _shape4(q)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if o is None:
+        o = torch.empty_like(q) if q.is_contiguous() else empty_token_major(B, H, T, D, q.device)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    ptrs = [_check_view(q, "q", q.shape), _check_view(k, "k", q.shape),
+            _check_view(v, "v", q.shape), _check_view(o, "o", q.shape),
+            _check(lse, "lse", torch.float32, (B, H, T))]
+    st = None if _all_contiguous(q, k, v, o) else _strides_of(q, k, v, o)
+    opts = _options(causal)
+    with torch.cuda.device(q.device):
+        _raise(_lib.attn_fwd_ex(*ptrs, B, H, T, D, scale, st, ctypes.byref(opts),
+                                _stream_handle(stream)), "attn_fwd_ex")
+    return o, lse
+
+
+def attn_bwd_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[float] = None,
+                causal: bool = True, workspace=None, stream=None):
+    """bf16 backward with options (``causal`` as given to attn_fwd_ex), on
+    contiguous or strided views.  Returns (dQ, dK, dV)."""
+    torch = _torch()
+    B, H, T, D = _shape4(q)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    contig = q.is_contiguous()
+    new = (lambda: torch.empty_like(q)) if contig else (lambda: empty_token_major(B, H, T, D, q.device))
+    dq = new() if dq is None else dq
+    dk = new() if dk is None else dk
+    dv = new() if dv is None else dv
+    need = attn_bwd_workspace_bytes(B, H, T, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ptrs = [_check_view(q, "q", q.shape), _check_view(k, "k", q.shape),
+            _check_view(v, "v", q.shape), _check_view(o, "o", q.shape),
+            _check(lse, "lse", torch.float32, (B, H, T)), _check_view(dO, "dO", q.shape),
+            _check_view(dq, "dq", q.shape), _check_view(dk, "dk", q.shape),
+            _check_view(dv, "dv", q.shape)]
+    views = (q, k, v, o, dO, dq, dk, dv)
+    st = None if _all_contiguous(*views) else _strides_of(*views)
+    opts = _options(causal)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        _raise(_lib.attn_bwd_ex(*ptrs, B, H, T, D, scale, st, ctypes.byref(opts),
+                                workspace.data_ptr(), ws_bytes, _stream_handle(stream)),
+               "attn_bwd_ex")
+    return dq, dk, dv
+
+
+def attn_fwd_f32_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = True,
+                    stream=None):
+    """float32 forward with options (contiguous tensors).  Returns (O, lse)."""
+    opts = _options(causal)
+    fn = lambda *a: _lib.attn_fwd_f32_ex(*a[:-1], ctypes.byref(opts), a[-1])
+    fn.__name__ = "attn_fwd_f32_ex"
+    return _fwd(fn, _torch().float32, q, k, v, o, lse, scale, stream)
+
+
+def attn_bwd_f32_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[float] = None,
+                    causal: bool = True, workspace=None, stream=None):
+    """float32 backward with options (contiguous tensors).  Returns (dQ, dK, dV)."""
+    opts = _options(causal)
+    fn = lambda *a: _lib.attn_bwd_f32_ex(*a[:-3], ctypes.byref(opts), *a[-3:])
+    fn.__name__ = "attn_bwd_f32_ex"
+    return _bwd(fn, _lib.attn_bwd_f32_workspace_bytes, _torch().float32, q, k, v, o, lse, dO, dq,
+                dk, dv, scale, workspace, stream)

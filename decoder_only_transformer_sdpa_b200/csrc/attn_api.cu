@@ -109,6 +109,7 @@ ATTN_API const char *attn_status_string(int status) {
         case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case ATTN_ERR_DEVICE: return "current device is not sm_100 (B200 class)";
         case ATTN_ERR_SCALE: return "scale must be finite and positive";
+        case ATTN_ERR_OPTION: return "unsupported attn_options value";
         default: return "unknown status";
     }
 }
@@ -135,8 +136,44 @@ bool strides_ok(const attn_strides &x) {
 
 TStrides to_tstrides(const attn_strides &x) { return TStrides{x.b, x.h, x.t}; }
 
+// Reads the options (NULL = the decoder's defaults) into `causal`.
+int read_options(const attn_options *opts, int &causal) {
+    causal = 1;
+    if (!opts) return ATTN_OK;
+    if (opts->causal != 0 && opts->causal != 1) return ATTN_ERR_OPTION;
+    causal = opts->causal;
+    return ATTN_OK;
+}
+
+int fwd_strides(const attn_strides *strides, const Shape &s, FwdStrides &str) {
+    if (!strides) {
+        const TStrides c = contiguous_strides(s);
+        str = FwdStrides{c, c, c, c};
+        return ATTN_OK;
+    }
+    for (int i = 0; i < 4; ++i)
+        if (!strides_ok(strides[i])) return ATTN_ERR_ALIGN;
+    str = FwdStrides{to_tstrides(strides[0]), to_tstrides(strides[1]), to_tstrides(strides[2]),
+                     to_tstrides(strides[3])};
+    return ATTN_OK;
+}
+
+int bwd_strides(const attn_strides *strides, const Shape &s, BwdStrides &str) {
+    if (!strides) {
+        const TStrides c = contiguous_strides(s);
+        str = BwdStrides{c, c, c, c, c, c, c, c};
+        return ATTN_OK;
+    }
+    for (int i = 0; i < 8; ++i)
+        if (!strides_ok(strides[i])) return ATTN_ERR_ALIGN;
+    TStrides *dst[8] = {&str.q, &str.k, &str.v, &str.o, &str.dO, &str.dq, &str.dk, &str.dv};
+    for (int i = 0; i < 8; ++i) *dst[i] = to_tstrides(strides[i]);
+    return ATTN_OK;
+}
+
 int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int T,
-             int D, float scale, const FwdStrides &str, cudaStream_t stream, LaunchInfo &li) {
+             int D, float scale, int causal, const FwdStrides &str, cudaStream_t stream,
+             LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 64);
     if (st != ATTN_OK) return st;
@@ -148,14 +185,14 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     if ((st = device_setup(&err)) != ATTN_OK) return st;
     cudaError_t e = sm100_fwd(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
                               static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), lse,
-                              Shape{B, H, T, D, scale}, str, err, stream, li);
+                              Shape{B, H, T, D, scale, causal}, str, err, stream, li);
     return finish(e, li);
 }
 
 int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
              const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D, float scale,
-             const BwdStrides &str, void *workspace, size_t workspace_bytes, cudaStream_t stream,
-             LaunchInfo &li) {
+             int causal, const BwdStrides &str, void *workspace, size_t workspace_bytes,
+             cudaStream_t stream, LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 64);
     if (st != ATTN_OK) return st;
@@ -179,29 +216,36 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
         static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(o), lse,
         static_cast<const __nv_bfloat16 *>(dO), static_cast<__nv_bfloat16 *>(dq),
         static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv), dq_acc, lse2, delta,
-        Shape{B, H, T, D, scale}, str, err, stream, li);
+        Shape{B, H, T, D, scale, causal}, str, err, stream, li);
     return finish(e, li);
 }
 
 }  // namespace
 
+ATTN_API int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                         int H, int T, int D, float scale, const attn_strides *strides,
+                         const attn_options *opts, cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    int causal, st;
+    if ((st = read_options(opts, causal)) != ATTN_OK) return st;
+    FwdStrides str;
+    if ((st = fwd_strides(strides, Shape{B, H, T, D, scale}, str)) != ATTN_OK) return st;
+    return fwd_impl(q, k, v, o, lse, B, H, T, D, scale, causal, str, stream, li);
+}
+
 ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                       int H, int T, int D, float scale, cudaStream_t stream) {
-    LaunchInfo li = take_launch_info();
-    const TStrides c = contiguous_strides(Shape{B, H, T, D, scale});
-    return fwd_impl(q, k, v, o, lse, B, H, T, D, scale, FwdStrides{c, c, c, c}, stream, li);
+    return attn_fwd_ex(q, k, v, o, lse, B, H, T, D, scale, nullptr, nullptr, stream);
 }
 
 ATTN_API int attn_fwd_strided(const void *q, const void *k, const void *v, void *o, float *lse,
                               int B, int H, int T, int D, float scale, const attn_strides *strides,
                               cudaStream_t stream) {
-    LaunchInfo li = take_launch_info();
-    if (!strides) return ATTN_ERR_NULL;
-    for (int i = 0; i < 4; ++i)
-        if (!strides_ok(strides[i])) return ATTN_ERR_ALIGN;
-    const FwdStrides str{to_tstrides(strides[0]), to_tstrides(strides[1]), to_tstrides(strides[2]),
-                         to_tstrides(strides[3])};
-    return fwd_impl(q, k, v, o, lse, B, H, T, D, scale, str, stream, li);
+    if (!strides) {
+        take_launch_info();  // the arming is consumed by this call
+        return ATTN_ERR_NULL;
+    }
+    return attn_fwd_ex(q, k, v, o, lse, B, H, T, D, scale, strides, nullptr, stream);
 }
 
 // Workspace of the bf16 backward: dQ float32 accumulator, padded lse, Delta.
@@ -210,33 +254,45 @@ ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
     return bwd_workspace_layout(B, H, T, D).total;
 }
 
+ATTN_API int attn_bwd_ex(const void *q, const void *k, const void *v, const void *o,
+                         const float *lse, const void *dO, void *dq, void *dk, void *dv, int B,
+                         int H, int T, int D, float scale, const attn_strides *strides,
+                         const attn_options *opts, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    int causal, st;
+    if ((st = read_options(opts, causal)) != ATTN_OK) return st;
+    BwdStrides str;
+    if ((st = bwd_strides(strides, Shape{B, H, T, D, scale}, str)) != ATTN_OK) return st;
+    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, causal, str, workspace,
+                    workspace_bytes, stream, li);
+}
+
 ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D,
                       float scale, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    LaunchInfo li = take_launch_info();
-    const TStrides c = contiguous_strides(Shape{B, H, T, D, scale});
-    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale,
-                    BwdStrides{c, c, c, c, c, c, c, c}, workspace, workspace_bytes, stream, li);
+    return attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, nullptr, nullptr,
+                       workspace, workspace_bytes, stream);
 }
 
 ATTN_API int attn_bwd_strided(const void *q, const void *k, const void *v, const void *o,
                               const float *lse, const void *dO, void *dq, void *dk, void *dv, int B,
                               int H, int T, int D, float scale, const attn_strides *strides,
                               void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    LaunchInfo li = take_launch_info();
-    if (!strides) return ATTN_ERR_NULL;
-    for (int i = 0; i < 8; ++i)
-        if (!strides_ok(strides[i])) return ATTN_ERR_ALIGN;
-    BwdStrides str;
-    TStrides *dst[8] = {&str.q, &str.k, &str.v, &str.o, &str.dO, &str.dq, &str.dk, &str.dv};
-    for (int i = 0; i < 8; ++i) *dst[i] = to_tstrides(strides[i]);
-    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, str, workspace,
-                    workspace_bytes, stream, li);
+    if (!strides) {
+        take_launch_info();
+        return ATTN_ERR_NULL;
+    }
+    return attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, strides, nullptr,
+                       workspace, workspace_bytes, stream);
 }
 
-ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
-                          int B, int H, int T, int D, float scale, cudaStream_t stream) {
+ATTN_API int attn_fwd_f32_ex(const float *q, const float *k, const float *v, float *o, float *lse,
+                             int B, int H, int T, int D, float scale, const attn_options *opts,
+                             cudaStream_t stream) {
     LaunchInfo li = take_launch_info();
+    int causal, st0;
+    if ((st0 = read_options(opts, causal)) != ATTN_OK) return st0;
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 128);
     if (st != ATTN_OK) return st;
@@ -244,8 +300,13 @@ ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float 
     if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(o, 4) || !aligned(lse, 4))
         return ATTN_ERR_ALIGN;
     if ((st = device_setup(nullptr)) != ATTN_OK) return st;
-    cudaError_t e = simt_fwd<float>(q, k, v, o, lse, Shape{B, H, T, D, scale}, stream, li);
+    cudaError_t e = simt_fwd<float>(q, k, v, o, lse, Shape{B, H, T, D, scale, causal}, stream, li);
     return finish(e, li);
+}
+
+ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
+                          int B, int H, int T, int D, float scale, cudaStream_t stream) {
+    return attn_fwd_f32_ex(q, k, v, o, lse, B, H, T, D, scale, nullptr, stream);
 }
 
 ATTN_API size_t attn_bwd_f32_workspace_bytes(int B, int H, int T, int D) {
@@ -253,11 +314,13 @@ ATTN_API size_t attn_bwd_f32_workspace_bytes(int B, int H, int T, int D) {
     return round_up((size_t)B * H * T * sizeof(float), 256);
 }
 
-ATTN_API int attn_bwd_f32(const float *q, const float *k, const float *v, const float *o,
-                          const float *lse, const float *dO, float *dq, float *dk, float *dv, int B,
-                          int H, int T, int D, float scale, void *workspace, size_t workspace_bytes,
-                          cudaStream_t stream) {
+ATTN_API int attn_bwd_f32_ex(const float *q, const float *k, const float *v, const float *o,
+                             const float *lse, const float *dO, float *dq, float *dk, float *dv,
+                             int B, int H, int T, int D, float scale, const attn_options *opts,
+                             void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     LaunchInfo li = take_launch_info();
+    int causal, st0;
+    if ((st0 = read_options(opts, causal)) != ATTN_OK) return st0;
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 128);
     if (st != ATTN_OK) return st;
@@ -269,8 +332,16 @@ ATTN_API int attn_bwd_f32(const float *q, const float *k, const float *v, const 
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
     if ((st = device_setup(nullptr)) != ATTN_OK) return st;
     cudaError_t e = simt_bwd<float>(q, k, v, o, lse, dO, dq, dk, dv, static_cast<float *>(workspace),
-                                    Shape{B, H, T, D, scale}, stream, li);
+                                    Shape{B, H, T, D, scale, causal}, stream, li);
     return finish(e, li);
+}
+
+ATTN_API int attn_bwd_f32(const float *q, const float *k, const float *v, const float *o,
+                          const float *lse, const float *dO, float *dq, float *dk, float *dv, int B,
+                          int H, int T, int D, float scale, void *workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+    return attn_bwd_f32_ex(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, nullptr, workspace,
+                           workspace_bytes, stream);
 }
 
 ATTN_API int attn_device_error(cudaStream_t stream) {

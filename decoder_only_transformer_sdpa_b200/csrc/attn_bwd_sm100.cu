@@ -1,4 +1,5 @@
-// attn_bwd_sm100.cu -- causal attention backward on B200 tensor cores.
+// attn_bwd_sm100.cu -- causal attention backward on B200 tensor cores (and
+// the same attention without the mask).
 //
 // The pages define the forward only ("How Andrej Karpathy built GPT from 200
 // lines of code", sections "Self-Attention: the mathematical trick" [55:20]
@@ -16,7 +17,9 @@
 //          get Delta = 0 and lse = +inf, so they contribute exactly 0), and the
 //          float32 dQ accumulator zeroed;
 //   main   one CTA per (128-row key tile j, head), looping over the query
-//          tiles i >= j; dK_j and dV_j accumulate in TMEM, the partial
+//          tiles i >= j (all query tiles without the mask, where keys past T
+//          are zero rows of K and V and so add nothing to dQ); dK_j and dV_j
+//          accumulate in TMEM, the partial
 //          dQ_i = dS_ij K_j is added into the float32 accumulator by TMA
 //          reduce-add;
 //   post   dQ = scale * accumulator, rounded to bf16.
@@ -152,7 +155,7 @@ __global__ void bwd_post_kernel(const float4 *__restrict__ acc, __nv_bfloat16 *_
 
 // ------------------------------------------------------------------ main
 
-template <int D>
+template <int D, bool Causal>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
@@ -175,7 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kt = (int)(blockIdx.x / BH);  // key tile; tile 0 sees the most query tiles
     const int bh = (int)(blockIdx.x % BH);
     const int hh = bh % H, bb = bh / H;
-    const int n_q = nt - kt;                // query tiles kt .. nt-1
+    const int q_first = Causal ? kt : 0;    // query tiles q_first .. nt-1
+    const int n_q = nt - q_first;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.kv_full, 1);
@@ -223,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int issued = 0;
         for (int idx = 0; idx < n_q; ++idx) {
             const int st = idx % kQStages;
-            const int i = kt + idx;
+            const int i = q_first + idx;
             if (!mbar_wait_warp(&sm.qdo_empty[st], (uint32_t)((idx / kQStages) & 1) ^ 1u, err, abort)) break;
             mbar_arrive_expect_tx_e(&sm.qdo_full[st], 2 * Smem::kTileBytes + 2 * kBT * 4);
             tma_load_4d_e(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, hh, bb);
@@ -315,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait_warp(&sm.sdp_full, (uint32_t)idx & 1u, err, abort);
             if (!ok) break;
             tc_fence_after();
-            const bool diag = (idx == 0);
+            const bool diag = Causal && (idx == 0);
             const uint32_t lse_addr = smem_u32(sm.lse2[st]), dl_addr = smem_u32(sm.delta[st]);
             const uint32_t ds_row = smem_u32(sm.ds[b][half]) + (uint32_t)kr * 128;
 #pragma unroll
@@ -437,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
                 if (leader) {
-                    tma_reduce_add_3d(&tdq, sm.stage, 32 * h, (kt + idx) * kBT, bh);
+                    tma_reduce_add_3d(&tdq, sm.stage, 32 * h, (q_first + idx) * kBT, bh);
                     bulk_commit();
                 }
             }
@@ -471,7 +475,7 @@ cudaError_t make_map(CUtensorMap *map, const void *ptr, int BH, int T, int D, bo
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D>
+template <int D, bool Causal>
 cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                        const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                        __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
@@ -498,11 +502,11 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     li.kernels += 1;
 
     const size_t smem = sizeof(BwdSmem<D>) + 1024;
-    if ((e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(bwd_main_kernel<D, Causal>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    bwd_main_kernel<D><<<(unsigned)blocks, kThreads, smem, st>>>(
+    bwd_main_kernel<D, Causal><<<(unsigned)blocks, kThreads, smem, st>>>(
         mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, str.dk, str.dv, s.T, Tpad, s.H, BH, nt,
         s.scale * kLog2e, s.scale, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -526,10 +530,15 @@ cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
                       float *lse2, float *delta, Shape s, const BwdStrides &str, int *err,
                       cudaStream_t st, LaunchInfo &li) {
-    if (s.D == 64)
-        return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, str, err, st, li);
-    if (s.D == 32)
-        return launch_bwd<32>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, str, err, st, li);
+#define ATTN_BWD_CASE(DD)                                                                          \
+    if (s.D == DD)                                                                                 \
+        return s.causal ? launch_bwd<DD, true>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, \
+                                               s, str, err, st, li)                                \
+                        : launch_bwd<DD, false>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2,      \
+                                                delta, s, str, err, st, li);
+    ATTN_BWD_CASE(64)
+    ATTN_BWD_CASE(32)
+#undef ATTN_BWD_CASE
     return cudaErrorInvalidValue;
 }
 

@@ -1,4 +1,5 @@
-// attn_fwd_sm100.cu -- causal attention forward on B200 tensor cores.
+// attn_fwd_sm100.cu -- causal attention forward on B200 tensor cores (and the
+// same attention without the mask).
 //
 // Computes, per head, O = softmax(scale * Q K^T with the upper triangle at
 // -inf) V and the natural-log row log-sum-exp ("How Andrej Karpathy built GPT
@@ -26,6 +27,8 @@
 //               the O accumulator, final O / l and lse per item.
 // Key tiles wholly above the diagonal are never loaded; only the diagonal
 // tile applies the element mask.  The score matrix never leaves the SM.
+// Without the mask (Causal = false) every query tile runs over all key tiles
+// and only the last key tile masks the keys past T.
 //
 // TMEM columns: S [0,128), P (bf16 pairs) [128,192), O [192, 192+D).
 #include "internal.h"
@@ -66,7 +69,7 @@ __device__ __forceinline__ int item_of(int c, int n, int G, int W) {
     return w < W ? (int)w : -1;
 }
 
-template <int D>
+template <int D, bool Causal>
 __global__ void __launch_bounds__(kThreads, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16 *__restrict__ o,
@@ -137,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
             tma_load_4d_e(sm.q[qb], &tq, &sm.q_full[qb], 0, qt * kBM, hh, bb);
             nq = n + 1;
-            for (int j = 0; j <= qt; ++j, ++gt) {
+            const int nk = Causal ? qt + 1 : ntiles;  // key tiles this item reads
+            for (int j = 0; j < nk; ++j, ++gt) {
                 const int s = gt % kStages;
                 const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
                 if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
@@ -202,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int qb = n & 1;
             if (!(ok = mbar_wait_warp(&sm.q_full[qb], (uint32_t)(n >> 1) & 1u, err, abort))) break;
             const uint64_t qd = smem_desc(smem_u32(sm.q[qb]), 16, kAtom, kSwz);
-            for (int j = 0; j <= qt; ++j, ++gt) {
+            const int nk = Causal ? qt + 1 : ntiles;
+            for (int j = 0; j < nk; ++j, ++gt) {
                 // S_g = Q K_j^T, once the softmax has read S_{g-1} out of TMEM.
                 const int s = gt % kStages;
                 if (!(ok = mbar_wait_warp(&sm.k_full[s], (uint32_t)(gt / kStages) & 1u, err, abort))) break;
@@ -216,12 +221,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                     mma_ss_x2<2, 2>(tS, qd, kd, idS, 0u);
                 mma_commit_e(&sm.s_full);
                 mma_commit_e(&sm.k_empty[s]);
-                if (j == qt) mma_commit_e(&sm.q_empty[qb]);  // this item's Q no longer read
+                if (j == nk - 1) mma_commit_e(&sm.q_empty[qb]);  // this item's Q no longer read
                 if (pv_g >= 0 && !(ok = issue_pv())) break;
                 pv_g = gt;
                 pv_n = n;
                 pv_j = j;
-                pv_last = (j == qt);
+                pv_last = (j == nk - 1);
             }
         }
         if (ok && pv_g >= 0) ok = issue_pv();
@@ -240,7 +245,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (w < 0) break;
             const int qt = ntiles - 1 - w / BH, bh = w % BH;
             float m_used = -INFINITY, l = 0.f;
-            for (int j = 0; j <= qt; ++j, ++gt) {
+            const int nk = Causal ? qt + 1 : ntiles;
+            for (int j = 0; j < nk; ++j, ++gt) {
                 ok = mbar_wait_warp(&sm.s_full, (uint32_t)gt & 1u, err, abort);
                 if (!ok) break;
                 tc_fence_after();
@@ -267,10 +273,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                         s[96 + x] = __uint_as_float(r3[x]);
                     }
                 }
-                if (j == qt) {  // diagonal tile: key column c is visible to row r iff c <= r
+                if constexpr (Causal) {
+                    if (j == qt) {  // diagonal tile: key column c is visible to row r iff c <= r
 #pragma unroll
-                    for (int c = 0; c < kBN; ++c)
-                        if (c > row) s[c] = -INFINITY;
+                        for (int c = 0; c < kBN; ++c)
+                            if (c > row) s[c] = -INFINITY;
+                    }
+                } else {
+                    const int lim = T - j * kBN;  // keys past T (zero-filled rows) are masked
+                    if (lim < kBN) {
+#pragma unroll
+                        for (int c = 0; c < kBN; ++c)
+                            if (c >= lim) s[c] = -INFINITY;
+                    }
                 }
                 // Row max as eight independent chains (short dependency depth).
                 float mc[8];
@@ -405,7 +420,7 @@ cudaError_t make_map_bf16(void *map, const void *ptr, const Shape &s, const TStr
 
 namespace {
 
-template <int D>
+template <int D, bool Causal>
 cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                        __nv_bfloat16 *o, float *lse, Shape s, const FwdStrides &str, int *err,
                        cudaStream_t st, LaunchInfo &li) {
@@ -425,13 +440,13 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if ((e = make_map_bf16(&mk, k, s, str.k)) != cudaSuccess) return e;
     if ((e = make_map_bf16(&mv, v, s, str.v)) != cudaSuccess) return e;
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
-    if ((e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(fwd_kernel<D, Causal>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
     const float scale_log2 = s.scale * 1.4426950408889634f;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    fwd_kernel<D><<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, o, str.o, lse, s.T, s.H, BH, ntiles,
-                                                            scale_log2, err);
+    fwd_kernel<D, Causal><<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, o, str.o, lse, s.T, s.H,
+                                                                    BH, ntiles, scale_log2, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
     return mark_main_end(li, st);
@@ -442,8 +457,12 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
 cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       __nv_bfloat16 *o, float *lse, Shape s, const FwdStrides &str, int *err,
                       cudaStream_t st, LaunchInfo &li) {
-    if (s.D == 64) return launch_fwd<64>(q, k, v, o, lse, s, str, err, st, li);
-    if (s.D == 32) return launch_fwd<32>(q, k, v, o, lse, s, str, err, st, li);
+    if (s.D == 64)
+        return s.causal ? launch_fwd<64, true>(q, k, v, o, lse, s, str, err, st, li)
+                        : launch_fwd<64, false>(q, k, v, o, lse, s, str, err, st, li);
+    if (s.D == 32)
+        return s.causal ? launch_fwd<32, true>(q, k, v, o, lse, s, str, err, st, li)
+                        : launch_fwd<32, false>(q, k, v, o, lse, s, str, err, st, li);
     return cudaErrorInvalidValue;
 }
 

@@ -11,7 +11,8 @@
 // values.  Here each thread owns one query row and walks the keys j <= i once
 // with a running maximum and running sum (online softmax), so the T x T score
 // matrix never exists in memory.  The backward recomputes P_ij from the saved
-// lse_i and follows the exact derivative.
+// lse_i and follows the exact derivative.  With causal = 0 the same kernels
+// run every row over all T keys (every key over all T queries).
 //
 // Block = 64 threads = 64 rows of one head; K/V (or Q/dO) tiles of 64 rows
 // are staged in shared memory as float32 and shared by the block.
@@ -51,7 +52,7 @@ template <typename T, int DMAX>
 __global__ void __launch_bounds__(kRows) fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                     const T *__restrict__ v, T *__restrict__ o,
                                                     float *__restrict__ lse, int Tn, int D,
-                                                    float scale) {
+                                                    float scale, int causal) {
     extern __shared__ float smem[];
     float *ks = smem;
     float *vs = smem + kRows * D;
@@ -70,14 +71,15 @@ __global__ void __launch_bounds__(kRows) fwd_kernel(const T *__restrict__ q, con
         acc[d] = 0.f;
     }
     float m = -INFINITY, l = 0.f;
-    const int last_row = min(tile * kRows + kRows, Tn) - 1;
-    for (int j0 = 0; j0 <= last_row; j0 += kRows) {
+    const int last_key = causal ? min(tile * kRows + kRows, Tn) - 1 : Tn - 1;
+    const int my_last = causal ? i : Tn - 1;
+    for (int j0 = 0; j0 <= last_key; j0 += kRows) {
         __syncthreads();
         stage_rows(ks, k + base, j0, Tn, D);
         stage_rows(vs, v + base, j0, Tn, D);
         __syncthreads();
         if (row_ok) {
-            const int jend = min(j0 + kRows - 1, i);
+            const int jend = min(j0 + kRows - 1, my_last);
             for (int j = j0; j <= jend; ++j) {
                 const float *kj = ks + (j - j0) * D;
                 const float *vj = vs + (j - j0) * D;
@@ -117,13 +119,14 @@ __global__ void delta_kernel(const T *__restrict__ o, const T *__restrict__ dO,
     delta[r] = acc;
 }
 
-// dQ_i = scale * sum_{j<=i} P_ij (dP_ij - Delta_i) k_j, thread per query row.
+// dQ_i = scale * sum_{j<=i} P_ij (dP_ij - Delta_i) k_j (all j when not
+// causal), thread per query row.
 template <typename T, int DMAX>
 __global__ void __launch_bounds__(kRows) dq_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                    const T *__restrict__ v, const float *__restrict__ lse,
                                                    const T *__restrict__ dO,
                                                    const float *__restrict__ delta, T *__restrict__ dq,
-                                                   int Tn, int D, float scale) {
+                                                   int Tn, int D, float scale, int causal) {
     extern __shared__ float smem[];
     float *ks = smem;
     float *vs = smem + kRows * D;
@@ -144,14 +147,15 @@ __global__ void __launch_bounds__(kRows) dq_kernel(const T *__restrict__ q, cons
     }
     const float lse_i = row_ok ? lse[(size_t)bh * Tn + i] : 0.f;
     const float delta_i = row_ok ? delta[(size_t)bh * Tn + i] : 0.f;
-    const int last_row = min(tile * kRows + kRows, Tn) - 1;
-    for (int j0 = 0; j0 <= last_row; j0 += kRows) {
+    const int last_key = causal ? min(tile * kRows + kRows, Tn) - 1 : Tn - 1;
+    const int my_last = causal ? i : Tn - 1;
+    for (int j0 = 0; j0 <= last_key; j0 += kRows) {
         __syncthreads();
         stage_rows(ks, k + base, j0, Tn, D);
         stage_rows(vs, v + base, j0, Tn, D);
         __syncthreads();
         if (row_ok) {
-            const int jend = min(j0 + kRows - 1, i);
+            const int jend = min(j0 + kRows - 1, my_last);
             for (int j = j0; j <= jend; ++j) {
                 const float *kj = ks + (j - j0) * D;
                 const float *vj = vs + (j - j0) * D;
@@ -177,8 +181,8 @@ __global__ void __launch_bounds__(kRows) dq_kernel(const T *__restrict__ q, cons
     }
 }
 
-// dV_j = sum_{i>=j} P_ij dO_i and dK_j = scale * sum_{i>=j} dS_ij q_i, thread
-// per key row.
+// dV_j = sum_{i>=j} P_ij dO_i and dK_j = scale * sum_{i>=j} dS_ij q_i (all i
+// when not causal), thread per key row.
 template <typename T, int DMAX>
 __global__ void __launch_bounds__(kRows) dkdv_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                      const T *__restrict__ v,
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(kRows) dkdv_kernel(const T *__restrict__ q, co
                                                      const T *__restrict__ dO,
                                                      const float *__restrict__ delta,
                                                      T *__restrict__ dk, T *__restrict__ dv, int Tn,
-                                                     int D, float scale) {
+                                                     int D, float scale, int causal) {
     extern __shared__ float smem[];
     float *qs = smem;
     float *gs = smem + kRows * D;
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(kRows) dkdv_kernel(const T *__restrict__ q, co
         dka[d] = 0.f;
         dva[d] = 0.f;
     }
-    for (int i0 = tile * kRows; i0 < Tn; i0 += kRows) {
+    for (int i0 = causal ? tile * kRows : 0; i0 < Tn; i0 += kRows) {
         __syncthreads();
         stage_rows(qs, q + base, i0, Tn, D);
         stage_rows(gs, dO + base, i0, Tn, D);
@@ -225,7 +229,7 @@ __global__ void __launch_bounds__(kRows) dkdv_kernel(const T *__restrict__ q, co
         __syncthreads();
         if (row_ok) {
             const int iend = min(i0 + kRows, Tn);
-            for (int i = max(i0, j); i < iend; ++i) {
+            for (int i = causal ? max(i0, j) : i0; i < iend; ++i) {
                 const float *qi = qs + (i - i0) * D;
                 const float *gi = gs + (i - i0) * D;
                 float s = 0.f, dp = 0.f;
@@ -274,7 +278,7 @@ cudaError_t simt_fwd(const T *q, const T *k, const T *v, T *o, float *lse, Shape
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     void *args[] = {(void *)&q, (void *)&k, (void *)&v, (void *)&o, (void *)&lse,
-                    (void *)&s.T, (void *)&s.D, (void *)&s.scale};
+                    (void *)&s.T, (void *)&s.D, (void *)&s.scale, (void *)&s.causal};
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     e = cudaLaunchKernel(fn, dim3((unsigned)blocks), dim3(kRows), args, smem, st);
     if (e != cudaSuccess) return e;
@@ -300,7 +304,8 @@ cudaError_t simt_bwd(const T *q, const T *k, const T *v, const T *o, const float
     if (e != cudaSuccess) return e;
     const float *delta_c = delta;
     void *a1[] = {(void *)&q, (void *)&k, (void *)&v, (void *)&lse, (void *)&dO,
-                  (void *)&delta_c, (void *)&dq, (void *)&s.T, (void *)&s.D, (void *)&s.scale};
+                  (void *)&delta_c, (void *)&dq, (void *)&s.T, (void *)&s.D, (void *)&s.scale,
+                  (void *)&s.causal};
     e = cudaLaunchKernel(fdq, dim3((unsigned)blocks), dim3(kRows), a1, smem_dq, st);
     if (e != cudaSuccess) return e;
     li.kernels += 1;
@@ -311,7 +316,7 @@ cudaError_t simt_bwd(const T *q, const T *k, const T *v, const T *o, const float
     if (e != cudaSuccess) return e;
     void *a2[] = {(void *)&q, (void *)&k, (void *)&v, (void *)&lse, (void *)&dO,
                   (void *)&delta_c, (void *)&dk, (void *)&dv, (void *)&s.T, (void *)&s.D,
-                  (void *)&s.scale};
+                  (void *)&s.scale, (void *)&s.causal};
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     e = cudaLaunchKernel(fkv, dim3((unsigned)blocks), dim3(kRows), a2, smem_kv, st);
     if (e != cudaSuccess) return e;

@@ -20,6 +20,7 @@ constexpr int kErrTimeout = 1;
 struct Shape {
     int B, H, T, D;
     float scale;
+    int causal = 1;  // 1: key j visible to query i iff j <= i; 0: all keys visible
 };
 
 // Element strides of a [B, H, T, D] view (the d stride is 1).  Contiguous

@@ -36,6 +36,9 @@
  *    asynchronously at the caller's next synchronisation.  Every internal wait
  *    of the kernels is bounded: a wait that runs out records a flag that
  *    attn_device_error() returns as ATTN_ERR_TIMEOUT.
+ *  - The plain entry points compute the decoder's causal attention; the _ex
+ *    entry points also take an attn_options (the mask) and, for bf16,
+ *    strides.
  *  - Calls are thread-safe; tensor descriptors travel as kernel parameters.
  *    Calls that write the same output buffers race like any CUDA work.
  */
@@ -62,7 +65,8 @@ typedef enum {
     ATTN_ERR_TIMEOUT = -6,       /* a bounded in-kernel wait ran out                */
     ATTN_ERR_WORKSPACE = -7,     /* workspace NULL or smaller than required         */
     ATTN_ERR_DEVICE = -8,        /* current device is not sm_100 (B200 class)       */
-    ATTN_ERR_SCALE = -9          /* scale is not finite and positive                */
+    ATTN_ERR_SCALE = -9,         /* scale is not finite and positive                */
+    ATTN_ERR_OPTION = -10        /* an attn_options field holds an unsupported value */
 } attn_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -147,6 +151,39 @@ int attn_bwd_strided(const void *q, const void *k, const void *v, const void *o,
                      int B, int H, int T, int D, float scale, const attn_strides *strides,
                      void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ---------------- options: the mask ------------------------------------- */
+
+/* Options of the _ex entry points.  A NULL options pointer means the
+ * defaults, which are the decoder's attention computed by attn_fwd/attn_bwd.
+ *
+ * causal: 1 (default) masks key j for query i when j > i -- the -inf upper
+ *   triangle that keeps a decoder token from seeing later tokens ("How Andrej
+ *   Karpathy built GPT from 200 lines of code", section "Self-Attention: the
+ *   mathematical trick" [55:20]).  0 drops the mask: every query attends to
+ *   all T keys (the encoder-style attention that the same passage contrasts
+ *   with the decoder's), lse_i = ln sum_{j<T} exp(S_ij), and the backward
+ *   sums over all i and j.  Any other value gives ATTN_ERR_OPTION. */
+typedef struct {
+    int32_t causal;
+} attn_options;
+
+/* attn_fwd with options, on strided views.  strides: NULL for contiguous
+ * [B, H, T, D] tensors, else strides[0..3] for q, k, v, o under the rules of
+ * attn_fwd_strided.  opts: NULL for the defaults.  Other rules as attn_fwd. */
+int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int H, int T, int D, float scale, const attn_strides *strides,
+                const attn_options *opts, cudaStream_t stream);
+
+/* attn_bwd with options, on strided views.  strides: NULL for contiguous
+ * tensors, else strides[0..7] as attn_bwd_strided.  opts must describe the
+ * same attention the forward computed (lse depends on it).  Workspace as
+ * attn_bwd (attn_bwd_workspace_bytes). */
+int attn_bwd_ex(const void *q, const void *k, const void *v, const void *o,
+                const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                int B, int H, int T, int D, float scale, const attn_strides *strides,
+                const attn_options *opts, void *workspace, size_t workspace_bytes,
+                cudaStream_t stream);
+
 /* ---------------- float32 path: CUDA cores, IEEE expf -------------------- */
 
 /* Forward in float32 (all tensors float32).  1 <= D <= 128. */
@@ -161,6 +198,16 @@ int attn_bwd_f32(const float *q, const float *k, const float *v, const float *o,
                  const float *lse, const float *dO, float *dq, float *dk, float *dv,
                  int B, int H, int T, int D, float scale,
                  void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* attn_fwd_f32 / attn_bwd_f32 with options (NULL = defaults); contiguous
+ * tensors only.  Workspace as attn_bwd_f32. */
+int attn_fwd_f32_ex(const float *q, const float *k, const float *v, float *o, float *lse,
+                    int B, int H, int T, int D, float scale, const attn_options *opts,
+                    cudaStream_t stream);
+int attn_bwd_f32_ex(const float *q, const float *k, const float *v, const float *o,
+                    const float *lse, const float *dO, float *dq, float *dk, float *dv,
+                    int B, int H, int T, int D, float scale, const attn_options *opts,
+                    void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* ---------------- diagnostics ------------------------------------------- */
 
@@ -180,7 +227,7 @@ int attn_selftest_wait_timeout(uint32_t polls, cudaStream_t stream);
  * enqueued (for launch accounting). */
 int attn_last_launch_count(void);
 
-/* Timing hook: arms the next attn_fwd / attn_bwd call made on this host
+/* Timing hook: arms the next forward or backward call made on this host
  * thread to record `start` just before and `end` just after enqueueing its
  * main kernel (the forward kernel, or the backward's tile kernel), on the
  * call's stream.  Both are cudaEvent_t handles owned by the caller; the call

@@ -21,12 +21,20 @@ BF16_TOL = dict(max_abs=2e-2, rel_l2=1e-2)
 LSE_BF16_MAX_ABS = 1e-3
 
 
-def run_gpu(inp, scale=None, dtype=torch.bfloat16):
-    """Forward + backward through the C ABI.  Returns CPU float64 numpy arrays."""
+def run_gpu(inp, scale=None, dtype=torch.bfloat16, causal=True):
+    """Forward + backward through the C ABI (the plain entry points for the
+    causal attention, the _ex ones with causal=False otherwise).  Returns CPU
+    float64 numpy arrays."""
     import decoder_only_transformer_sdpa_b200 as A
     dev = torch.device("cuda", 0)
     q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
-    if dtype == torch.bfloat16:
+    if not causal and dtype == torch.bfloat16:
+        o, lse = A.attn_fwd_ex(q, k, v, scale=scale, causal=False)
+        dq, dk, dv = A.attn_bwd_ex(q, k, v, o, lse, do, scale=scale, causal=False)
+    elif not causal:
+        o, lse = A.attn_fwd_f32_ex(q, k, v, scale=scale, causal=False)
+        dq, dk, dv = A.attn_bwd_f32_ex(q, k, v, o, lse, do, scale=scale, causal=False)
+    elif dtype == torch.bfloat16:
         o, lse = A.attn_fwd(q, k, v, scale=scale)
         dq, dk, dv = A.attn_bwd(q, k, v, o, lse, do, scale=scale)
     else:
@@ -48,15 +56,15 @@ def sample_heads(B: int, H: int, n: int, seed: int):
     return np.array(sorted(pick))
 
 
-def run_oracle(inp, heads=None, scale=None):
+def run_oracle(inp, heads=None, scale=None, causal=True):
     """Oracle outputs on all heads, or only the flat head indices `heads`
     (heads are independent, so a subset is computed exactly)."""
     arrs = {n: inp[n].to(torch.float64).numpy() for n in ("q", "k", "v", "do")}
     B, H, T, D = arrs["q"].shape
     if heads is not None:
         arrs = {n: a.reshape(B * H, T, D)[heads][None] for n, a in arrs.items()}
-    o, lse = oracle.attn_fwd(arrs["q"], arrs["k"], arrs["v"], scale)
-    dq, dk, dv = oracle.attn_bwd(arrs["q"], arrs["k"], arrs["v"], arrs["do"], scale)
+    o, lse = oracle.attn_fwd(arrs["q"], arrs["k"], arrs["v"], scale, causal=causal)
+    dq, dk, dv = oracle.attn_bwd(arrs["q"], arrs["k"], arrs["v"], arrs["do"], scale, causal=causal)
     return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv)
 
 

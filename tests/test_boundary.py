@@ -146,3 +146,37 @@ def test_strided_argument_errors(bad):
         assert lib.attn_bwd_strided(*([P] * 9), 1, 1, 8, 64, 0.125, st, P, 1 << 30, None) == E_ALIGN
     # valid strides still hit the ordinary checks first-class (unsupported D)
     assert lib.attn_fwd_strided(P, P, P, P, P, 1, 1, 8, 48, 0.125, good, None) == E_D
+
+
+def _opts(causal):
+    return ctypes.byref(lib_mod.attn_options(causal))
+
+
+@pytest.mark.parametrize("causal", [2, -1, 7])
+def test_options_reject_unknown_mask(causal):
+    lib = lib_mod.lib()
+    E_OPTION = -10
+    assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.125, None, _opts(causal), None) == E_OPTION
+    assert lib.attn_bwd_ex(*([P] * 9), 1, 1, 8, 64, 0.125, None, _opts(causal), P, 1 << 30,
+                           None) == E_OPTION
+    assert lib.attn_fwd_f32_ex(P, P, P, P, P, 1, 1, 8, 8, 0.35, _opts(causal), None) == E_OPTION
+    assert lib.attn_bwd_f32_ex(*([P] * 9), 1, 1, 8, 8, 0.35, _opts(causal), P, 1 << 30,
+                               None) == E_OPTION
+    assert lib_mod.attn_status_string(E_OPTION) != lib_mod.attn_status_string(12345)
+
+
+@pytest.mark.parametrize("causal", [0, 1])
+def test_options_pass_to_the_ordinary_checks(causal):
+    """Valid options (and NULL options or strides) reach the same argument
+    checks as the plain entry points, before anything touches CUDA."""
+    lib = lib_mod.lib()
+    for o in (_opts(causal), None):
+        assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 48, 0.125, None, o, None) == E_D
+        assert lib.attn_fwd_ex(None, P, P, P, P, 1, 1, 8, 64, 0.125, None, o, None) == E_NULL
+        assert lib.attn_fwd_ex(P, P, P, P, P, 0, 1, 8, 64, 0.125, None, o, None) == E_SHAPE
+        assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, float("nan"), None, o, None) == E_SCALE
+        assert lib.attn_bwd_ex(*([P] * 9), 1, 1, 8, 64, 0.125, None, o, None, 0, None) == E_WS
+        assert lib.attn_fwd_f32_ex(P, P, P, P, P, 1, 1, 8, 129, 0.1, o, None) == E_D
+        bad = _strides(8, t=3)
+        assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.125, bad, o, None) == E_ALIGN
+        assert lib.attn_bwd_ex(*([P] * 9), 1, 1, 8, 64, 0.125, bad, o, P, 1 << 30, None) == E_ALIGN
