@@ -1,5 +1,7 @@
-"""Double-precision CPU oracle of causal multi-head attention (fwd + bwd), and
-of the same attention without the mask (``causal=False``).
+"""Double-precision CPU oracle of causal multi-head attention (fwd + bwd), of
+the same attention without the mask (``causal=False``) and of both with
+dropout on the attention weights (``dropout_p``, ``seed``, ``offset``; the
+keep mask is drawn by the oracle's own Philox4x32-10).
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
 bench's CPU-baseline leg may import this package.  The product path (the CUDA
@@ -53,6 +55,19 @@ class OracleLib:
             f = getattr(lib, "oracle_attn_bwd" + suffix)
             f.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double]
             f.restype = None
+        u32, u64 = ctypes.c_uint32, ctypes.c_uint64
+        lib.oracle_philox4x32_10.argtypes = [ctypes.POINTER(u32), ctypes.POINTER(u32),
+                                             ctypes.POINTER(u32)]
+        lib.oracle_philox4x32_10.restype = None
+        lib.oracle_dropout_mask.argtypes = [i, i, i, ctypes.c_double, u64, u32,
+                                            ctypes.POINTER(ctypes.c_uint8)]
+        lib.oracle_dropout_mask.restype = None
+        lib.oracle_attn_fwd_dropout.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double, i,
+                                                ctypes.c_double, u64, u32]
+        lib.oracle_attn_fwd_dropout.restype = None
+        lib.oracle_attn_bwd_dropout.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i,
+                                                ctypes.c_double, i, ctypes.c_double, u64, u32]
+        lib.oracle_attn_bwd_dropout.restype = None
         lib.oracle_threads.argtypes = []
         lib.oracle_threads.restype = i
         self.lib = lib
@@ -60,13 +75,18 @@ class OracleLib:
     def _fn(self, name: str, causal: bool):
         return getattr(self.lib, name if causal else name + "_nc")
 
-    def attn_fwd(self, q, k, v, scale=None, causal=True):
+    def attn_fwd(self, q, k, v, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0):
         """Returns (O [B,H,T,D], lse [B,H,T]) in float64."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, H, T, D = _shape(q)
         scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
         o = np.empty_like(q)
         lse = np.empty((B, H, T), dtype=np.float64)
+        if dropout_p:
+            self.lib.oracle_attn_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D,
+                                             scale, int(bool(causal)), float(dropout_p), int(seed),
+                                             int(offset))
+            return o, lse
         self._fn("oracle_attn_fwd", causal)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                             B, H, T, D, scale)
         return o, lse
@@ -80,15 +100,35 @@ class OracleLib:
         self._fn("oracle_attn_probs", causal)(_ptr(q), _ptr(k), _ptr(p), B, H, T, D, scale)
         return p
 
-    def attn_bwd(self, q, k, v, do, scale=None, causal=True):
+    def attn_bwd(self, q, k, v, do, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0):
         """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
         q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
         B, H, T, D = _shape(q)
         scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
         dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        if dropout_p:
+            self.lib.oracle_attn_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk),
+                                             _ptr(dv), B, H, T, D, scale, int(bool(causal)),
+                                             float(dropout_p), int(seed), int(offset))
+            return dq, dk, dv
         self._fn("oracle_attn_bwd", causal)(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq),
                                             _ptr(dk), _ptr(dv), B, H, T, D, scale)
         return dq, dk, dv
+
+    def philox4x32_10(self, ctr, key):
+        """Philox4x32-10 of one 4-word counter under a 2-word key."""
+        c = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in ctr])
+        kk = (ctypes.c_uint32 * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+        out = (ctypes.c_uint32 * 4)()
+        self.lib.oracle_philox4x32_10(c, kk, out)
+        return [int(x) for x in out]
+
+    def dropout_mask(self, B, H, T, p, seed=0, offset=0):
+        """The keep mask [B,H,T,T] (uint8, 1 = kept) over all (i, j)."""
+        m = np.empty((B, H, T, T), dtype=np.uint8)
+        self.lib.oracle_dropout_mask(B, H, T, float(p), int(seed), int(offset),
+                                     m.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+        return m
 
     def threads_used(self) -> int:
         """OpenMP threads the most recent call ran on."""
@@ -120,9 +160,9 @@ def _shape(q: np.ndarray):
     return tuple(int(s) for s in q.shape)
 
 
-def attn_fwd(q, k, v, scale=None, causal=True):
+def attn_fwd(q, k, v, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0):
     """Returns (O [B,H,T,D], lse [B,H,T]) in float64."""
-    return _load().attn_fwd(q, k, v, scale, causal)
+    return _load().attn_fwd(q, k, v, scale, causal, dropout_p, seed, offset)
 
 
 def attn_probs(q, k, scale=None, causal=True):
@@ -130,9 +170,19 @@ def attn_probs(q, k, scale=None, causal=True):
     return _load().attn_probs(q, k, scale, causal)
 
 
-def attn_bwd(q, k, v, do, scale=None, causal=True):
+def attn_bwd(q, k, v, do, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0):
     """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
-    return _load().attn_bwd(q, k, v, do, scale, causal)
+    return _load().attn_bwd(q, k, v, do, scale, causal, dropout_p, seed, offset)
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32-10 of one counter (4 words) under one key (2 words)."""
+    return _load().philox4x32_10(ctr, key)
+
+
+def dropout_mask(B, H, T, p, seed=0, offset=0):
+    """The dropout keep mask [B,H,T,T] (uint8, 1 = kept)."""
+    return _load().dropout_mask(B, H, T, p, seed, offset)
 
 
 def threads_used() -> int:

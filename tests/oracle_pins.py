@@ -31,6 +31,15 @@ permutation relabels every output the same way (nothing depends on position);
 its last row equals the causal last row (both see all T keys); shift
 invariance, finite differences, torch's ``is_causal=False`` witness and a
 hand-derived golden example.
+
+Dropout on the attention weights (keep mask drawn by Philox4x32-10) is pinned
+by: the generator against cuRAND's host Philox4x32-10 generator (a library
+routine, run on the CPU), word by word and as the whole keep mask of a head;
+the keep rate within binomial bounds and distinct masks per head, offset and
+seed; p below 1/131072 (threshold 0) giving back the plain attention bit for
+bit; the uniform-weight closed form; unbiasedness of O and dV over seeds;
+finite differences with the mask held fixed; and torch float64 autograd of
+the same dropped-weight attention.
 """
 from __future__ import annotations
 
@@ -340,3 +349,218 @@ ALL_PINS = [check_probs_rows, check_averaging_trick, check_causality, check_sing
             check_nc_probs_rows, check_nc_averaging, check_nc_permutation,
             check_nc_last_row_and_single_token, check_nc_shift_invariance,
             check_nc_finite_differences, check_nc_torch_witness]
+
+
+# ---------------------------------------------------------------- dropout
+
+def _curand():
+    """cuRAND's host-side generator (runs on the CPU, no GPU needed), or None."""
+    import ctypes
+    import glob
+    paths = sorted(glob.glob("/usr/local/cuda/lib64/libcurand.so*"))
+    try:
+        import nvidia.curand
+        paths += sorted(glob.glob(os.path.join(os.path.dirname(nvidia.curand.__file__), "lib",
+                                               "libcurand.so*")))
+    except ImportError:
+        pass
+    for path in paths:
+        try:
+            return ctypes.CDLL(path)
+        except OSError:
+            continue
+    return None
+
+
+def curand_philox_block(seed: int, block: int):
+    """Four 32-bit outputs of cuRAND's host PHILOX4_32_10 generator at output
+    offset 4 * block, under key (seed low word, seed high word).  Its host
+    generator places output block b at counter words (b div 2^16 over words 0
+    and 1, b mod 2^16, 0); see curand_block_of."""
+    import ctypes
+    lib = _curand()
+    assert lib is not None
+    g = ctypes.c_void_p()
+    assert lib.curandCreateGeneratorHost(ctypes.byref(g), 161) == 0   # PHILOX4_32_10
+    try:
+        assert lib.curandSetPseudoRandomGeneratorSeed(g, ctypes.c_ulonglong(seed)) == 0
+        assert lib.curandSetGeneratorOffset(g, ctypes.c_ulonglong(4 * block)) == 0
+        buf = (ctypes.c_uint32 * 4)()
+        assert lib.curandGenerate(g, buf, ctypes.c_size_t(4)) == 0
+        return [int(x) for x in buf]
+    finally:
+        lib.curandDestroyGenerator(g)
+
+
+def curand_block_of(c0: int, c1: int, c2: int) -> int:
+    """The cuRAND host output block holding counter (c0, c1, c2, 0), c2 < 2^16."""
+    assert 0 <= c2 < (1 << 16) and c1 < (1 << 14)
+    return (((c1 << 32) | c0) << 16) | c2
+
+
+def _threshold(p):
+    return int(math.floor(p * 65536.0 + 0.5))
+
+
+def check_philox_against_curand(impl):
+    import pytest
+    if _curand() is None:
+        pytest.skip("libcurand not found")
+    for seed in (0, 1, 0xFFFFFFFF, (5 << 32) + 17, 0x123456789ABCDEF0):
+        key = [seed & 0xFFFFFFFF, seed >> 32]
+        for ctr in ((0, 0, 0), (0, 0, 1), (1, 0, 0), (0, 1, 0), (12345, 0, 65535),
+                    (0xFFFFFFFF, 0x3FFF, 0xFFFF), (0xDEADBEEF, 0x1234, 0x0F0F)):
+            want = curand_philox_block(seed, curand_block_of(*ctr))
+            got = impl.philox4x32_10(list(ctr) + [0], key)
+            assert got == want, f"Philox4x32-10 differs from cuRAND (seed {seed:#x}, ctr {ctr})"
+
+
+def check_dropout_mask_against_curand(impl):
+    """Head bh at offset 0 uses counters (i, j / 8, bh, 0): its whole keep
+    mask follows from cuRAND's outputs and the 16-bit split of the words."""
+    import pytest
+    if _curand() is None:
+        pytest.skip("libcurand not found")
+    T, p, seed = 40, 0.3, 0xC0FFEE
+    t = _threshold(p)
+    masks = impl.dropout_mask(1, 3, T, p, seed, 0)[0]
+    for bh in (0, 2):
+        for i in range(T):
+            for g in range((T + 7) // 8):
+                words = curand_philox_block(seed, curand_block_of(i, g, bh))
+                for e in range(8):
+                    j = 8 * g + e
+                    if j < T:
+                        u = (words[e >> 1] >> (16 * (e & 1))) & 0xFFFF
+                        assert masks[bh, i, j] == (1 if u >= t else 0), f"mask {bh} ({i},{j}) differs"
+
+
+def check_dropout_mask_statistics(impl):
+    B, H, T = 2, 3, 256
+    for p in (0.1, 0.5):
+        m = impl.dropout_mask(B, H, T, p, seed=11, offset=3)
+        n = m.size
+        keep = 1.0 - _threshold(p) / 65536.0
+        sigma = math.sqrt(n * keep * (1 - keep))
+        assert abs(int(m.sum()) - n * keep) <= 5 * sigma, f"keep rate off for p={p}"
+        assert np.array_equal(m, impl.dropout_mask(B, H, T, p, seed=11, offset=3))
+        flat = m.reshape(B * H, T * T).astype(np.float64)
+        for a, b in ((0, 1), (0, B * H - 1)):
+            assert not np.array_equal(flat[a], flat[b]), "heads must get different masks"
+        # neighbouring elements (same 16-bit word and across words) uncorrelated
+        x = m.reshape(-1, T).astype(np.float64)
+        c = np.corrcoef(x[:, :-1].ravel(), x[:, 1:].ravel())[0, 1]
+        assert abs(c) < 0.01, f"neighbouring keep bits correlated ({c:.3f})"
+    base = impl.dropout_mask(1, 2, 64, 0.5, seed=11, offset=3)
+    assert not np.array_equal(base, impl.dropout_mask(1, 2, 64, 0.5, seed=11, offset=4))
+    assert not np.array_equal(base, impl.dropout_mask(1, 2, 64, 0.5, seed=12, offset=3))
+    assert not np.array_equal(base, impl.dropout_mask(1, 2, 64, 0.5, seed=11 + (1 << 32), offset=3))
+
+
+def check_dropout_zero_threshold_is_plain(impl, seed=21):
+    """p < 1/131072 rounds to threshold 0: every weight kept with scale 1, so
+    the dropout path must give back the plain attention bit for bit."""
+    r = _rng(seed)
+    B, H, T, D = 2, 2, 19, 4
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    for causal in (True, False):
+        o, lse = impl.attn_fwd(q, k, v, causal=causal)
+        o2, lse2 = impl.attn_fwd(q, k, v, causal=causal, dropout_p=1e-6, seed=5, offset=1)
+        assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+        for a, b in zip(impl.attn_bwd(q, k, v, do, causal=causal),
+                        impl.attn_bwd(q, k, v, do, causal=causal, dropout_p=1e-6, seed=5, offset=1)):
+            assert np.array_equal(a, b)
+
+
+def check_dropout_uniform_closed_form(impl, seed=22):
+    """Q = 0: the weights are uniform over the visible keys, so O_i is the keep
+    scale times the mean over the visible keys of M_ij v_j; lse is unchanged."""
+    r = _rng(seed)
+    B, H, T, D = 2, 2, 23, 5
+    k, v = r.standard_normal((B, H, T, D)), r.standard_normal((B, H, T, D))
+    zero = np.zeros_like(k)
+    p, sd, off = 0.25, 99, 7
+    c = 65536.0 / (65536.0 - _threshold(p))
+    m = impl.dropout_mask(B, H, T, p, sd, off).astype(np.float64)
+    for causal in (True, False):
+        vis = np.tril(np.ones((T, T))) if causal else np.ones((T, T))
+        n = vis.sum(-1)
+        o, lse = impl.attn_fwd(zero, k, v, causal=causal, dropout_p=p, seed=sd, offset=off)
+        ref = c * np.einsum("bhij,bhjd->bhid", m * vis, v) / n[:, None]
+        np.testing.assert_allclose(o, ref, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse, np.broadcast_to(np.log(n), lse.shape), rtol=0, atol=1e-14)
+
+
+def check_dropout_unbiased(impl, seed=23):
+    """Over many seeds the dropped output and dV average to the plain ones."""
+    r = _rng(seed)
+    B, H, T, D = 1, 1, 6, 3
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    o_ref, _ = impl.attn_fwd(q, k, v, causal=False)
+    dv_ref = impl.attn_bwd(q, k, v, do, causal=False)[2]
+    N = 600
+    os_, dvs = [], []
+    for s in range(N):
+        os_.append(impl.attn_fwd(q, k, v, causal=False, dropout_p=0.5, seed=s)[0])
+        dvs.append(impl.attn_bwd(q, k, v, do, causal=False, dropout_p=0.5, seed=s)[2])
+    for samples, ref, name in ((np.array(os_), o_ref, "O"), (np.array(dvs), dv_ref, "dV")):
+        mean, sd = samples.mean(0), samples.std(0) + 1e-12
+        z = np.abs(mean - ref) / (sd / math.sqrt(N))
+        assert np.all(z < 5.0), f"E[{name}] with dropout differs from {name} (max z {z.max():.1f})"
+
+
+def check_dropout_finite_differences(impl, seed=24):
+    r = _rng(seed)
+    B, H, T, D = 1, 2, 6, 3
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    kw = dict(dropout_p=0.3, seed=77, offset=2)
+    for causal in (True, False):
+        dq, dk, dv = impl.attn_bwd(q, k, v, do, causal=causal, **kw)
+
+        def loss(q_, k_, v_):
+            return float(np.sum(impl.attn_fwd(q_, k_, v_, causal=causal, **kw)[0] * do))
+
+        h = 1e-6
+        for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+            fd = np.zeros_like(grad)
+            for idx in np.ndindex(*grad.shape):
+                args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+                args[which][idx] += h
+                lp = loss(args["q"], args["k"], args["v"])
+                args[which][idx] -= 2 * h
+                lm = loss(args["q"], args["k"], args["v"])
+                fd[idx] = (lp - lm) / (2 * h)
+            err = np.linalg.norm(fd - grad) / max(np.linalg.norm(grad), 1e-300)
+            assert err <= 1e-7, f"dropout d{which} (causal={causal}): rel {err:.2e}"
+
+
+def check_dropout_torch_witness(impl, seed=25):
+    """torch float64 autograd of softmax -> keep mask * scale -> @ V."""
+    import torch
+    r = _rng(seed)
+    B, H, T, D = 2, 2, 37, 8
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    p, sd, off = 0.2, 1234, 5
+    c = 65536.0 / (65536.0 - _threshold(p))
+    m = torch.tensor(impl.dropout_mask(B, H, T, p, sd, off), dtype=torch.float64)
+    for causal in (True, False):
+        tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+        s = tq @ tk.transpose(-1, -2) / math.sqrt(D)
+        if causal:
+            s = s.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), float("-inf"))
+        lse_t = torch.logsumexp(s, -1)
+        o_t = (torch.softmax(s, -1) * m * c) @ tv
+        o_t.backward(torch.tensor(do))
+        o, lse = impl.attn_fwd(q, k, v, causal=causal, dropout_p=p, seed=sd, offset=off)
+        np.testing.assert_allclose(o, o_t.detach().numpy(), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, lse_t.detach().numpy(), rtol=0, atol=1e-12)
+        grads = impl.attn_bwd(q, k, v, do, causal=causal, dropout_p=p, seed=sd, offset=off)
+        for mine, ref in zip(grads, (tq.grad, tk.grad, tv.grad)):
+            np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-12)
+
+
+DROPOUT_PINS = [check_philox_against_curand, check_dropout_mask_against_curand,
+                check_dropout_mask_statistics, check_dropout_zero_threshold_is_plain,
+                check_dropout_uniform_closed_form, check_dropout_unbiased,
+                check_dropout_finite_differences, check_dropout_torch_witness]
+ALL_PINS = ALL_PINS + DROPOUT_PINS
