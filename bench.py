@@ -53,6 +53,8 @@ def parse_args():
                    help="skip the secondary measurement on c_attn-layout (strided) buffers")
     p.add_argument("--no-noncausal", action="store_true",
                    help="skip the secondary measurement of the non-causal variant")
+    p.add_argument("--no-dropout", action="store_true",
+                   help="skip the secondary measurement with attention dropout 0.1")
     p.add_argument("--layers", type=int, default=None,
                    help="layer instances per step (default: the workload's 12); fewer only for profiling")
     return p.parse_args()
@@ -445,50 +447,57 @@ def run_ours(args, w):
                    "layout": "q,k,v slices of [B,T,3C]; O, dO [B,T,C]; dq|dk|dv into [B,T,3C]"}
         del pk
 
-    # ---- secondary: the non-causal variant (every query sees all T keys) on
-    # the same buffers, through the _ex entry points; FLOPs 12 * D per pair
-    # over all B*H*T*T pairs
-    noncausal = None
-    if not args.no_noncausal:
-        n_nc = max(3, min(args.steps, 30))
-        evn = [([(mk(), mk()) for _ in range(L)], [(mk(), mk()) for _ in range(L)]) for _ in range(n_nc)]
+    # ---- secondary legs on the same buffers through the _ex entry points:
+    # the non-causal variant (every query sees all T keys; FLOPs 12 * D over
+    # all B*H*T*T pairs) and attention dropout at rate 0.1 (a fresh keep mask
+    # per layer and step; the generator's work is not credited)
+    def variant_leg(causal, dropout_p):
+        n_v = max(3, min(args.steps, 30))
+        evn = [([(mk(), mk()) for _ in range(L)], [(mk(), mk()) for _ in range(L)]) for _ in range(n_v + 1)]
         for e in evn:
             for pair in e[0] + e[1]:
                 for x in pair:
                     x.record(stream)
 
-        def nc_step(ev_fwd=None, ev_bwd=None):
+        def v_step(it, ev_fwd=None, ev_bwd=None):
             for l, b in enumerate(layers):
                 if ev_fwd is not None:
                     A.attn_profile_next_call(*ev_fwd[l])
-                A.attn_fwd_ex(b["q"], b["k"], b["v"], b["o"], b["lse"], causal=False)
+                A.attn_fwd_ex(b["q"], b["k"], b["v"], b["o"], b["lse"], causal=causal,
+                              dropout_p=dropout_p, seed=args.seed + 1, offset=it * L + l)
             for l in range(L - 1, -1, -1):
                 b = layers[l]
                 if ev_bwd is not None:
                     A.attn_profile_next_call(*ev_bwd[l])
                 A.attn_bwd_ex(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"],
-                              b["dv"], causal=False, workspace=b["ws"])
-        nc_step()
+                              b["dv"], causal=causal, dropout_p=dropout_p, seed=args.seed + 1,
+                              offset=it * L + l, workspace=b["ws"])
+        v_step(0)
         barrier()
         s0, s1 = mk(), mk()
         s0.record(stream)
-        for i in range(n_nc):
-            nc_step(*evn[i])
+        for i in range(n_v):
+            v_step(i + 1, *evn[i])
         s1.record(stream)
         barrier()
         if A.attn_device_error() != 0:
-            raise RuntimeError("a bounded in-kernel wait timed out in the non-causal leg")
-        nc_ms = reduce_max(s0.elapsed_time(s1), world, dev)
-        pairs_nc = w.B * w.H * w.T * w.T
-        nf = statistics.mean(a.elapsed_time(b) for e in evn for a, b in e[0])
-        nb = statistics.mean(a.elapsed_time(b) for e in evn for a, b in e[1])
-        noncausal = {"value": whole_job_tflops(12 * w.D * pairs_nc * L, world, n_nc, nc_ms),
-                     "unit": "TFLOP/s", "ms_per_step": nc_ms / n_nc, "steps": n_nc,
-                     "flops_per_layer": 12 * w.D * pairs_nc,
-                     "fwd_main": {"avg_launch_ms": nf, "tflops": 4 * w.D * pairs_nc / (nf * 1e-3) / 1e12,
-                                  "frac": 4 * w.D * pairs_nc / (nf * 1e-3) / 1e12 / peak},
-                     "bwd_main": {"avg_launch_ms": nb, "tflops": 8 * w.D * pairs_nc / (nb * 1e-3) / 1e12,
-                                  "frac": 8 * w.D * pairs_nc / (nb * 1e-3) / 1e12 / peak}}
+            raise RuntimeError("a bounded in-kernel wait timed out in a secondary leg")
+        v_ms = reduce_max(s0.elapsed_time(s1), world, dev)
+        pairs_v = w.causal_pairs() if causal else w.B * w.H * w.T * w.T
+        nf = statistics.mean(a.elapsed_time(b) for e in evn[:n_v] for a, b in e[0])
+        nb = statistics.mean(a.elapsed_time(b) for e in evn[:n_v] for a, b in e[1])
+        tf = lambda fl, ms_: fl / (ms_ * 1e-3) / 1e12
+        return {"value": whole_job_tflops(12 * w.D * pairs_v * L, world, n_v, v_ms),
+                "unit": "TFLOP/s", "ms_per_step": v_ms / n_v, "steps": n_v,
+                "causal": causal, "dropout_p": dropout_p,
+                "flops_per_layer": 12 * w.D * pairs_v,
+                "fwd_main": {"avg_launch_ms": nf, "tflops": tf(4 * w.D * pairs_v, nf),
+                             "frac": tf(4 * w.D * pairs_v, nf) / peak},
+                "bwd_main": {"avg_launch_ms": nb, "tflops": tf(8 * w.D * pairs_v, nb),
+                             "frac": tf(8 * w.D * pairs_v, nb) / peak}}
+
+    noncausal = None if args.no_noncausal else variant_leg(False, 0.0)
+    dropout = None if args.no_dropout else variant_leg(True, 0.1)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -505,7 +514,7 @@ def run_ours(args, w):
                             "measured_sustained": value / world / float(peaks.get("bf16_tflops_sustained", peak)),
                             "datasheet_2250": value / world / 2250.0},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "strided_io": strided,
-            "noncausal": noncausal,
+            "noncausal": noncausal, "dropout": dropout,
             "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -51,8 +51,11 @@ _lib.attn_fwd_strided.restype = _i
 _lib.attn_bwd_strided.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _sp, _vp, _sz, _vp]
 _lib.attn_bwd_strided.restype = _i
 class attn_options(ctypes.Structure):
-    """Options of the _ex entry points (include/attn.h): the mask."""
-    _fields_ = [("causal", ctypes.c_int32)]
+    """Options of the _ex entry points (include/attn.h): the mask and
+    attention dropout."""
+    _fields_ = [("causal", ctypes.c_int32), ("dropout_p", ctypes.c_float),
+                ("dropout_seed", ctypes.c_uint64), ("dropout_offset", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32)]
 
 
 _op = ctypes.POINTER(attn_options)
@@ -337,9 +340,9 @@ def attn_bwd_strided(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Opti
     return dq, dk, dv
 
 
-def _options(causal: bool):
-    opts = attn_options(1 if causal else 0)
-    return opts
+def _options(causal: bool, dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+    return attn_options(1 if causal else 0, float(dropout_p), int(seed) & (2**64 - 1),
+                        int(offset) & 0xFFFFFFFF, 0)
 
 
 def _all_contiguous(*tensors) -> bool:
@@ -347,10 +350,12 @@ def _all_contiguous(*tensors) -> bool:
 
 
 def attn_fwd_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = True,
-                stream=None):
+                dropout_p: float = 0.0, seed: int = 0, offset: int = 0, stream=None):
     """bf16 forward with options: ``causal=False`` drops the mask (every query
-    sees all T keys).  Contiguous or strided [B, H, T, D] views; O defaults to
-    the layout of q (contiguous, else a [B, T, C] buffer).  Returns (O, lse)."""
+    sees all T keys); ``dropout_p`` > 0 drops attention weights with the
+    Philox keep mask of (seed, offset).  Contiguous or strided [B, H, T, D]
+    views; O defaults to the layout of q (contiguous, else a [B, T, C]
+    buffer).  Returns (O, lse)."""
     torch = _torch()
     B, H, T, D = _shape4(q)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -361,7 +366,7 @@ def attn_fwd_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal
             _check_view(v, "v", q.shape), _check_view(o, "o", q.shape),
             _check(lse, "lse", torch.float32, (B, H, T))]
     st = None if _all_contiguous(q, k, v, o) else _strides_of(q, k, v, o)
-    opts = _options(causal)
+    opts = _options(causal, dropout_p, seed, offset)
     with torch.cuda.device(q.device):
         _raise(_lib.attn_fwd_ex(*ptrs, B, H, T, D, scale, st, ctypes.byref(opts),
                                 _stream_handle(stream)), "attn_fwd_ex")
@@ -369,9 +374,11 @@ def attn_fwd_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal
 
 
 def attn_bwd_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[float] = None,
-                causal: bool = True, workspace=None, stream=None):
-    """bf16 backward with options (``causal`` as given to attn_fwd_ex), on
-    contiguous or strided views.  Returns (dQ, dK, dV)."""
+                causal: bool = True, dropout_p: float = 0.0, seed: int = 0, offset: int = 0,
+                workspace=None, stream=None):
+    """bf16 backward with options (the same ``causal``, ``dropout_p``, ``seed``
+    and ``offset`` as given to attn_fwd_ex), on contiguous or strided views.
+    Returns (dQ, dK, dV)."""
     torch = _torch()
     B, H, T, D = _shape4(q)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -390,7 +397,7 @@ def attn_bwd_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[
             _check_view(dv, "dv", q.shape)]
     views = (q, k, v, o, dO, dq, dk, dv)
     st = None if _all_contiguous(*views) else _strides_of(*views)
-    opts = _options(causal)
+    opts = _options(causal, dropout_p, seed, offset)
     ws_bytes = workspace.numel() * workspace.element_size()
     with torch.cuda.device(q.device):
         _raise(_lib.attn_bwd_ex(*ptrs, B, H, T, D, scale, st, ctypes.byref(opts),
@@ -400,18 +407,19 @@ def attn_bwd_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[
 
 
 def attn_fwd_f32_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = True,
-                    stream=None):
+                    dropout_p: float = 0.0, seed: int = 0, offset: int = 0, stream=None):
     """float32 forward with options (contiguous tensors).  Returns (O, lse)."""
-    opts = _options(causal)
+    opts = _options(causal, dropout_p, seed, offset)
     fn = lambda *a: _lib.attn_fwd_f32_ex(*a[:-1], ctypes.byref(opts), a[-1])
     fn.__name__ = "attn_fwd_f32_ex"
     return _fwd(fn, _torch().float32, q, k, v, o, lse, scale, stream)
 
 
 def attn_bwd_f32_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[float] = None,
-                    causal: bool = True, workspace=None, stream=None):
+                    causal: bool = True, dropout_p: float = 0.0, seed: int = 0, offset: int = 0,
+                    workspace=None, stream=None):
     """float32 backward with options (contiguous tensors).  Returns (dQ, dK, dV)."""
-    opts = _options(causal)
+    opts = _options(causal, dropout_p, seed, offset)
     fn = lambda *a: _lib.attn_bwd_f32_ex(*a[:-3], ctypes.byref(opts), *a[-3:])
     fn.__name__ = "attn_bwd_f32_ex"
     return _bwd(fn, _lib.attn_bwd_f32_workspace_bytes, _torch().float32, q, k, v, o, lse, dO, dq,

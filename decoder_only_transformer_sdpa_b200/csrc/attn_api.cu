@@ -136,13 +136,41 @@ bool strides_ok(const attn_strides &x) {
 
 TStrides to_tstrides(const attn_strides &x) { return TStrides{x.b, x.h, x.t}; }
 
-// Reads the options (NULL = the decoder's defaults) into `causal`.
-int read_options(const attn_options *opts, int &causal) {
-    causal = 1;
+// The options of one call, as the kernels take them.
+struct Opts {
+    int causal = 1;
+    bool dropout = false;
+    DropoutParams drop{};
+};
+
+// Reads the options (NULL = the decoder's defaults: causal, no dropout).
+int read_options(const attn_options *opts, Opts &out) {
+    out = Opts{};
     if (!opts) return ATTN_OK;
     if (opts->causal != 0 && opts->causal != 1) return ATTN_ERR_OPTION;
-    causal = opts->causal;
+    if (opts->reserved != 0) return ATTN_ERR_OPTION;
+    const double p = opts->dropout_p;
+    if (!(p >= 0.0 && p < 1.0)) return ATTN_ERR_OPTION;  // also rejects NaN
+    const double t = floor(p * 65536.0 + 0.5);
+    if (t >= 65536.0) return ATTN_ERR_OPTION;
+    out.causal = opts->causal;
+    if (t > 0.0) {  // threshold 0 keeps every weight with scale 1: no dropout
+        out.dropout = true;
+        out.drop.k0 = (uint32_t)opts->dropout_seed;
+        out.drop.k1 = (uint32_t)(opts->dropout_seed >> 32);
+        out.drop.thr = (uint32_t)t;
+        out.drop.offset = opts->dropout_offset;
+        out.drop.keep_scale = (float)(65536.0 / (65536.0 - t));
+    }
     return ATTN_OK;
+}
+
+Shape make_shape(int B, int H, int T, int D, float scale, const Opts &op) {
+    Shape s{B, H, T, D, scale};
+    s.causal = op.causal;
+    s.dropout = op.dropout;
+    s.drop = op.drop;
+    return s;
 }
 
 int fwd_strides(const attn_strides *strides, const Shape &s, FwdStrides &str) {
@@ -172,7 +200,7 @@ int bwd_strides(const attn_strides *strides, const Shape &s, BwdStrides &str) {
 }
 
 int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int T,
-             int D, float scale, int causal, const FwdStrides &str, cudaStream_t stream,
+             int D, float scale, const Opts &op, const FwdStrides &str, cudaStream_t stream,
              LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 64);
@@ -185,13 +213,13 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     if ((st = device_setup(&err)) != ATTN_OK) return st;
     cudaError_t e = sm100_fwd(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
                               static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), lse,
-                              Shape{B, H, T, D, scale, causal}, str, err, stream, li);
+                              make_shape(B, H, T, D, scale, op), str, err, stream, li);
     return finish(e, li);
 }
 
 int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
              const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D, float scale,
-             int causal, const BwdStrides &str, void *workspace, size_t workspace_bytes,
+             const Opts &op, const BwdStrides &str, void *workspace, size_t workspace_bytes,
              cudaStream_t stream, LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 64);
@@ -216,7 +244,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
         static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(o), lse,
         static_cast<const __nv_bfloat16 *>(dO), static_cast<__nv_bfloat16 *>(dq),
         static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv), dq_acc, lse2, delta,
-        Shape{B, H, T, D, scale, causal}, str, err, stream, li);
+        make_shape(B, H, T, D, scale, op), str, err, stream, li);
     return finish(e, li);
 }
 
@@ -226,11 +254,12 @@ ATTN_API int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, f
                          int H, int T, int D, float scale, const attn_strides *strides,
                          const attn_options *opts, cudaStream_t stream) {
     LaunchInfo li = take_launch_info();
-    int causal, st;
-    if ((st = read_options(opts, causal)) != ATTN_OK) return st;
+    Opts op;
+    int st;
+    if ((st = read_options(opts, op)) != ATTN_OK) return st;
     FwdStrides str;
     if ((st = fwd_strides(strides, Shape{B, H, T, D, scale}, str)) != ATTN_OK) return st;
-    return fwd_impl(q, k, v, o, lse, B, H, T, D, scale, causal, str, stream, li);
+    return fwd_impl(q, k, v, o, lse, B, H, T, D, scale, op, str, stream, li);
 }
 
 ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
@@ -260,11 +289,12 @@ ATTN_API int attn_bwd_ex(const void *q, const void *k, const void *v, const void
                          const attn_options *opts, void *workspace, size_t workspace_bytes,
                          cudaStream_t stream) {
     LaunchInfo li = take_launch_info();
-    int causal, st;
-    if ((st = read_options(opts, causal)) != ATTN_OK) return st;
+    Opts op;
+    int st;
+    if ((st = read_options(opts, op)) != ATTN_OK) return st;
     BwdStrides str;
     if ((st = bwd_strides(strides, Shape{B, H, T, D, scale}, str)) != ATTN_OK) return st;
-    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, causal, str, workspace,
+    return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, op, str, workspace,
                     workspace_bytes, stream, li);
 }
 
@@ -291,8 +321,9 @@ ATTN_API int attn_fwd_f32_ex(const float *q, const float *k, const float *v, flo
                              int B, int H, int T, int D, float scale, const attn_options *opts,
                              cudaStream_t stream) {
     LaunchInfo li = take_launch_info();
-    int causal, st0;
-    if ((st0 = read_options(opts, causal)) != ATTN_OK) return st0;
+    Opts op;
+    int st0;
+    if ((st0 = read_options(opts, op)) != ATTN_OK) return st0;
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 128);
     if (st != ATTN_OK) return st;
@@ -300,7 +331,7 @@ ATTN_API int attn_fwd_f32_ex(const float *q, const float *k, const float *v, flo
     if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(o, 4) || !aligned(lse, 4))
         return ATTN_ERR_ALIGN;
     if ((st = device_setup(nullptr)) != ATTN_OK) return st;
-    cudaError_t e = simt_fwd<float>(q, k, v, o, lse, Shape{B, H, T, D, scale, causal}, stream, li);
+    cudaError_t e = simt_fwd<float>(q, k, v, o, lse, make_shape(B, H, T, D, scale, op), stream, li);
     return finish(e, li);
 }
 
@@ -319,8 +350,9 @@ ATTN_API int attn_bwd_f32_ex(const float *q, const float *k, const float *v, con
                              int B, int H, int T, int D, float scale, const attn_options *opts,
                              void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     LaunchInfo li = take_launch_info();
-    int causal, st0;
-    if ((st0 = read_options(opts, causal)) != ATTN_OK) return st0;
+    Opts op;
+    int st0;
+    if ((st0 = read_options(opts, op)) != ATTN_OK) return st0;
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 128);
     if (st != ATTN_OK) return st;
@@ -332,7 +364,7 @@ ATTN_API int attn_bwd_f32_ex(const float *q, const float *k, const float *v, con
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
     if ((st = device_setup(nullptr)) != ATTN_OK) return st;
     cudaError_t e = simt_bwd<float>(q, k, v, o, lse, dO, dq, dk, dv, static_cast<float *>(workspace),
-                                    Shape{B, H, T, D, scale, causal}, stream, li);
+                                    make_shape(B, H, T, D, scale, op), stream, li);
     return finish(e, li);
 }
 

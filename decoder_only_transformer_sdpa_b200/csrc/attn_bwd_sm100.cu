@@ -42,6 +42,12 @@
 // dS^T tile).  The next tile's S^T / dP^T are issued as soon as the current
 // ones have been read out of TMEM, so they overlap the elementwise work.
 //
+// With attention dropout (Drop) the keep bit of (query i, key j) is the one
+// the forward drew (philox.cuh): the eight lanes holding keys 8g .. 8g+7 each
+// draw the bits of four queries for all eight keys and trade them with
+// shuffles; P^T in TMEM keeps only the kept weights (dV is scaled by the keep
+// scale at the end) and dS^T = P^T (keep_scale M dP^T - Delta).
+//
 // TMEM columns: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D),
 // dQ [256+2D, 256+3D), P^T (bf16 pairs) [256+3D, 256+3D+64).
 #include "internal.h"
@@ -155,7 +161,7 @@ __global__ void bwd_post_kernel(const float4 *__restrict__ acc, __nv_bfloat16 *_
 
 // ------------------------------------------------------------------ main
 
-template <int D, bool Causal>
+template <int D, bool Causal, bool Drop>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
@@ -163,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float *__restrict__ delta, __nv_bfloat16 *__restrict__ dk,
                     __nv_bfloat16 *__restrict__ dv, const TStrides sdk, const TStrides sdv,
                     int T, int Tpad, int H, int BH, int nt, float scale_log2, float scale,
-                    int *err) {
+                    const DropoutParams dp, int *err) {
     using Smem = BwdSmem<D>;
     constexpr int kRowBytes = D * 2;
     constexpr uint32_t kSwz = (D == 64) ? kSwizzle128B : kSwizzle64B;
@@ -335,6 +341,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_before();
                     mbar_arrive(&sm.sdp_free);
                 }
+                // keep bit of query q0 + x for this thread's key: bit x of keepm
+                uint32_t keepm = 0xFFFFFFFFu;
+                if constexpr (Drop) {
+                    const uint32_t sub = (uint32_t)(lane & 7);
+                    const uint32_t jg = (uint32_t)((kt * kBT + quad * 32 + (lane & ~7)) >> 3);
+                    const uint32_t ib = (uint32_t)((q_first + idx) * kBT + q0) + sub;
+                    uint32_t wbits = 0;  // byte r: keys 8 jg .. +7 of query ib + 8 r
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        wbits |= philox::keep_byte(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
+                    keepm = 0;
+#pragma unroll
+                    for (int s = 0; s < 8; ++s) {
+                        const uint32_t w = __shfl_sync(0xffffffffu, wbits, (lane & ~7) | s);
+                        keepm |= ((w >> sub) & 0x01010101u) << s;
+                    }
+                }
                 uint32_t pw[16], dw[16];
 #pragma unroll
                 for (int x = 0; x < 32; x += 4) {
@@ -347,8 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int y = 0; y < 4; ++y) {
                         float pv = ex2(fmaf(__uint_as_float(rs[x + y]), scale_log2, -lv[y]));
                         if (diag && (q0 + x + y) < kr) pv = 0.f;  // query before key: masked
-                        pp[y] = pv;
-                        dd[y] = pv * (__uint_as_float(rp[x + y]) - dvv[y]);
+                        if constexpr (Drop) {
+                            const bool keep = (keepm >> (x + y)) & 1u;
+                            pp[y] = keep ? pv : 0.f;
+                            dd[y] = pv * ((keep ? dp.keep_scale * __uint_as_float(rp[x + y]) : 0.f) - dvv[y]);
+                        } else {
+                            pp[y] = pv;
+                            dd[y] = pv * (__uint_as_float(rp[x + y]) - dvv[y]);
+                        }
                     }
                     pw[x / 2] = pack_bf16x2(pp[0], pp[1]);
                     pw[x / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
@@ -386,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int t = kt * kBT + kr;
             const uint32_t src = half == 0 ? tdK : tdV;
-            const float mul = half == 0 ? scale : 1.f;
+            const float mul = half == 0 ? scale : (Drop ? dp.keep_scale : 1.f);
             const TStrides so = half == 0 ? sdk : sdv;
             __nv_bfloat16 *out = (half == 0 ? dk : dv) + (long long)bb * so.b + (long long)hh * so.h +
                                  (long long)t * so.t;
@@ -475,7 +504,7 @@ cudaError_t make_map(CUtensorMap *map, const void *ptr, int BH, int T, int D, bo
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, bool Causal>
+template <int D, bool Causal, bool Drop>
 cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                        const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                        __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
@@ -502,13 +531,13 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     li.kernels += 1;
 
     const size_t smem = sizeof(BwdSmem<D>) + 1024;
-    if ((e = cudaFuncSetAttribute(bwd_main_kernel<D, Causal>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(bwd_main_kernel<D, Causal, Drop>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    bwd_main_kernel<D, Causal><<<(unsigned)blocks, kThreads, smem, st>>>(
+    bwd_main_kernel<D, Causal, Drop><<<(unsigned)blocks, kThreads, smem, st>>>(
         mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, str.dk, str.dv, s.T, Tpad, s.H, BH, nt,
-        s.scale * kLog2e, s.scale, err);
+        s.scale * kLog2e, s.scale, s.drop, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
     if ((e = mark_main_end(li, st)) != cudaSuccess) return e;
@@ -530,14 +559,18 @@ cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
                       float *lse2, float *delta, Shape s, const BwdStrides &str, int *err,
                       cudaStream_t st, LaunchInfo &li) {
-#define ATTN_BWD_CASE(DD)                                                                          \
-    if (s.D == DD)                                                                                 \
-        return s.causal ? launch_bwd<DD, true>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, \
-                                               s, str, err, st, li)                                \
-                        : launch_bwd<DD, false>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2,      \
-                                                delta, s, str, err, st, li);
-    ATTN_BWD_CASE(64)
-    ATTN_BWD_CASE(32)
+#define ATTN_BWD_CASE(DD, C, R)                                                          \
+    if (s.D == DD && (s.causal != 0) == C && s.dropout == R)                             \
+        return launch_bwd<DD, C, R>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, \
+                                    str, err, st, li);
+    ATTN_BWD_CASE(64, true, false)
+    ATTN_BWD_CASE(64, false, false)
+    ATTN_BWD_CASE(64, true, true)
+    ATTN_BWD_CASE(64, false, true)
+    ATTN_BWD_CASE(32, true, false)
+    ATTN_BWD_CASE(32, false, false)
+    ATTN_BWD_CASE(32, true, true)
+    ATTN_BWD_CASE(32, false, true)
 #undef ATTN_BWD_CASE
     return cudaErrorInvalidValue;
 }

@@ -28,7 +28,10 @@
 // Key tiles wholly above the diagonal are never loaded; only the diagonal
 // tile applies the element mask.  The score matrix never leaves the SM.
 // Without the mask (Causal = false) every query tile runs over all key tiles
-// and only the last key tile masks the keys past T.
+// and only the last key tile masks the keys past T.  With dropout (Drop) each
+// softmax thread draws its row's keep bits from Philox4x32-10, eight keys per
+// call (philox.cuh): the row sum l takes every weight, P_j in TMEM only the
+// kept ones, and the final O is scaled by keep_scale / l.
 //
 // TMEM columns: S [0,128), P (bf16 pairs) [128,192), O [192, 192+D).
 #include "internal.h"
@@ -69,12 +72,12 @@ __device__ __forceinline__ int item_of(int c, int n, int G, int W) {
     return w < W ? (int)w : -1;
 }
 
-template <int D, bool Causal>
+template <int D, bool Causal, bool Drop>
 __global__ void __launch_bounds__(kThreads, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16 *__restrict__ o,
                const TStrides so, float *__restrict__ lse, int T, int H, int BH, int ntiles,
-               float scale_log2, int *err) {
+               float scale_log2, const DropoutParams dp, int *err) {
     using Smem = FwdSmem<D>;
     constexpr int kRowBytes = D * 2;                      // 128 (D=64) or 64 (D=32)
     constexpr uint32_t kSwz = (D == 64) ? kSwizzle128B : kSwizzle64B;
@@ -333,13 +336,33 @@ __global__ void __launch_bounds__(kThreads, 2)
                 // of the tile, where the previous PV has had the most time.
                 uint32_t pk[kBN / 2];
                 float la = 0.f, lb = 0.f;
+                if constexpr (Drop) {
+                    // Keep bits of this row, eight keys per generator call.
+                    const uint32_t ti = (uint32_t)(qt * kBM + row);
 #pragma unroll
-                for (int x = 0; x < kBN / 2; ++x) {
-                    const float p0 = ex2(fmaf(s[2 * x], scale_log2, neg_m));
-                    const float p1 = ex2(fmaf(s[2 * x + 1], scale_log2, neg_m));
-                    la += p0;
-                    lb += p1;
-                    pk[x] = pack_bf16x2(p0, p1);
+                    for (int g = 0; g < kBN / 8; ++g) {
+                        const uint32_t kb = philox::keep_byte(dp, ti, (uint32_t)(j * (kBN / 8) + g),
+                                                              (uint32_t)bh);
+#pragma unroll
+                        for (int y = 0; y < 4; ++y) {
+                            const int x = 4 * g + y;
+                            const float p0 = ex2(fmaf(s[2 * x], scale_log2, neg_m));
+                            const float p1 = ex2(fmaf(s[2 * x + 1], scale_log2, neg_m));
+                            la += p0;
+                            lb += p1;
+                            pk[x] = pack_bf16x2((kb >> (2 * y)) & 1u ? p0 : 0.f,
+                                                (kb >> (2 * y + 1)) & 1u ? p1 : 0.f);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < kBN / 2; ++x) {
+                        const float p0 = ex2(fmaf(s[2 * x], scale_log2, neg_m));
+                        const float p1 = ex2(fmaf(s[2 * x + 1], scale_log2, neg_m));
+                        la += p0;
+                        lb += p1;
+                        pk[x] = pack_bf16x2(p0, p1);
+                    }
                 }
                 l += la + lb;
                 if (!pv_done) {
@@ -370,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_arrive(&sm.o_free);
             const int t = qt * kBM + row;
             if (t < T) {
-                const float inv = 1.f / l;
+                const float inv = (Drop ? dp.keep_scale : 1.f) / l;
                 const size_t grow = (size_t)bh * T + t;
                 __nv_bfloat16 *orow = o + (long long)(bh / H) * so.b + (long long)(bh % H) * so.h +
                                       (long long)t * so.t;
@@ -420,7 +443,7 @@ cudaError_t make_map_bf16(void *map, const void *ptr, const Shape &s, const TStr
 
 namespace {
 
-template <int D, bool Causal>
+template <int D, bool Causal, bool Drop>
 cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                        __nv_bfloat16 *o, float *lse, Shape s, const FwdStrides &str, int *err,
                        cudaStream_t st, LaunchInfo &li) {
@@ -440,13 +463,13 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if ((e = make_map_bf16(&mk, k, s, str.k)) != cudaSuccess) return e;
     if ((e = make_map_bf16(&mv, v, s, str.v)) != cudaSuccess) return e;
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
-    if ((e = cudaFuncSetAttribute(fwd_kernel<D, Causal>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(fwd_kernel<D, Causal, Drop>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
     const float scale_log2 = s.scale * 1.4426950408889634f;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    fwd_kernel<D, Causal><<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, o, str.o, lse, s.T, s.H,
-                                                                    BH, ntiles, scale_log2, err);
+    fwd_kernel<D, Causal, Drop><<<(unsigned)grid, kThreads, smem, st>>>(
+        mq, mk, mv, o, str.o, lse, s.T, s.H, BH, ntiles, scale_log2, s.drop, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     li.kernels += 1;
     return mark_main_end(li, st);
@@ -457,12 +480,18 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
 cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       __nv_bfloat16 *o, float *lse, Shape s, const FwdStrides &str, int *err,
                       cudaStream_t st, LaunchInfo &li) {
-    if (s.D == 64)
-        return s.causal ? launch_fwd<64, true>(q, k, v, o, lse, s, str, err, st, li)
-                        : launch_fwd<64, false>(q, k, v, o, lse, s, str, err, st, li);
-    if (s.D == 32)
-        return s.causal ? launch_fwd<32, true>(q, k, v, o, lse, s, str, err, st, li)
-                        : launch_fwd<32, false>(q, k, v, o, lse, s, str, err, st, li);
+#define ATTN_FWD_CASE(DD, C, R)                                    \
+    if (s.D == DD && (s.causal != 0) == C && s.dropout == R)       \
+        return launch_fwd<DD, C, R>(q, k, v, o, lse, s, str, err, st, li);
+    ATTN_FWD_CASE(64, true, false)
+    ATTN_FWD_CASE(64, false, false)
+    ATTN_FWD_CASE(64, true, true)
+    ATTN_FWD_CASE(64, false, true)
+    ATTN_FWD_CASE(32, true, false)
+    ATTN_FWD_CASE(32, false, false)
+    ATTN_FWD_CASE(32, true, true)
+    ATTN_FWD_CASE(32, false, true)
+#undef ATTN_FWD_CASE
     return cudaErrorInvalidValue;
 }
 

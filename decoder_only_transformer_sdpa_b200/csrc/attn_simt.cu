@@ -12,7 +12,10 @@
 // with a running maximum and running sum (online softmax), so the T x T score
 // matrix never exists in memory.  The backward recomputes P_ij from the saved
 // lse_i and follows the exact derivative.  With causal = 0 the same kernels
-// run every row over all T keys (every key over all T queries).
+// run every row over all T keys (every key over all T queries).  With drop
+// set, attention dropout on the weights uses the keep bits of philox.cuh:
+// row sums take every weight, O and dV only the kept ones, scaled by the
+// keep scale.
 //
 // Block = 64 threads = 64 rows of one head; K/V (or Q/dO) tiles of 64 rows
 // are staged in shared memory as float32 and shared by the block.
@@ -52,7 +55,8 @@ template <typename T, int DMAX>
 __global__ void __launch_bounds__(kRows) fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                     const T *__restrict__ v, T *__restrict__ o,
                                                     float *__restrict__ lse, int Tn, int D,
-                                                    float scale, int causal) {
+                                                    float scale, int causal, int drop,
+                                                    DropoutParams dp) {
     extern __shared__ float smem[];
     float *ks = smem;
     float *vs = smem + kRows * D;
@@ -80,9 +84,12 @@ __global__ void __launch_bounds__(kRows) fwd_kernel(const T *__restrict__ q, con
         __syncthreads();
         if (row_ok) {
             const int jend = min(j0 + kRows - 1, my_last);
+            uint32_t kb = 0xFFu;  // keep bits of keys (j & ~7) .. +7
             for (int j = j0; j <= jend; ++j) {
                 const float *kj = ks + (j - j0) * D;
                 const float *vj = vs + (j - j0) * D;
+                if (drop && (j & 7) == 0)
+                    kb = philox::keep_byte(dp, (uint32_t)i, (uint32_t)j >> 3, (uint32_t)bh);
                 float s = 0.f;
 #pragma unroll
                 for (int d = 0; d < DMAX; ++d)
@@ -92,15 +99,16 @@ __global__ void __launch_bounds__(kRows) fwd_kernel(const T *__restrict__ q, con
                 const float corr = expf(m - mn);
                 const float p = expf(s - mn);
                 l = fmaf(l, corr, p);
+                const float pz = ((kb >> (j & 7)) & 1u) ? p : 0.f;
 #pragma unroll
                 for (int d = 0; d < DMAX; ++d)
-                    if (d < D) acc[d] = fmaf(p, vj[d], acc[d] * corr);
+                    if (d < D) acc[d] = fmaf(pz, vj[d], acc[d] * corr);
                 m = mn;
             }
         }
     }
     if (row_ok) {
-        const float inv = 1.f / l;
+        const float inv = (drop ? dp.keep_scale : 1.f) / l;
 #pragma unroll
         for (int d = 0; d < DMAX; ++d)
             if (d < D) from_f(&o[base + (size_t)i * D + d], acc[d] * inv);
@@ -126,7 +134,8 @@ __global__ void __launch_bounds__(kRows) dq_kernel(const T *__restrict__ q, cons
                                                    const T *__restrict__ v, const float *__restrict__ lse,
                                                    const T *__restrict__ dO,
                                                    const float *__restrict__ delta, T *__restrict__ dq,
-                                                   int Tn, int D, float scale, int causal) {
+                                                   int Tn, int D, float scale, int causal, int drop,
+                                                   DropoutParams dp) {
     extern __shared__ float smem[];
     float *ks = smem;
     float *vs = smem + kRows * D;
@@ -156,18 +165,22 @@ __global__ void __launch_bounds__(kRows) dq_kernel(const T *__restrict__ q, cons
         __syncthreads();
         if (row_ok) {
             const int jend = min(j0 + kRows - 1, my_last);
+            uint32_t kb = 0xFFu;
             for (int j = j0; j <= jend; ++j) {
                 const float *kj = ks + (j - j0) * D;
                 const float *vj = vs + (j - j0) * D;
-                float s = 0.f, dp = 0.f;
+                if (drop && (j & 7) == 0)
+                    kb = philox::keep_byte(dp, (uint32_t)i, (uint32_t)j >> 3, (uint32_t)bh);
+                float s = 0.f, dpv = 0.f;
 #pragma unroll
                 for (int d = 0; d < DMAX; ++d)
                     if (d < D) {
                         s = fmaf(qr[d], kj[d], s);
-                        dp = fmaf(gr[d], vj[d], dp);
+                        dpv = fmaf(gr[d], vj[d], dpv);
                     }
                 const float p = expf(s * scale - lse_i);
-                const float ds = p * (dp - delta_i);
+                const float dz = drop ? (((kb >> (j & 7)) & 1u) ? dp.keep_scale * dpv : 0.f) : dpv;
+                const float ds = p * (dz - delta_i);
 #pragma unroll
                 for (int d = 0; d < DMAX; ++d)
                     if (d < D) acc[d] = fmaf(ds, kj[d], acc[d]);
@@ -190,7 +203,8 @@ __global__ void __launch_bounds__(kRows) dkdv_kernel(const T *__restrict__ q, co
                                                      const T *__restrict__ dO,
                                                      const float *__restrict__ delta,
                                                      T *__restrict__ dk, T *__restrict__ dv, int Tn,
-                                                     int D, float scale, int causal) {
+                                                     int D, float scale, int causal, int drop,
+                                                     DropoutParams dp) {
     extern __shared__ float smem[];
     float *qs = smem;
     float *gs = smem + kRows * D;
@@ -232,19 +246,25 @@ __global__ void __launch_bounds__(kRows) dkdv_kernel(const T *__restrict__ q, co
             for (int i = causal ? max(i0, j) : i0; i < iend; ++i) {
                 const float *qi = qs + (i - i0) * D;
                 const float *gi = gs + (i - i0) * D;
-                float s = 0.f, dp = 0.f;
+                float s = 0.f, dpv = 0.f;
 #pragma unroll
                 for (int d = 0; d < DMAX; ++d)
                     if (d < D) {
                         s = fmaf(qi[d], kr[d], s);
-                        dp = fmaf(gi[d], vr[d], dp);
+                        dpv = fmaf(gi[d], vr[d], dpv);
                     }
                 const float p = expf(s * scale - ls[i - i0]);
-                const float dsv = p * (dp - ds_[i - i0]);
+                bool keep = true;
+                if (drop)
+                    keep = (philox::keep_byte(dp, (uint32_t)i, (uint32_t)j >> 3, (uint32_t)bh) >>
+                            (j & 7)) & 1u;
+                const float dz = drop ? (keep ? dp.keep_scale * dpv : 0.f) : dpv;
+                const float dsv = p * (dz - ds_[i - i0]);
+                const float pz = keep ? p : 0.f;
 #pragma unroll
                 for (int d = 0; d < DMAX; ++d)
                     if (d < D) {
-                        dva[d] = fmaf(p, gi[d], dva[d]);
+                        dva[d] = fmaf(pz, gi[d], dva[d]);
                         dka[d] = fmaf(dsv, qi[d], dka[d]);
                     }
             }
@@ -255,7 +275,7 @@ __global__ void __launch_bounds__(kRows) dkdv_kernel(const T *__restrict__ q, co
         for (int d = 0; d < DMAX; ++d)
             if (d < D) {
                 from_f(&dk[base + (size_t)j * D + d], dka[d] * scale);
-                from_f(&dv[base + (size_t)j * D + d], dva[d]);
+                from_f(&dv[base + (size_t)j * D + d], dva[d] * (drop ? dp.keep_scale : 1.f));
             }
     }
 }
@@ -275,10 +295,12 @@ cudaError_t simt_fwd(const T *q, const T *k, const T *v, T *o, float *lse, Shape
     const long long blocks = (long long)s.B * s.H * ntiles;
     const size_t smem = 2ull * kRows * s.D * sizeof(float);
     const void *fn = ATTN_SIMT_DISPATCH(s.D, fwd_kernel, T);
+    int drop = s.dropout ? 1 : 0;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     void *args[] = {(void *)&q, (void *)&k, (void *)&v, (void *)&o, (void *)&lse,
-                    (void *)&s.T, (void *)&s.D, (void *)&s.scale, (void *)&s.causal};
+                    (void *)&s.T, (void *)&s.D, (void *)&s.scale, (void *)&s.causal,
+                    (void *)&drop, (void *)&s.drop};
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     e = cudaLaunchKernel(fn, dim3((unsigned)blocks), dim3(kRows), args, smem, st);
     if (e != cudaSuccess) return e;
@@ -293,6 +315,7 @@ cudaError_t simt_bwd(const T *q, const T *k, const T *v, const T *o, const float
     const long long rows = (long long)s.B * s.H * s.T;
     const int ntiles = (s.T + kRows - 1) / kRows;
     const long long blocks = (long long)s.B * s.H * ntiles;
+    int drop = s.dropout ? 1 : 0;
     delta_kernel<T><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(o, dO, delta, rows, s.D);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -305,7 +328,7 @@ cudaError_t simt_bwd(const T *q, const T *k, const T *v, const T *o, const float
     const float *delta_c = delta;
     void *a1[] = {(void *)&q, (void *)&k, (void *)&v, (void *)&lse, (void *)&dO,
                   (void *)&delta_c, (void *)&dq, (void *)&s.T, (void *)&s.D, (void *)&s.scale,
-                  (void *)&s.causal};
+                  (void *)&s.causal, (void *)&drop, (void *)&s.drop};
     e = cudaLaunchKernel(fdq, dim3((unsigned)blocks), dim3(kRows), a1, smem_dq, st);
     if (e != cudaSuccess) return e;
     li.kernels += 1;
@@ -316,7 +339,7 @@ cudaError_t simt_bwd(const T *q, const T *k, const T *v, const T *o, const float
     if (e != cudaSuccess) return e;
     void *a2[] = {(void *)&q, (void *)&k, (void *)&v, (void *)&lse, (void *)&dO,
                   (void *)&delta_c, (void *)&dk, (void *)&dv, (void *)&s.T, (void *)&s.D,
-                  (void *)&s.scale, (void *)&s.causal};
+                  (void *)&s.scale, (void *)&s.causal, (void *)&drop, (void *)&s.drop};
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     e = cudaLaunchKernel(fkv, dim3((unsigned)blocks), dim3(kRows), a2, smem_kv, st);
     if (e != cudaSuccess) return e;

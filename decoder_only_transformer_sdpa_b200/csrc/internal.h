@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "philox.cuh"
+
 namespace attn {
 
 // Upper bound on the polls of any in-kernel wait (mbarrier or flag).  A wait
@@ -20,7 +22,9 @@ constexpr int kErrTimeout = 1;
 struct Shape {
     int B, H, T, D;
     float scale;
-    int causal = 1;  // 1: key j visible to query i iff j <= i; 0: all keys visible
+    int causal = 1;        // 1: key j visible to query i iff j <= i; 0: all keys visible
+    bool dropout = false;  // attention dropout on the weights (drop.thr > 0)
+    DropoutParams drop{};
 };
 
 // Element strides of a [B, H, T, D] view (the d stride is 1).  Contiguous

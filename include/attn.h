@@ -151,10 +151,11 @@ int attn_bwd_strided(const void *q, const void *k, const void *v, const void *o,
                      int B, int H, int T, int D, float scale, const attn_strides *strides,
                      void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
-/* ---------------- options: the mask ------------------------------------- */
+/* ---------------- options: the mask and attention dropout --------------- */
 
 /* Options of the _ex entry points.  A NULL options pointer means the
- * defaults, which are the decoder's attention computed by attn_fwd/attn_bwd.
+ * defaults, which are the decoder's attention computed by attn_fwd/attn_bwd
+ * (causal, no dropout).
  *
  * causal: 1 (default) masks key j for query i when j > i -- the -inf upper
  *   triangle that keeps a decoder token from seeing later tokens ("How Andrej
@@ -162,9 +163,31 @@ int attn_bwd_strided(const void *q, const void *k, const void *v, const void *o,
  *   mathematical trick" [55:20]).  0 drops the mask: every query attends to
  *   all T keys (the encoder-style attention that the same passage contrasts
  *   with the decoder's), lse_i = ln sum_{j<T} exp(S_ij), and the backward
- *   sums over all i and j.  Any other value gives ATTN_ERR_OPTION. */
+ *   sums over all i and j.  Any other value gives ATTN_ERR_OPTION.
+ *
+ * dropout_p, dropout_seed, dropout_offset: attention dropout on the weights
+ *   after the softmax, before they meet the values.  The pages train with a
+ *   dropout rate ("GPT da zero", table "Come funziona": 0.1) without saying
+ *   where in attention it acts; here it is the plain reading, weights zeroed
+ *   at random and the kept ones rescaled.  Element (i, j) of head b*H + h is
+ *   kept iff 16-bit lane (j mod 8) of Philox4x32-10 (Salmon et al., "Parallel
+ *   Random Numbers: As Easy as 1, 2, 3", SC 2011) at counter
+ *   (i, j / 8, b*H + h, dropout_offset) under key (low, high word of
+ *   dropout_seed) is >= t = floor(dropout_p * 65536 + 1/2); lane e is bits
+ *   16 (e mod 2) .. +15 of output word e / 2.  Kept weights are scaled by
+ *   65536 / (65536 - t), so p acts rounded to a multiple of 1/65536.
+ *   lse stays the log-sum-exp of the undropped scores.  Pass the same seed
+ *   and offset to the backward; use a new offset (or seed) per call that
+ *   needs a fresh mask (each layer, each step).  0 <= dropout_p < 1 with
+ *   t < 65536, else ATTN_ERR_OPTION; t = 0 (p < 1/131072) is no dropout.
+ *
+ * reserved: must be 0 (ATTN_ERR_OPTION otherwise). */
 typedef struct {
     int32_t causal;
+    float dropout_p;
+    uint64_t dropout_seed;
+    uint32_t dropout_offset;
+    uint32_t reserved;
 } attn_options;
 
 /* attn_fwd with options, on strided views.  strides: NULL for contiguous

@@ -63,10 +63,11 @@ class OracleLib:
                                             ctypes.POINTER(ctypes.c_uint8)]
         lib.oracle_dropout_mask.restype = None
         lib.oracle_attn_fwd_dropout.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, ctypes.c_double, i,
-                                                ctypes.c_double, u64, u32]
+                                                ctypes.c_double, u64, u32, ctypes.c_int64]
         lib.oracle_attn_fwd_dropout.restype = None
         lib.oracle_attn_bwd_dropout.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i,
-                                                ctypes.c_double, i, ctypes.c_double, u64, u32]
+                                                ctypes.c_double, i, ctypes.c_double, u64, u32,
+                                                ctypes.c_int64]
         lib.oracle_attn_bwd_dropout.restype = None
         lib.oracle_threads.argtypes = []
         lib.oracle_threads.restype = i
@@ -75,8 +76,10 @@ class OracleLib:
     def _fn(self, name: str, causal: bool):
         return getattr(self.lib, name if causal else name + "_nc")
 
-    def attn_fwd(self, q, k, v, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0):
-        """Returns (O [B,H,T,D], lse [B,H,T]) in float64."""
+    def attn_fwd(self, q, k, v, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0,
+                 head0=0):
+        """Returns (O [B,H,T,D], lse [B,H,T]) in float64.  With dropout, head0
+        is the flat head index (b*H + h) of q's first head in the full call."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, H, T, D = _shape(q)
         scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
@@ -85,7 +88,7 @@ class OracleLib:
         if dropout_p:
             self.lib.oracle_attn_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D,
                                              scale, int(bool(causal)), float(dropout_p), int(seed),
-                                             int(offset))
+                                             int(offset), int(head0))
             return o, lse
         self._fn("oracle_attn_fwd", causal)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                             B, H, T, D, scale)
@@ -100,7 +103,8 @@ class OracleLib:
         self._fn("oracle_attn_probs", causal)(_ptr(q), _ptr(k), _ptr(p), B, H, T, D, scale)
         return p
 
-    def attn_bwd(self, q, k, v, do, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0):
+    def attn_bwd(self, q, k, v, do, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0,
+                 head0=0):
         """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
         q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
         B, H, T, D = _shape(q)
@@ -109,7 +113,7 @@ class OracleLib:
         if dropout_p:
             self.lib.oracle_attn_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk),
                                              _ptr(dv), B, H, T, D, scale, int(bool(causal)),
-                                             float(dropout_p), int(seed), int(offset))
+                                             float(dropout_p), int(seed), int(offset), int(head0))
             return dq, dk, dv
         self._fn("oracle_attn_bwd", causal)(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq),
                                             _ptr(dk), _ptr(dv), B, H, T, D, scale)
@@ -160,9 +164,9 @@ def _shape(q: np.ndarray):
     return tuple(int(s) for s in q.shape)
 
 
-def attn_fwd(q, k, v, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0):
+def attn_fwd(q, k, v, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0, head0=0):
     """Returns (O [B,H,T,D], lse [B,H,T]) in float64."""
-    return _load().attn_fwd(q, k, v, scale, causal, dropout_p, seed, offset)
+    return _load().attn_fwd(q, k, v, scale, causal, dropout_p, seed, offset, head0)
 
 
 def attn_probs(q, k, scale=None, causal=True):
@@ -170,9 +174,9 @@ def attn_probs(q, k, scale=None, causal=True):
     return _load().attn_probs(q, k, scale, causal)
 
 
-def attn_bwd(q, k, v, do, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0):
+def attn_bwd(q, k, v, do, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0, head0=0):
     """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
-    return _load().attn_bwd(q, k, v, do, scale, causal, dropout_p, seed, offset)
+    return _load().attn_bwd(q, k, v, do, scale, causal, dropout_p, seed, offset, head0)
 
 
 def philox4x32_10(ctr, key):

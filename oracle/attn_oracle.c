@@ -142,21 +142,24 @@ static int keep_bit(uint64_t seed, uint32_t offset, int64_t bh, int i, int j, ui
     return u >= t;
 }
 
-/* Dropout parameters of one call; p = 0 means no dropout. */
+/* Dropout parameters of one call; p = 0 means no dropout.  head0 is the flat
+ * head index (b * H + h) of the first head held by the tensors, so that a
+ * subset of a larger problem's heads draws that problem's masks. */
 typedef struct {
     double p;
     uint64_t seed;
     uint32_t offset;
+    int64_t head0;
 } dropout_t;
 
-static const dropout_t no_dropout = {0.0, 0, 0};
+static const dropout_t no_dropout = {0.0, 0, 0, 0};
 
 /* Keep scale c * M_ij of element (i, j) of head bh (1 when p = 0). */
 static double keep_factor(const dropout_t *dr, int64_t bh, int i, int j)
 {
     if (dr->p == 0.0) return 1.0;
     const uint32_t t = drop_threshold(dr->p);
-    if (!keep_bit(dr->seed, dr->offset, bh, i, j, t)) return 0.0;
+    if (!keep_bit(dr->seed, dr->offset, dr->head0 + bh, i, j, t)) return 0.0;
     return 65536.0 / (65536.0 - (double)t);
 }
 
@@ -356,17 +359,17 @@ void oracle_attn_bwd_nc(const double *q, const double *k, const double *v, const
  * generator's seed and counter offset as in the header comment. */
 void oracle_attn_fwd_dropout(const double *q, const double *k, const double *v, double *o,
                              double *lse, int B, int H, int T, int D, double scale, int causal,
-                             double p, uint64_t seed, uint32_t offset)
+                             double p, uint64_t seed, uint32_t offset, int64_t head0)
 {
-    const dropout_t dr = {p, seed, offset};
+    const dropout_t dr = {p, seed, offset, head0};
     attn_fwd(q, k, v, o, lse, B, H, T, D, scale, causal, &dr);
 }
 
 void oracle_attn_bwd_dropout(const double *q, const double *k, const double *v,
                              const double *dO, double *dq, double *dk, double *dv, int B, int H,
                              int T, int D, double scale, int causal, double p, uint64_t seed,
-                             uint32_t offset)
+                             uint32_t offset, int64_t head0)
 {
-    const dropout_t dr = {p, seed, offset};
+    const dropout_t dr = {p, seed, offset, head0};
     attn_bwd(q, k, v, dO, dq, dk, dv, B, H, T, D, scale, causal, &dr);
 }

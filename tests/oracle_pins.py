@@ -559,8 +559,27 @@ def check_dropout_torch_witness(impl, seed=25):
             np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-12)
 
 
+def check_dropout_head_subset(impl, seed=26):
+    """A single head computed alone with head0 = its flat index matches that
+    head of the full call (so sampled heads can be checked one by one)."""
+    r = _rng(seed)
+    B, H, T, D = 2, 3, 21, 4
+    q, k, v, do = (r.standard_normal((B, H, T, D)) for _ in range(4))
+    kw = dict(dropout_p=0.3, seed=5, offset=9)
+    o, lse = impl.attn_fwd(q, k, v, **kw)
+    g = impl.attn_bwd(q, k, v, do, **kw)
+    for h in (0, 4, 5):
+        b, hh = divmod(h, H)
+        sl = lambda a: a[b:b + 1, hh:hh + 1]
+        o1, lse1 = impl.attn_fwd(sl(q), sl(k), sl(v), head0=h, **kw)
+        assert np.array_equal(o1, sl(o)) and np.array_equal(lse1, sl(lse))
+        for a, b1 in zip(g, impl.attn_bwd(sl(q), sl(k), sl(v), sl(do), head0=h, **kw)):
+            assert np.array_equal(b1, sl(a))
+
+
 DROPOUT_PINS = [check_philox_against_curand, check_dropout_mask_against_curand,
                 check_dropout_mask_statistics, check_dropout_zero_threshold_is_plain,
                 check_dropout_uniform_closed_form, check_dropout_unbiased,
-                check_dropout_finite_differences, check_dropout_torch_witness]
+                check_dropout_finite_differences, check_dropout_torch_witness,
+                check_dropout_head_subset]
 ALL_PINS = ALL_PINS + DROPOUT_PINS

@@ -180,3 +180,35 @@ def test_options_pass_to_the_ordinary_checks(causal):
         bad = _strides(8, t=3)
         assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.125, bad, o, None) == E_ALIGN
         assert lib.attn_bwd_ex(*([P] * 9), 1, 1, 8, 64, 0.125, bad, o, P, 1 << 30, None) == E_ALIGN
+
+
+@pytest.mark.parametrize("p", [-0.1, 1.0, 1.5, float("nan"), float("inf"), 0.999995])
+def test_options_reject_bad_dropout(p):
+    lib = lib_mod.lib()
+    E_OPTION = -10
+    o = ctypes.byref(lib_mod.attn_options(1, p, 7, 0, 0))
+    assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.125, None, o, None) == E_OPTION
+    assert lib.attn_bwd_ex(*([P] * 9), 1, 1, 8, 64, 0.125, None, o, P, 1 << 30, None) == E_OPTION
+    assert lib.attn_fwd_f32_ex(P, P, P, P, P, 1, 1, 8, 8, 0.35, o, None) == E_OPTION
+
+
+def test_options_reserved_must_be_zero():
+    lib = lib_mod.lib()
+    o = ctypes.byref(lib_mod.attn_options(1, 0.1, 7, 0, 1))
+    assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 64, 0.125, None, o, None) == -10
+
+
+def test_options_struct_layout():
+    """The ctypes mirror of attn_options matches the C layout: int32, float,
+    uint64 (8-aligned), uint32, uint32 = 24 bytes."""
+    assert ctypes.sizeof(lib_mod.attn_options) == 24
+    assert lib_mod.attn_options.dropout_seed.offset == 8
+    assert lib_mod.attn_options.dropout_offset.offset == 16
+
+
+@pytest.mark.parametrize("p", [0.0, 1e-6, 0.1, 0.99999])
+def test_valid_dropout_reaches_ordinary_checks(p):
+    lib = lib_mod.lib()
+    o = ctypes.byref(lib_mod.attn_options(0, p, 1 << 40, 3, 0))
+    assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 48, 0.125, None, o, None) == E_D
+    assert lib.attn_bwd_ex(*([P] * 9), 1, 1, 8, 64, 0.125, None, o, None, 0, None) == E_WS

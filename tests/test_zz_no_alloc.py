@@ -42,7 +42,7 @@ def test_noalloc_matches_attn_bwd_on_two_calls(case):
             assert np.all(np.isfinite(g))
             ma, rel = parity.errors(g, r)
             assert ma <= parity.BF16_TOL["max_abs"], f"call {call} {name}: max-abs {ma:.3e}"
-            assert rel <= parity.BF16_TOL["rel_l2"], f"call {call} {name}: rel-L2 {rel:.3e}"
+            assert rel is None or rel <= parity.BF16_TOL["rel_l2"], f"call {call} {name}: rel-L2 {rel}"
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
