@@ -69,6 +69,8 @@ class OracleLib:
                                                 ctypes.c_double, i, ctypes.c_double, u64, u32,
                                                 ctypes.c_int64]
         lib.oracle_attn_bwd_dropout.restype = None
+        lib.oracle_attn_decode.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, ctypes.c_double]
+        lib.oracle_attn_decode.restype = None
         lib.oracle_threads.argtypes = []
         lib.oracle_threads.restype = i
         self.lib = lib
@@ -118,6 +120,22 @@ class OracleLib:
         self._fn("oracle_attn_bwd", causal)(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq),
                                             _ptr(dk), _ptr(dv), B, H, T, D, scale)
         return dq, dk, dv
+
+    def attn_decode(self, q, k, v, scale=None):
+        """Decode: q [B,H,Tq,D] are the Tq newest tokens' queries, k, v
+        [B,H,Tk,D] all Tk tokens' keys and values.  Returns (O [B,H,Tq,D],
+        lse [B,H,Tq])."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, Tq, D = _shape(q)
+        Tk = k.shape[2]
+        if k.shape != (B, H, Tk, D) or v.shape != k.shape or not 1 <= Tq <= Tk:
+            raise ValueError("q [B,H,Tq,D], k and v [B,H,Tk,D] with 1 <= Tq <= Tk")
+        scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+        o = np.empty_like(q)
+        lse = np.empty((B, H, Tq), dtype=np.float64)
+        self.lib.oracle_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Tq, Tk, D,
+                                    scale)
+        return o, lse
 
     def philox4x32_10(self, ctr, key):
         """Philox4x32-10 of one 4-word counter under a 2-word key."""
@@ -177,6 +195,11 @@ def attn_probs(q, k, scale=None, causal=True):
 def attn_bwd(q, k, v, do, scale=None, causal=True, dropout_p=0.0, seed=0, offset=0, head0=0):
     """Returns (dQ, dK, dV) in float64 for the loss sum(O * dO)."""
     return _load().attn_bwd(q, k, v, do, scale, causal, dropout_p, seed, offset, head0)
+
+
+def attn_decode(q, k, v, scale=None):
+    """Decode attention of the Tq newest queries over Tk cached keys/values."""
+    return _load().attn_decode(q, k, v, scale)
 
 
 def philox4x32_10(ctr, key):

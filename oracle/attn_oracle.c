@@ -62,6 +62,14 @@
  * iff that value is >= t, t = floor(p * 65536 + 1/2) for the drop probability
  * p, and c = 65536 / (65536 - t), so E[c M] = 1 exactly.
  *
+ * Decode ("oracle_attn_decode"): generating text appends one token at a time
+ * and each new token's query attends to every earlier token and itself
+ * ("nanoGPT — 架构与原理", section 5 "边界与局限": generate recomputes the
+ * whole forward for every new token, with no KV cache).  With the keys
+ * and values of all Tk tokens kept, the Tq newest queries (positions
+ * Tk - Tq .. Tk - 1) need only their own rows of the causal attention: query
+ * r sees keys 0 .. Tk - Tq + r.
+ *
  * Layout: every tensor is [B, H, T, D] contiguous float64; lse is [B, H, T].
  * No blocking, no fusion, no reordering beyond the definition.  The softmax
  * subtracts the row maximum before exponentiating, which changes nothing in
@@ -372,4 +380,32 @@ void oracle_attn_bwd_dropout(const double *q, const double *k, const double *v,
 {
     const dropout_t dr = {p, seed, offset, head0};
     attn_bwd(q, k, v, dO, dq, dk, dv, B, H, T, D, scale, causal, &dr);
+}
+
+/* Decode: q, o [B,H,Tq,D], k, v [B,H,Tk,D], lse [B,H,Tq] (may be NULL);
+ * query r is the token at position Tk - Tq + r and sees keys 0 .. Tk - Tq + r. */
+void oracle_attn_decode(const double *q, const double *k, const double *v, double *o,
+                        double *lse, int B, int H, int Tq, int Tk, int D, double scale)
+{
+    const int64_t heads = (int64_t)B * H;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)(Tk > 0 ? Tk : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < heads; ++bh) {
+            const double *kh = k + bh * (int64_t)Tk * D, *vh = v + bh * (int64_t)Tk * D;
+            for (int r = 0; r < Tq; ++r) {
+                const int last = Tk - Tq + r;
+                const double *qr = q + (bh * Tq + r) * (int64_t)D;
+                double li = softmax_row(qr, kh, last, D, scale, p);
+                if (lse) lse[bh * Tq + r] = li;
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int j = 0; j <= last; ++j) acc += p[j] * vh[(int64_t)j * D + d];
+                    o[(bh * Tq + r) * (int64_t)D + d] = acc;
+                }
+            }
+        }
+        free(p);
+    }
 }

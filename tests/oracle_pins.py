@@ -583,3 +583,49 @@ DROPOUT_PINS = [check_philox_against_curand, check_dropout_mask_against_curand,
                 check_dropout_finite_differences, check_dropout_torch_witness,
                 check_dropout_head_subset]
 ALL_PINS = ALL_PINS + DROPOUT_PINS
+
+
+# ---------------------------------------------------------------- decode
+
+def check_decode_rows_of_causal(impl, seed=31):
+    """The Tq newest queries over Tk cached keys are exactly the last Tq rows
+    of the causal attention over all Tk tokens (bit for bit: the same row
+    computation), for every Tq from 1 to Tk."""
+    r = _rng(seed)
+    B, H, Tk, D = 2, 3, 13, 5
+    q, k, v = (r.standard_normal((B, H, Tk, D)) for _ in range(3))
+    o, lse = impl.attn_fwd(q, k, v)
+    for tq in (1, 2, 5, Tk):
+        od, lsed = impl.attn_decode(q[:, :, Tk - tq:], k, v)
+        assert np.array_equal(od, o[:, :, Tk - tq:]), f"decode Tq={tq} differs from causal rows"
+        assert np.array_equal(lsed, lse[:, :, Tk - tq:])
+
+
+def check_decode_uniform_closed_form(impl, seed=32):
+    """Q = 0: query r averages the values of keys 0 .. Tk - Tq + r."""
+    r = _rng(seed)
+    B, H, Tk, D, tq = 2, 2, 17, 4, 3
+    k, v = r.standard_normal((B, H, Tk, D)), r.standard_normal((B, H, Tk, D))
+    o, lse = impl.attn_decode(np.zeros((B, H, tq, D)), k, v)
+    for rr in range(tq):
+        n = Tk - tq + rr + 1
+        np.testing.assert_allclose(o[:, :, rr], v[:, :, :n].mean(axis=2), rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, rr], math.log(n), rtol=0, atol=1e-14)
+
+
+def check_decode_torch_witness(impl, seed=33):
+    import torch
+    r = _rng(seed)
+    B, H, Tk, D, tq = 2, 2, 40, 8, 4
+    q = r.standard_normal((B, H, tq, D))
+    k, v = r.standard_normal((B, H, Tk, D)), r.standard_normal((B, H, Tk, D))
+    allowed = torch.arange(Tk)[None, :] <= (Tk - tq + torch.arange(tq))[:, None]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q), torch.tensor(k), torch.tensor(v), attn_mask=allowed)
+    o, _ = impl.attn_decode(q, k, v)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+
+
+DECODE_PINS = [check_decode_rows_of_causal, check_decode_uniform_closed_form,
+               check_decode_torch_witness]
+ALL_PINS = ALL_PINS + DECODE_PINS

@@ -12,7 +12,10 @@ MUTATIONS = {
     "scale_dropped": ("s *= scale;", "s *= 1.0;"),
     "lse_log2": ("return m + log(l);", "return m + log2(l);"),
     "softmax_not_normalised": ("for (int j = 0; j <= i; ++j) p[j] /= l;", ""),
-    "pv_wrong_value_row": ("acc += p[j] * vh[(int64_t)j * D + d];", "acc += p[j] * vh[(int64_t)i * D + d];"),
+    "pv_wrong_value_row": ("acc += p[j] * vh[(int64_t)j * D + d];\n                    oh[",
+                           "acc += p[j] * vh[(int64_t)i * D + d];\n                    oh["),
+    "decode_pv_wrong_value_row": ("acc += p[j] * vh[(int64_t)j * D + d];\n                    o[(bh",
+                                  "acc += p[j] * vh[(int64_t)r * D + d];\n                    o[(bh"),
     "dv_transposed_p": ("acc += Z[(int64_t)i * T + j] * gh[(int64_t)i * D + d];",
                         "acc += Z[(int64_t)j * T + i] * gh[(int64_t)i * D + d];"),
     "ds_sign_flipped": ("keep_factor(dr, bh, i, j) * dp - delta)", "delta - keep_factor(dr, bh, i, j) * dp)"),
@@ -37,6 +40,9 @@ MUTATIONS = {
     "dropout_dv_uses_p": ("acc += Z[(int64_t)i * T + j] * gh[(int64_t)i * D + d];",
                           "acc += P[(int64_t)i * T + j] * gh[(int64_t)i * D + d];"),
     "dropout_ds_ignores_mask": ("(keep_factor(dr, bh, i, j) * dp - delta)", "(dp - delta)"),
+    "decode_sees_one_key_too_few": ("const int last = Tk - Tq + r;", "const int last = Tk - Tq + r - 1;"),
+    "decode_wrong_query_row": ("const double *qr = q + (bh * Tq + r) * (int64_t)D;",
+                               "const double *qr = q + (bh * Tq) * (int64_t)D;"),
 }
 
 
