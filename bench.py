@@ -55,6 +55,8 @@ def parse_args():
                    help="skip the secondary measurement of the non-causal variant")
     p.add_argument("--no-dropout", action="store_true",
                    help="skip the secondary measurement with attention dropout 0.1")
+    p.add_argument("--no-decode", action="store_true",
+                   help="skip the secondary measurement of decode attention")
     p.add_argument("--layers", type=int, default=None,
                    help="layer instances per step (default: the workload's 12); fewer only for profiling")
     return p.parse_args()
@@ -499,6 +501,81 @@ def run_ours(args, w):
     noncausal = None if args.no_noncausal else variant_leg(False, 0.0)
     dropout = None if args.no_dropout else variant_leg(True, 0.1)
 
+    # ---- secondary: decode, one new token per sequence against the kept keys
+    # and values of all T = 1024 tokens, every layer of the step (the caches
+    # of 12 layers, 453 MB, exceed L2).  HBM bytes per launch: K and V read,
+    # q read, O written, lse written.
+    decode = None
+    if not args.no_decode:
+        from workloads import make_decode_inputs
+        tq = 1
+        dl = []
+        for l in range(L):
+            di = make_decode_inputs(w, tq, seed=args.seed + 7919 * rank, layer=l)
+            dl.append({n: t.to(dev) for n, t in di.items()})
+            dl[-1]["o"] = torch.empty_like(dl[-1]["q"])
+            dl[-1]["lse"] = torch.empty((w.B, w.H, tq), dtype=torch.float32, device=dev)
+        n_d = max(10, min(args.steps, 100))
+        evd = [[(mk(), mk()) for _ in range(L)] for _ in range(n_d)]
+        for e in evd:
+            for pair in e:
+                for x in pair:
+                    x.record(stream)
+
+        def d_step(evs=None):
+            for l, b in enumerate(dl):
+                if evs is not None:
+                    A.attn_profile_next_call(*evs[l])
+                A.attn_decode(b["q"], b["k"], b["v"], b["o"], b["lse"])
+        for _ in range(3):
+            d_step()
+        barrier()
+        s0, s1 = mk(), mk()
+        s0.record(stream)
+        for i in range(n_d):
+            d_step(evd[i])
+        s1.record(stream)
+        barrier()
+        d_ms = reduce_max(s0.elapsed_time(s1), world, dev) / n_d
+        k_ms = statistics.mean(a.elapsed_time(b) for e in evd for a, b in e)
+        bytes_launch = w.B * w.H * (2 * w.T * w.D * 2 + 2 * tq * w.D * 2 + tq * 4)
+        hbm_peak = float(peaks.get("hbm_gbs"))
+        # the same step replayed from a CUDA graph (no per-launch host cost)
+        graph = None
+        try:
+            gs = torch.cuda.Stream(dev)
+            gs.wait_stream(stream)
+            with torch.cuda.stream(gs):
+                d_step()
+            stream.wait_stream(gs)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                d_step()
+            g.replay()
+            barrier()
+            s0.record(stream)
+            for _ in range(n_d):
+                g.replay()
+            s1.record(stream)
+            barrier()
+            g_ms = reduce_max(s0.elapsed_time(s1), world, dev) / n_d
+            graph = {"ms_per_step": g_ms, "gbs": bytes_launch * L / (g_ms * 1e-3) / 1e9,
+                     "tokens_per_s": world * w.B / (g_ms * 1e-3)}
+            del g
+        except RuntimeError as exc:  # capture unsupported here: report, do not fail the bench
+            graph = {"unavailable": str(exc).splitlines()[0][:200]}
+        if A.attn_device_error() != 0:
+            raise RuntimeError("a bounded in-kernel wait timed out in the decode leg")
+        decode = {"workload": f"{w.name} decode: B={w.B} H={w.H} D={w.D}, {tq} new token over "
+                              f"{w.T} kept keys/values, {L} layers per step",
+                  "ms_per_step": d_ms, "tokens_per_s": world * w.B / (d_ms * 1e-3),
+                  "steps": n_d, "bytes_per_launch": bytes_launch,
+                  "kernel": {"avg_launch_ms": k_ms, "gbs": bytes_launch / (k_ms * 1e-3) / 1e9,
+                             "peak_gbs": hbm_peak,
+                             "frac": bytes_launch / (k_ms * 1e-3) / 1e9 / hbm_peak},
+                  "graph": graph}
+        del dl
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.seed)
@@ -514,7 +591,7 @@ def run_ours(args, w):
                             "measured_sustained": value / world / float(peaks.get("bf16_tflops_sustained", peak)),
                             "datasheet_2250": value / world / 2250.0},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "strided_io": strided,
-            "noncausal": noncausal, "dropout": dropout,
+            "noncausal": noncausal, "dropout": dropout, "decode": decode,
             "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -69,6 +69,9 @@ _lib.attn_fwd_f32_ex.restype = _i
 _lib.attn_bwd_f32_ex.argtypes = [_fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _op,
                                  _vp, _sz, _vp]
 _lib.attn_bwd_f32_ex.restype = _i
+_lib.attn_decode.argtypes = [_vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _i, _f, _sp, _vp]
+_lib.attn_decode.restype = _i
+DECODE_MAX_QUERIES = 16
 _lib.attn_fwd_f32.argtypes = [_fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _vp]
 _lib.attn_fwd_f32.restype = _i
 _lib.attn_bwd_f32_workspace_bytes.argtypes = [_i, _i, _i, _i]
@@ -86,7 +89,8 @@ EXPORTED = ("attn_status_string", "attn_version", "attn_last_launch_count", "att
             "attn_bwd_workspace_bytes", "attn_bwd", "attn_fwd_f32", "attn_bwd_f32_workspace_bytes",
             "attn_bwd_f32", "attn_device_error", "attn_profile_next_call",
             "attn_selftest_wait_timeout", "attn_bwd_noalloc", "attn_fwd_strided",
-            "attn_bwd_strided", "attn_fwd_ex", "attn_bwd_ex", "attn_fwd_f32_ex", "attn_bwd_f32_ex")
+            "attn_bwd_strided", "attn_fwd_ex", "attn_bwd_ex", "attn_fwd_f32_ex", "attn_bwd_f32_ex",
+            "attn_decode")
 
 
 class AttnError(RuntimeError):
@@ -424,3 +428,25 @@ def attn_bwd_f32_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optio
     fn.__name__ = "attn_bwd_f32_ex"
     return _bwd(fn, _lib.attn_bwd_f32_workspace_bytes, _torch().float32, q, k, v, o, lse, dO, dq,
                 dk, dv, scale, workspace, stream)
+
+
+def attn_decode(q, k, v, o=None, lse=None, scale: Optional[float] = None, stream=None):
+    """Decode attention: q [B, H, Tq, D] holds the Tq newest tokens' queries
+    (Tq <= 16), k and v [B, H, Tk, D] the kept keys and values of all Tk
+    tokens (views into a larger cache are fine: only the D stride must be 1).
+    Query r is the token at position Tk - Tq + r.  Returns (O [B, H, Tq, D],
+    lse [B, H, Tq])."""
+    torch = _torch()
+    B, H, Tq, D = _shape4(q)
+    Tk = int(k.shape[2])
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    o = torch.empty_like(q, memory_format=torch.contiguous_format) if o is None else o
+    lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device) if lse is None else lse
+    ptrs = [_check_view(q, "q", (B, H, Tq, D)), _check_view(k, "k", (B, H, Tk, D)),
+            _check_view(v, "v", (B, H, Tk, D)), _check_view(o, "o", (B, H, Tq, D)),
+            _check(lse, "lse", torch.float32, (B, H, Tq))]
+    st = None if _all_contiguous(q, k, v, o) else _strides_of(q, k, v, o)
+    with torch.cuda.device(q.device):
+        _raise(_lib.attn_decode(*ptrs, B, H, Tq, Tk, D, scale, st, _stream_handle(stream)),
+               "attn_decode")
+    return o, lse

@@ -277,6 +277,37 @@ ATTN_API int attn_fwd_strided(const void *q, const void *k, const void *v, void 
     return attn_fwd_ex(q, k, v, o, lse, B, H, T, D, scale, strides, nullptr, stream);
 }
 
+ATTN_API int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                         int H, int Tq, int Tk, int D, float scale, const attn_strides *strides,
+                         cudaStream_t stream) {
+    LaunchInfo li = take_launch_info();
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    int st = check_shape(B, H, Tk, D, 64);
+    if (st != ATTN_OK) return st;
+    if (Tq < 1 || Tq > ATTN_DECODE_MAX_QUERIES || Tq > Tk) return ATTN_ERR_SHAPE;
+    if (!bf16_d_supported(D)) return ATTN_ERR_UNSUPPORTED_D;
+    if ((st = check_scale(scale)) != ATTN_OK) return st;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return ATTN_ERR_ALIGN;
+    FwdStrides str;
+    if (strides) {
+        for (int i = 0; i < 4; ++i)
+            if (!strides_ok(strides[i])) return ATTN_ERR_ALIGN;
+        str = FwdStrides{to_tstrides(strides[0]), to_tstrides(strides[1]), to_tstrides(strides[2]),
+                         to_tstrides(strides[3])};
+    } else {
+        const TStrides kv = contiguous_strides(Shape{B, H, Tk, D, scale});
+        const TStrides qo = contiguous_strides(Shape{B, H, Tq, D, scale});
+        str = FwdStrides{qo, kv, kv, qo};
+    }
+    int *err = nullptr;
+    if ((st = device_setup(&err)) != ATTN_OK) return st;
+    cudaError_t e = sm100_decode(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                                 static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), lse,
+                                 DecodeShape{B, H, Tq, Tk, D, scale}, str, err, stream, li);
+    return finish(e, li);
+}
+
 // Workspace of the bf16 backward: dQ float32 accumulator, padded lse, Delta.
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
     if (check_shape(B, H, T, D, 64) != ATTN_OK || !bf16_d_supported(D)) return 0;

@@ -64,6 +64,17 @@ inline cudaError_t mark_main_end(const LaunchInfo &li, cudaStream_t st) {
     return li.main_end ? cudaEventRecord(li.main_end, st) : cudaSuccess;
 }
 
+// ---- decode: the Tq newest queries against the keys/values of Tk tokens
+constexpr int kMaxDecodeQueries = 16;
+struct DecodeShape {
+    int B, H, Tq, Tk, D;
+    float scale;
+};
+// bf16, D in {32, 64}; strides of q, k, v, o (k, v over Tk tokens; q, o over Tq).
+cudaError_t sm100_decode(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                         __nv_bfloat16 *o, float *lse, const DecodeShape &s, const FwdStrides &str,
+                         int *err, cudaStream_t st, LaunchInfo &li);
+
 // ---- SIMT kernels (float32 math on CUDA cores), element type float or bf16
 template <typename T>
 cudaError_t simt_fwd(const T *q, const T *k, const T *v, T *o, float *lse, Shape s,

@@ -207,6 +207,31 @@ int attn_bwd_ex(const void *q, const void *k, const void *v, const void *o,
                 const attn_options *opts, void *workspace, size_t workspace_bytes,
                 cudaStream_t stream);
 
+/* ---------------- decode: new tokens against kept keys and values ------- */
+
+/* Text generation appends one token at a time and each new token attends to
+ * every earlier token and to itself ("nanoGPT — 架构与原理", section 5
+ * "边界与局限": nanoGPT's generate has no KV cache and recomputes the whole
+ * forward per token).  With the keys and values of all Tk tokens kept, the
+ * Tq newest tokens need only their rows of the causal attention:
+ *
+ *   query r (0 <= r < Tq) is the token at position Tk - Tq + r and attends to
+ *   keys 0 .. Tk - Tq + r;  o_r = softmax(scale q_r K^T) V over those keys,
+ *   lse_r = ln sum_j exp(scale q_r . k_j) over the same keys.
+ *
+ * q: bf16 [B, H, Tq, D]; k, v: bf16 [B, H, Tk, D] (the kept keys/values, e.g.
+ * the first Tk rows of a cache of larger capacity); o: bf16 [B, H, Tq, D];
+ * lse: float32 [B, H, Tq] contiguous.  1 <= Tq <= ATTN_DECODE_MAX_QUERIES and
+ * Tq <= Tk (else ATTN_ERR_SHAPE); D 32 or 64.  strides: NULL for contiguous
+ * tensors (a cache of capacity Tmax is {H*Tmax*D, Tmax*D, D}), else
+ * strides[0..3] for q, k, v, o under the rules of attn_fwd_strided.  Forward
+ * only (generation does not differentiate), no dropout, one kernel launch, no
+ * workspace.  Other rules as attn_fwd. */
+#define ATTN_DECODE_MAX_QUERIES 16
+int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int H, int Tq, int Tk, int D, float scale, const attn_strides *strides,
+                cudaStream_t stream);
+
 /* ---------------- float32 path: CUDA cores, IEEE expf -------------------- */
 
 /* Forward in float32 (all tensors float32).  1 <= D <= 128. */

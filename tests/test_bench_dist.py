@@ -29,7 +29,10 @@ def _rank_main(rank, world, port, out_dir):
 
 
 def test_max_over_ranks_and_whole_job_value(tmp_path):
-    port = 29500 + (os.getpid() % 2000)
+    import socket
+    with socket.socket() as sock:  # a port that is free right now
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
     mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True,
                        start_method="spawn")
     res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(2)]

@@ -212,3 +212,21 @@ def test_valid_dropout_reaches_ordinary_checks(p):
     o = ctypes.byref(lib_mod.attn_options(0, p, 1 << 40, 3, 0))
     assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 8, 48, 0.125, None, o, None) == E_D
     assert lib.attn_bwd_ex(*([P] * 9), 1, 1, 8, 64, 0.125, None, o, None, 0, None) == E_WS
+
+
+@pytest.mark.parametrize("B,H,Tq,Tk,D,expect", [
+    (1, 1, 0, 8, 64, E_SHAPE), (1, 1, 17, 64, 64, E_SHAPE), (1, 1, 9, 8, 64, E_SHAPE),
+    (0, 1, 1, 8, 64, E_SHAPE), (1, 1, 1, 0, 64, E_SHAPE), (1, 1, 1, 8, 48, E_D),
+    (1, 1, 1, 8, 128, E_D)])
+def test_decode_argument_errors(B, H, Tq, Tk, D, expect):
+    lib = lib_mod.lib()
+    assert lib.attn_decode(P, P, P, P, P, B, H, Tq, Tk, D, 0.125, None, None) == expect
+
+
+def test_decode_pointer_and_stride_errors():
+    lib = lib_mod.lib()
+    assert lib.attn_decode(None, P, P, P, P, 1, 1, 1, 8, 64, 0.125, None, None) == E_NULL
+    assert lib.attn_decode(P + 2, P, P, P, P, 1, 1, 1, 8, 64, 0.125, None, None) == E_ALIGN
+    assert lib.attn_decode(P, P, P, P, P, 1, 1, 1, 8, 64, -1.0, None, None) == E_SCALE
+    bad = _strides(4, t=12)
+    assert lib.attn_decode(P, P, P, P, P, 1, 1, 1, 8, 64, 0.125, bad, None) == E_ALIGN

@@ -31,6 +31,9 @@ Input recipe (no dataset or trained weight is used anywhere):
 * Everything is drawn in float32 from ``torch.Generator`` seeded with
   ``seed + 1000 * workload_index + layer`` and then rounded to the workload's
   dtype (bf16 or kept float32).
+* Decode (``make_decode_inputs``): the same Q, K, V of a workload; the Tq
+  newest tokens' queries are Q's last Tq rows, and K and V of all T tokens
+  are the kept keys and values (T plays Tk).
 """
 from __future__ import annotations
 
@@ -164,3 +167,10 @@ def random_qkv(seed: int, B: int, H: int, T: int, D: int, dtype=torch.float32,
     for name, s in (("q", std), ("k", std), ("v", std), ("do", do_std)):
         out[name] = (torch.randn(B, H, T, D, generator=g, dtype=torch.float32) * s).to(dtype).contiguous()
     return out
+
+
+def make_decode_inputs(w: Workload, tq: int, seed: int = 0, layer: int = 0) -> Dict[str, torch.Tensor]:
+    """Decode inputs from the workload's Q, K, V: "q" [B, H, tq, D] = the last
+    tq rows of Q (the newest tokens), "k", "v" [B, H, T, D] all T tokens."""
+    inp = make_inputs(w, seed=seed, layer=layer)
+    return {"q": inp["q"][:, :, w.T - tq:].contiguous(), "k": inp["k"], "v": inp["v"]}
