@@ -82,7 +82,7 @@ def test_f32_odd_shapes_dropout(B, H, T, D):
 
 
 def test_bf16_char_gpt_dropout_all_heads():
-    """The character-level GPT shape at the Shakespeare config's rate 0.2."""
+    """The character-level GPT shape, all heads, at a second rate (0.2)."""
     inp = make_inputs(WORKLOADS["char_gpt"], seed=3)
     kw = dict(dropout_p=0.2, seed=1234, offset=5)
     got = parity.run_gpu(inp, **kw)
