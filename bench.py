@@ -156,13 +156,20 @@ def gpu_uuid(torch, dev):
         return str(dev)
 
 
-def kernel_source_hash():
+# The sources each timed kernel is built from (its own file plus the shared headers).
+KERNEL_SOURCES = {
+    "attn_fwd": ["attn_fwd_sm100.cu", "sm100.cuh", "internal.h", "philox.cuh"],
+    "attn_bwd": ["attn_bwd_sm100.cu", "sm100.cuh", "internal.h", "philox.cuh"],
+    "attn_decode": ["attn_decode_sm100.cu", "sm100.cuh", "internal.h", "philox.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "decoder_only_transformer_sdpa_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -175,7 +182,7 @@ def measured_traffic(kernel: str):
     with open(path) as f:
         d = json.load(f)
     ent = d.get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("bytes_per_launch")
 
@@ -572,7 +579,8 @@ def run_ours(args, w):
                   "steps": n_d, "bytes_per_launch": bytes_launch,
                   "kernel": {"avg_launch_ms": k_ms, "gbs": bytes_launch / (k_ms * 1e-3) / 1e9,
                              "peak_gbs": hbm_peak,
-                             "frac": bytes_launch / (k_ms * 1e-3) / 1e9 / hbm_peak},
+                             "frac": bytes_launch / (k_ms * 1e-3) / 1e9 / hbm_peak,
+                             "traffic": measured_traffic("attn_decode")},
                   "graph": graph}
         del dl
 
