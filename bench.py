@@ -57,6 +57,8 @@ def parse_args():
                    help="skip the secondary measurement with attention dropout 0.1")
     p.add_argument("--no-decode", action="store_true",
                    help="skip the secondary measurement of decode attention")
+    p.add_argument("--no-d128", action="store_true",
+                   help="skip the secondary measurement at head_dim 128")
     p.add_argument("--layers", type=int, default=None,
                    help="layer instances per step (default: the workload's 12); fewer only for profiling")
     return p.parse_args()
@@ -584,6 +586,65 @@ def run_ours(args, w):
                   "graph": graph}
         del dl
 
+    # ---- secondary: head_dim 128 -- the same n_embd (768) as 6 heads of 128
+    # at the GPT-2 batch and context, 12 layer instances, causal
+    d128 = None
+    if not args.no_d128:
+        from workloads import random_qkv
+        H2, D2 = 6, 128
+        wl = []
+        for l in range(L):
+            ri = random_qkv(args.seed + 50000 + 7919 * rank + l, w.B, H2, w.T, D2,
+                            dtype=torch.bfloat16, std=0.55, do_std=1e-2)
+            b = {n: t.to(dev) for n, t in ri.items()}
+            b["o"] = torch.empty_like(b["q"])
+            b["lse"] = torch.empty((w.B, H2, w.T), dtype=torch.float32, device=dev)
+            b["dq"], b["dk"], b["dv"] = (torch.empty_like(b["q"]) for _ in range(3))
+            b["ws"] = torch.empty(A.attn_bwd_workspace_bytes(w.B, H2, w.T, D2), dtype=torch.uint8,
+                                  device=dev)
+            wl.append(b)
+        n_w = max(3, min(args.steps, 30))
+        evw = [([(mk(), mk()) for _ in range(L)], [(mk(), mk()) for _ in range(L)]) for _ in range(n_w)]
+        for e in evw:
+            for pair in e[0] + e[1]:
+                for x in pair:
+                    x.record(stream)
+
+        def w_step(ev_fwd=None, ev_bwd=None):
+            for l, b in enumerate(wl):
+                if ev_fwd is not None:
+                    A.attn_profile_next_call(*ev_fwd[l])
+                A.attn_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"])
+            for l in range(L - 1, -1, -1):
+                b = wl[l]
+                if ev_bwd is not None:
+                    A.attn_profile_next_call(*ev_bwd[l])
+                A.attn_bwd(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"],
+                           b["dv"], workspace=b["ws"])
+        w_step()
+        barrier()
+        s0, s1 = mk(), mk()
+        s0.record(stream)
+        for i in range(n_w):
+            w_step(*evw[i])
+        s1.record(stream)
+        barrier()
+        if A.attn_device_error() != 0:
+            raise RuntimeError("a bounded in-kernel wait timed out in the head_dim 128 leg")
+        w_ms = reduce_max(s0.elapsed_time(s1), world, dev)
+        pairs_w = w.B * H2 * w.T * (w.T + 1) // 2
+        nf = statistics.mean(a.elapsed_time(b) for e in evw for a, b in e[0])
+        nb = statistics.mean(a.elapsed_time(b) for e in evw for a, b in e[1])
+        tf = lambda fl, ms_: fl / (ms_ * 1e-3) / 1e12
+        d128 = {"workload": f"B={w.B} H={H2} T={w.T} D={D2} (n_embd {H2 * D2}), {L} layers, causal",
+                "value": whole_job_tflops(12 * D2 * pairs_w * L, world, n_w, w_ms), "unit": "TFLOP/s",
+                "ms_per_step": w_ms / n_w, "steps": n_w,
+                "fwd_main": {"avg_launch_ms": nf, "tflops": tf(4 * D2 * pairs_w, nf),
+                             "frac": tf(4 * D2 * pairs_w, nf) / peak},
+                "bwd_main": {"avg_launch_ms": nb, "tflops": tf(8 * D2 * pairs_w, nb),
+                             "frac": tf(8 * D2 * pairs_w, nb) / peak}}
+        del wl
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.seed)
@@ -599,7 +660,7 @@ def run_ours(args, w):
                             "measured_sustained": value / world / float(peaks.get("bf16_tflops_sustained", peak)),
                             "datasheet_2250": value / world / 2250.0},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "strided_io": strided,
-            "noncausal": noncausal, "dropout": dropout, "decode": decode,
+            "noncausal": noncausal, "dropout": dropout, "decode": decode, "d128": d128,
             "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

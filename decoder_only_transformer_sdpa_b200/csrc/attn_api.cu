@@ -90,7 +90,8 @@ int finish(cudaError_t e, const LaunchInfo &li) {
     return ATTN_OK;
 }
 
-bool bf16_d_supported(int D) { return D == 32 || D == 64; }
+bool bf16_d_supported(int D) { return D == 32 || D == 64 || D == 128; }
+bool decode_d_supported(int D) { return D == 32 || D == 64; }
 
 }  // namespace
 }  // namespace attn
@@ -203,7 +204,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
              int D, float scale, const Opts &op, const FwdStrides &str, cudaStream_t stream,
              LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
-    int st = check_shape(B, H, T, D, 64);
+    int st = check_shape(B, H, T, D, 128);
     if (st != ATTN_OK) return st;
     if (!bf16_d_supported(D)) return ATTN_ERR_UNSUPPORTED_D;
     if ((st = check_scale(scale)) != ATTN_OK) return st;
@@ -222,7 +223,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
              const Opts &op, const BwdStrides &str, void *workspace, size_t workspace_bytes,
              cudaStream_t stream, LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
-    int st = check_shape(B, H, T, D, 64);
+    int st = check_shape(B, H, T, D, 128);
     if (st != ATTN_OK) return st;
     if (!bf16_d_supported(D)) return ATTN_ERR_UNSUPPORTED_D;
     if ((st = check_scale(scale)) != ATTN_OK) return st;
@@ -282,10 +283,10 @@ ATTN_API int attn_decode(const void *q, const void *k, const void *v, void *o, f
                          cudaStream_t stream) {
     LaunchInfo li = take_launch_info();
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
-    int st = check_shape(B, H, Tk, D, 64);
+    int st = check_shape(B, H, Tk, D, 128);
     if (st != ATTN_OK) return st;
     if (Tq < 1 || Tq > ATTN_DECODE_MAX_QUERIES || Tq > Tk) return ATTN_ERR_SHAPE;
-    if (!bf16_d_supported(D)) return ATTN_ERR_UNSUPPORTED_D;
+    if (!decode_d_supported(D)) return ATTN_ERR_UNSUPPORTED_D;
     if ((st = check_scale(scale)) != ATTN_OK) return st;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
         return ATTN_ERR_ALIGN;
@@ -310,7 +311,7 @@ ATTN_API int attn_decode(const void *q, const void *k, const void *v, void *o, f
 
 // Workspace of the bf16 backward: dQ float32 accumulator, padded lse, Delta.
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
-    if (check_shape(B, H, T, D, 64) != ATTN_OK || !bf16_d_supported(D)) return 0;
+    if (check_shape(B, H, T, D, 128) != ATTN_OK || !bf16_d_supported(D)) return 0;
     return bwd_workspace_layout(B, H, T, D).total;
 }
 

@@ -552,6 +552,36 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     return cudaSuccess;
 }
 
+// head_dim 128: the same prep and post kernels around the D = 128 main kernel
+// (attn_bwd128_sm100.cu).
+cudaError_t launch_bwd128(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                          const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
+                          __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
+                          float *lse2, float *delta, Shape s, const BwdStrides &str, int *err,
+                          cudaStream_t st, LaunchInfo &li) {
+    constexpr int D = 128;
+    const int BH = s.B * s.H;
+    const int Tpad = (s.T + kBT - 1) / kBT * kBT;
+    const long long prows = (long long)BH * Tpad;
+    const long long prep_threads = prows * (D / 8);
+    bwd_prep_kernel<D><<<(unsigned)((prep_threads + 255) / 256), 256, 0, st>>>(
+        o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows, s.H, str.o, str.dO);
+    cudaError_t e;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    li.kernels += 1;
+    if ((e = sm100_bwd128_main(q, k, v, dO, dk, dv, dq_acc, lse2, delta, s, str, err, st, li)) !=
+        cudaSuccess)
+        return e;
+    const long long n8 = (long long)BH * s.T * D / 8;
+    const long long want = (n8 + 255) / 256;
+    const int post_blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+    bwd_post_kernel<<<post_blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc), dq, n8,
+                                                  s.scale, s.T, s.H, D, str.dq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    li.kernels += 1;
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
@@ -572,6 +602,8 @@ cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     ATTN_BWD_CASE(32, true, true)
     ATTN_BWD_CASE(32, false, true)
 #undef ATTN_BWD_CASE
+    if (s.D == 128)
+        return launch_bwd128(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, str, err, st, li);
     return cudaErrorInvalidValue;
 }
 

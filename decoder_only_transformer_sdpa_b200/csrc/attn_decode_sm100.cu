@@ -65,7 +65,10 @@ struct DecSmem {
     // O, [warp][NQ][D] floats)
     alignas(1024) __nv_bfloat16 k[kStages][kTile * D];
     alignas(1024) __nv_bfloat16 v[kStages][kTile * D];
-    float q[NQ][D];                 // queries times scale * log2(e); zero rows past Tq
+    // queries times scale * log2(e), zero rows past Tq, as two half rows; the
+    // pad puts the halves on different banks (the two lanes of a key read one
+    // half each with the same instruction)
+    float q[NQ][2][D / 2 + 4];
     float mw[kWarps][NQ], lw[kWarps][NQ];  // per warp: running max (log2 units), sum
     float o[NQ][D];                 // this CTA's unnormalised partial O
     float mc[NQ], lc[NQ];           // this CTA's max and sum (read by CTA 0 of the cluster)
@@ -127,11 +130,12 @@ __global__ void __launch_bounds__(kThreads)
             w = *reinterpret_cast<const uint4 *>(q + (long long)bb * sq.b + (long long)hh * sq.h +
                                                  (long long)r * sq.t + 8 * c);
         const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
+        float *dst = &sm.q[r][(8 * c) / (D / 2)][(8 * c) % (D / 2)];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
             const float2 f = __bfloat1622float2(w2[x]);
-            sm.q[r][8 * c + 2 * x] = f.x * qscale;
-            sm.q[r][8 * c + 2 * x + 1] = f.y * qscale;
+            dst[2 * x] = f.x * qscale;
+            dst[2 * x + 1] = f.y * qscale;
         }
     }
     __syncthreads();
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(kThreads)
             float pw[NQ];
 #pragma unroll
             for (int r = 0; r < NQ; ++r) {
-                const float *qr = &sm.q[r][hf * kHalfChunks * 8];
+                const float *qr = &sm.q[r][hf][0];
                 float d0 = 0.f, d1 = 0.f;
 #pragma unroll
                 for (int x = 0; x < kHalfChunks * 8; x += 2) {

@@ -8,9 +8,12 @@
 // the value aggregation; section "Self-Attention: the mathematical trick"
 // [55:20] for the -inf upper triangle and the softmax).
 //
-// Persistent kernel: two CTAs per SM (256 TMEM columns, ~97 KB shared
-// memory and <= 168 registers each), so one CTA's softmax overlaps the other's
-// MMAs and both keep the exp unit busy.  Work items are (128-row query tile,
+// Persistent kernel: two CTAs per SM at D <= 64 (256 TMEM columns, ~97 KB
+// shared memory and <= 168 registers each), so one CTA's softmax overlaps the
+// other's MMAs and both keep the exp unit busy; one CTA per SM at D = 128
+// (320 TMEM columns, 192 KB of tiles).  Rows of D = 128 are kept as two
+// 64-column slabs with the 128-byte swizzle; the S MMAs run over both slabs
+// and the PV MMA's N = 128 spans them.  Work items are (128-row query tile,
 // head) pairs ordered heaviest first (most key tiles under the causal mask);
 // CTA c takes items c, 2G-1-c, 2G+c, ... (a snake over rounds of G = grid size
 // items), which balances the causal work as well as greedy longest-first.
@@ -48,7 +51,9 @@ constexpr int kBM = 128;          // query rows per CTA (= TMEM lanes)
 constexpr int kBN = 128;          // key rows per tile
 constexpr int kStages = 2;        // K/V ring depth
 constexpr int kThreads = 192;     // 6 warps
-constexpr uint32_t kTmemCols = 256;
+// TMEM columns: 256 at D <= 64, 512 (of which 320 used) at D = 128
+template <int D>
+__host__ __device__ constexpr uint32_t tmem_cols() { return D > 64 ? 512u : 256u; }
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
 
 template <int D>
@@ -73,15 +78,19 @@ __device__ __forceinline__ int item_of(int c, int n, int G, int W) {
 }
 
 template <int D, bool Causal, bool Drop>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16 *__restrict__ o,
                const TStrides so, float *__restrict__ lse, int T, int H, int BH, int ntiles,
                float scale_log2, const DropoutParams dp, int *err) {
     using Smem = FwdSmem<D>;
-    constexpr int kRowBytes = D * 2;                      // 128 (D=64) or 64 (D=32)
-    constexpr uint32_t kSwz = (D == 64) ? kSwizzle128B : kSwizzle64B;
+    constexpr int kSlabCols = D > 64 ? 64 : D;            // columns per swizzle slab
+    constexpr int kSlabs = D / kSlabCols;                 // 1, or 2 at D = 128
+    constexpr int kRowBytes = kSlabCols * 2;              // 128 (D >= 64) or 64 (D = 32)
+    constexpr uint32_t kSwz = (kRowBytes == 128) ? kSwizzle128B : kSwizzle64B;
     constexpr uint32_t kAtom = 8 * kRowBytes;             // 8-row swizzle atom
+    constexpr uint32_t kSlabBytes = 128 * kRowBytes;      // one 128-row slab
+    constexpr uint32_t kTmemCols = tmem_cols<D>();
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                          ~uintptr_t(1023));
@@ -141,7 +150,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int qb = n & 1;
             if (!(ok = mbar_wait_warp(&sm.q_empty[qb], (uint32_t)((n >> 1) & 1) ^ 1u, err, abort))) break;
             mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
-            tma_load_4d_e(sm.q[qb], &tq, &sm.q_full[qb], 0, qt * kBM, hh, bb);
+#pragma unroll
+            for (int sl = 0; sl < kSlabs; ++sl)
+                tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.q[qb]) + sl * kSlabBytes, &tq,
+                              &sm.q_full[qb], sl * kSlabCols, qt * kBM, hh, bb);
             nq = n + 1;
             const int nk = Causal ? qt + 1 : ntiles;  // key tiles this item reads
             for (int j = 0; j < nk; ++j, ++gt) {
@@ -149,14 +161,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
                 if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
                 mbar_arrive_expect_tx_e(&sm.k_full[s], Smem::kTileBytes);
-                tma_load_4d_e(sm.k[s], &tk, &sm.k_full[s], 0, j * kBN, hh, bb);
+#pragma unroll
+                for (int sl = 0; sl < kSlabs; ++sl)
+                    tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.k[s]) + sl * kSlabBytes, &tk,
+                                  &sm.k_full[s], sl * kSlabCols, j * kBN, hh, bb);
                 if (!(ok = mbar_wait_warp(&sm.v_empty[s], ph ^ 1u, err, abort))) {
                     // K of this tile is in flight: let it land before leaving.
                     for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
                     break;
                 }
                 mbar_arrive_expect_tx_e(&sm.v_full[s], Smem::kTileBytes);
-                tma_load_4d_e(sm.v[s], &tv, &sm.v_full[s], 0, j * kBN, hh, bb);
+#pragma unroll
+                for (int sl = 0; sl < kSlabs; ++sl)
+                    tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.v[s]) + sl * kSlabBytes, &tv,
+                                  &sm.v_full[s], sl * kSlabCols, j * kBN, hh, bb);
             }
         }
         // Drain: the last loads this warp issued have landed before exit (on the
@@ -193,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             tc_fence_after();
             // 8 MMAs of K = 16 keys: P from TMEM (8 columns per step), V MN-major
             // (16 rows = kRowBytes 16-byte units per step).
-            const uint64_t vd = smem_desc(smem_u32(sm.v[s]), kBN * kRowBytes, kAtom, kSwz);
+            // (The LBO is the slab stride: N = 128 spans two slabs at D = 128.)
+            const uint64_t vd = smem_desc(smem_u32(sm.v[s]), kSlabBytes, kAtom, kSwz);
             mma_ts_x4<kRowBytes>(tO, tP, vd, idO, pv_j > 0 ? 1u : 0u);
             mma_ts_x4<kRowBytes>(tO, tP + 32, vd + 4 * kRowBytes, idO, 1u);
             mma_commit_e(&sm.o_done);  // PV complete: O stable, P region free
@@ -218,10 +237,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tc_fence_after();
                 // D / 16 MMAs of K = 16: Q and K both K-major (32 bytes per step).
                 const uint64_t kd = smem_desc(smem_u32(sm.k[s]), 16, kAtom, kSwz);
-                if constexpr (D == 64)
+                if constexpr (D == 128) {
                     mma_ss_x4<2, 2>(tS, qd, kd, idS, 0u);
-                else
+                    mma_ss_x4<2, 2>(tS, qd + (kSlabBytes >> 4), kd + (kSlabBytes >> 4), idS, 1u);
+                } else if constexpr (D == 64) {
+                    mma_ss_x4<2, 2>(tS, qd, kd, idS, 0u);
+                } else {
                     mma_ss_x2<2, 2>(tS, qd, kd, idS, 0u);
+                }
                 mma_commit_e(&sm.s_full);
                 mma_commit_e(&sm.k_empty[s]);
                 if (j == nk - 1) mma_commit_e(&sm.q_empty[qb]);  // this item's Q no longer read
@@ -431,12 +454,15 @@ cudaError_t make_map_bf16(void *map, const void *ptr, const Shape &s, const TStr
     if (!enc) return cudaErrorInitializationError;
     const cuuint64_t dims[4] = {(cuuint64_t)s.D, (cuuint64_t)s.T, (cuuint64_t)s.H, (cuuint64_t)s.B};
     const cuuint64_t strides[3] = {(cuuint64_t)st.t * 2, (cuuint64_t)st.h * 2, (cuuint64_t)st.b * 2};
-    const cuuint32_t box[4] = {(cuuint32_t)s.D, 128, 1, 1};
+    // Box: one 128-row slab of at most 64 columns (128 bytes, the swizzle span);
+    // D = 128 rows load as two slabs.
+    const cuuint32_t box_x = s.D > 64 ? 64 : (cuuint32_t)s.D;
+    const cuuint32_t box[4] = {box_x, 128, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r = enc(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                            const_cast<void *>(ptr), dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           s.D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                           box_x * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -455,8 +481,10 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     cudaError_t e0;
     if ((e0 = cudaGetDevice(&dev)) != cudaSuccess) return e0;
     if ((e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e0;
-    // Persistent grid: two CTAs per SM, never more CTAs than work items.
-    const long long grid = items < 2LL * sms ? items : 2LL * sms;
+    // Persistent grid: two CTAs per SM (one at D = 128), never more CTAs than
+    // work items.
+    const long long per_sm = D > 64 ? 1 : 2;
+    const long long grid = items < per_sm * sms ? items : per_sm * sms;
     CUtensorMap mq, mk, mv;
     cudaError_t e;
     if ((e = make_map_bf16(&mq, q, s, str.q)) != cudaSuccess) return e;
@@ -483,6 +511,10 @@ cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
 #define ATTN_FWD_CASE(DD, C, R)                                    \
     if (s.D == DD && (s.causal != 0) == C && s.dropout == R)       \
         return launch_fwd<DD, C, R>(q, k, v, o, lse, s, str, err, st, li);
+    ATTN_FWD_CASE(128, true, false)
+    ATTN_FWD_CASE(128, false, false)
+    ATTN_FWD_CASE(128, true, true)
+    ATTN_FWD_CASE(128, false, true)
     ATTN_FWD_CASE(64, true, false)
     ATTN_FWD_CASE(64, false, false)
     ATTN_FWD_CASE(64, true, true)

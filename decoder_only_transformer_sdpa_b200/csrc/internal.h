@@ -44,8 +44,9 @@ struct BwdStrides {
 };
 
 // Builds a 4-D TMA map over a bf16 [B, H, T, D] view with the given element
-// strides: dimensions (D, T, H, B), box (D, 128, 1, 1), swizzle matching a
-// D * 2-byte row (128 B at D = 64, 64 B at D = 32).
+// strides: dimensions (D, T, H, B), box (min(D, 64), 128, 1, 1), swizzle
+// matching the box row (128 B at D >= 64, 64 B at D = 32); D = 128 tiles load
+// as two 64-column slabs.
 cudaError_t make_map_bf16(void *map, const void *ptr, const Shape &s, const TStrides &st);
 
 // Per-call bookkeeping: kernels enqueued, and the optional event pair to
@@ -84,7 +85,7 @@ cudaError_t simt_bwd(const T *q, const T *k, const T *v, const T *o, const float
                      const T *dO, T *dq, T *dk, T *dv, float *delta, Shape s,
                      cudaStream_t st, LaunchInfo &li);
 
-// ---- tcgen05 / TMA kernels for bf16, D in {32, 64}
+// ---- tcgen05 / TMA kernels for bf16, D in {32, 64, 128}
 cudaError_t sm100_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       __nv_bfloat16 *o, float *lse, Shape s, const FwdStrides &str, int *err,
                       cudaStream_t st, LaunchInfo &li);
@@ -93,6 +94,14 @@ cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv,
                       float *dq_acc, float *lse2, float *delta, Shape s, const BwdStrides &str,
                       int *err, cudaStream_t st, LaunchInfo &li);
+
+// The backward main kernel at D = 128 (prep and post kernels run around it in
+// sm100_bwd).
+cudaError_t sm100_bwd128_main(const __nv_bfloat16 *q, const __nv_bfloat16 *k,
+                              const __nv_bfloat16 *v, const __nv_bfloat16 *dO, __nv_bfloat16 *dk,
+                              __nv_bfloat16 *dv, float *dq_acc, const float *lse2,
+                              const float *delta, const Shape &s, const BwdStrides &str, int *err,
+                              cudaStream_t st, LaunchInfo &li);
 
 // Workspace layout of the bf16 backward (offsets in bytes, each 256-aligned):
 // float32 dQ accumulator [B*H*T*D], then log2-scaled lse and Delta, each

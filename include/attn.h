@@ -76,7 +76,7 @@ const char *attn_status_string(int status);
 
 /* Forward.  q, k, v: bf16 inputs; o: bf16 output; lse: float32 output, the
  * natural-log log-sum-exp of each row's scaled, masked scores (needed by
- * attn_bwd).  D must be 32 or 64.  Any T >= 1. */
+ * attn_bwd).  D must be 32, 64 or 128.  Any T >= 1. */
 int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              int B, int H, int T, int D, float scale, cudaStream_t stream);
 
@@ -90,7 +90,7 @@ size_t attn_bwd_workspace_bytes(int B, int H, int T, int D);
  * upstream gradient; dq, dk, dv: bf16 outputs (fully overwritten).
  * workspace: caller-owned device scratch of at least
  * attn_bwd_workspace_bytes(B,H,T,D) bytes, 256-byte aligned; its contents on
- * entry do not matter and are clobbered.  D must be 32 or 64. */
+ * entry do not matter and are clobbered.  D must be 32, 64 or 128. */
 int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
              const void *dO, void *dq, void *dk, void *dv,
              int B, int H, int T, int D, float scale,

@@ -83,7 +83,7 @@ def fwd32(q=P, o=P, B=1, H=1, T=8, D=8, scale=0.3):
 @pytest.mark.parametrize("kw,expect", [
     (dict(q=None), E_NULL), (dict(lse=None), E_NULL),
     (dict(B=0), E_SHAPE), (dict(H=-1), E_SHAPE), (dict(T=0), E_SHAPE),
-    (dict(D=48), E_D), (dict(D=128), E_D), (dict(D=0), E_D), (dict(D=16), E_D),
+    (dict(D=48), E_D), (dict(D=256), E_D), (dict(D=0), E_D), (dict(D=16), E_D),
     (dict(scale=0.0), E_SCALE), (dict(scale=float("nan")), E_SCALE), (dict(scale=-1.0), E_SCALE),
     (dict(scale=float("inf")), E_SCALE),
     (dict(q=P + 8), E_ALIGN), (dict(o=P + 2), E_ALIGN), (dict(lse=P + 2), E_ALIGN),
