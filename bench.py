@@ -387,7 +387,13 @@ def run_ours(args, w):
                               "tflops": kern[n]["flops"] / (kern[n]["ms"] * 1e-3) / 1e12}
                           for n in kern}}
 
-    # ---- end to end through the public API with pinned host buffers
+    # ---- end to end through the public API with pinned host buffers: every
+    # step uploads its inputs (q, k, v, dO of all layers) and downloads its
+    # results (O, dQ, dK, dV).  Uploads run on one copy stream, downloads on
+    # another, the kernels on the launching stream; events order each layer's
+    # upload before its forward and its downloads after its forward /
+    # backward.  Two device buffer sets alternate between steps, so a step's
+    # uploads overlap the previous step's downloads (the link is full duplex).
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
         host = [{n: b[n].cpu().pin_memory() for n in ("q", "k", "v", "do")} for b in layers]
@@ -395,30 +401,61 @@ def run_ours(args, w):
                      for n in ("o", "dq", "dk", "dv")} for b in layers]
         h2d = sum(t.numel() * t.element_size() for hb in host for t in hb.values())
         d2h = sum(t.numel() * t.element_size() for hb in out_host for t in hb.values())
+        sets = [layers, [{n: torch.empty_like(t) for n, t in b.items()} for b in layers]]
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        released = [None, None]  # per buffer set: its last downloads are done
 
-        def e2e_step():
-            for l, b in enumerate(layers):
-                for n in ("q", "k", "v", "do"):
-                    b[n].copy_(host[l][n], non_blocking=True)
+        def e2e_step(it):
+            bs = sets[it % 2]
+            ev_in, ev_f, ev_b = [], [], [None] * L
+            with torch.cuda.stream(up):
+                if released[it % 2] is not None:
+                    up.wait_event(released[it % 2])
+                for l, b in enumerate(bs):
+                    for n in ("q", "k", "v", "do"):
+                        b[n].copy_(host[l][n], non_blocking=True)
+                    ev_in.append(torch.cuda.Event())
+                    ev_in[-1].record(up)
+            for l, b in enumerate(bs):
+                stream.wait_event(ev_in[l])
                 A.attn_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"])
+                ev_f.append(torch.cuda.Event())
+                ev_f[-1].record(stream)
             for l in range(L - 1, -1, -1):
-                b = layers[l]
+                b = bs[l]
                 A.attn_bwd(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"],
                            b["dv"], workspace=b["ws"])
-                for n in ("o", "dq", "dk", "dv"):
-                    out_host[l][n].copy_(b[n], non_blocking=True)
-        e2e_step()
+                ev_b[l] = torch.cuda.Event()
+                ev_b[l].record(stream)
+            with torch.cuda.stream(down):
+                for l, b in enumerate(bs):
+                    down.wait_event(ev_f[l])
+                    out_host[l]["o"].copy_(b["o"], non_blocking=True)
+                for l in range(L - 1, -1, -1):
+                    down.wait_event(ev_b[l])
+                    for n in ("dq", "dk", "dv"):
+                        out_host[l][n].copy_(bs[l][n], non_blocking=True)
+                released[it % 2] = torch.cuda.Event()
+                released[it % 2].record(down)
+        for it in range(2):
+            e2e_step(it)
+        stream.wait_stream(down)
         barrier()
         s0, s1 = mk(), mk()
         s0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        for it in range(args.e2e_steps):
+            e2e_step(it)
+        stream.wait_stream(up)
+        stream.wait_stream(down)  # the step's results are on the host
         s1.record(stream)
         barrier()
         e2e_ms = reduce_max(s0.elapsed_time(s1), world, dev)
         e2e = {"value": whole_job_tflops(flops_step, world, args.e2e_steps, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps}
+               "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
+               "copies": "uploads and downloads on two copy streams, overlapping the kernels and each "
+                         "other; two device buffer sets alternate between steps"}
+        del sets[1]
 
     # ---- secondary: the same step on the layouts nanoGPT's attention sees
     # (q, k, v slices of a [B, T, 3C] c_attn output; O, dO as [B, T, C];
