@@ -19,15 +19,20 @@
 // items), which balances the causal work as well as greedy longest-first.
 // Barrier phases run on across items, so the next item's Q and K/V tiles
 // stream in and its first S MMA issues while the current item drains.
-// Six warps:
+// Eight warps in two warpgroups:
 //   warp 0      TMA producer: Q of each item into a 2-buffer ring, K_j / V_j
 //               tiles into a 2-stage ring
 //   warp 1      tcgen05 issuer: S = Q K_j^T into TMEM, O += P_j V_j with P_j
 //               read from TMEM; owns the TMEM allocation.  S of the next tile
 //               is issued as soon as the softmax has read the current one.
-//   warps 2..5  softmax: one query row per thread (TMEM lane), online max and
+//   warps 2, 3  idle (they complete the first warpgroup)
+//   warps 4..7  softmax: one query row per thread (TMEM lane), online max and
 //               sum in registers, P_j written to TMEM as bf16, lazy rescale of
 //               the O accumulator, final O / l and lse per item.
+// At D <= 64 (two CTAs per SM, 128 registers per thread at launch) the first
+// warpgroup hands registers to the softmax warpgroup with setmaxnreg: 56 and
+// 200 per thread, 128 x 56 + 128 x 200 = the block's 256 x 128; the launch
+// checks that the kernel was built with exactly 128 registers per thread.
 // Key tiles wholly above the diagonal are never loaded; only the diagonal
 // tile applies the element mask.  The score matrix never leaves the SM.
 // Without the mask (Causal = false) every query tile runs over all key tiles
@@ -50,7 +55,12 @@ using namespace sm100;
 constexpr int kBM = 128;          // query rows per CTA (= TMEM lanes)
 constexpr int kBN = 128;          // key rows per tile
 constexpr int kStages = 2;        // K/V ring depth
-constexpr int kThreads = 192;     // 6 warps
+constexpr int kThreads = 256;     // 8 warps (two warpgroups)
+constexpr int kSoftmaxWarp0 = 4;  // first softmax warp (the second warpgroup)
+constexpr int kRegsLaunch = 128;  // registers per thread at launch (D <= 64)
+constexpr int kRegsLow = 56;      // first warpgroup after the hand-over
+constexpr int kRegsHigh = 200;    // softmax warpgroup after the hand-over
+static_assert(kRegsLow + kRegsHigh == 2 * kRegsLaunch, "the register split must add up");
 // TMEM columns: 256 at D <= 64, 512 (of which 320 used) at D = 128
 template <int D>
 __host__ __device__ constexpr uint32_t tmem_cols() { return D > 64 ? 512u : 256u; }
@@ -129,7 +139,9 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
     const uint32_t tS = tmem;
     const uint32_t tP = tmem + 128;
     const uint32_t tO = tmem + 192;
-
+    if (warp < kSoftmaxWarp0) {
+    // ==================================================== first warpgroup
+    if constexpr (D <= 64) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (whole warp,
         // one elected lane issues)
@@ -259,8 +271,11 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
         // All MMAs this warp issued are complete once `drain` fires.
         mma_commit_e(&sm.drain);
         mbar_wait_warp(&sm.drain, 0, err, abort);
+    }
     } else {
-        // ------------------------------------------------ softmax warps
+    // ==================================================== softmax warpgroup
+    if constexpr (D <= 64) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+    {
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
         const int row = quad * 32 + lane;          // row within the query tile
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -437,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
             }
         }
     }
+    }
 
     tc_fence_before();
     __syncthreads();
@@ -494,6 +510,17 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if ((e = cudaFuncSetAttribute(fwd_kernel<D, Causal, Drop>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
+    if constexpr (D <= 64) {
+        // The setmaxnreg hand-over assumes the block holds 256 x 128
+        // registers; any other build would make the increase wait forever.
+        static int checked = 0;  // 0 unknown, 1 good, -1 bad
+        if (checked == 0) {
+            cudaFuncAttributes fa;
+            if ((e = cudaFuncGetAttributes(&fa, fwd_kernel<D, Causal, Drop>)) != cudaSuccess) return e;
+            checked = (fa.numRegs == kRegsLaunch) ? 1 : -1;
+        }
+        if (checked < 0) return cudaErrorInvalidConfiguration;
+    }
     const float scale_log2 = s.scale * 1.4426950408889634f;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     fwd_kernel<D, Causal, Drop><<<(unsigned)grid, kThreads, smem, st>>>(
