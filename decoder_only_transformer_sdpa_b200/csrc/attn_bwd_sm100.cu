@@ -24,17 +24,23 @@
 //          reduce-add;
 //   post   dQ = scale * accumulator, rounded to bf16.
 //
-// Main kernel, fourteen warps:
+// Main kernel, sixteen warps in four warpgroups:
 //   warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, Delta_i per tile
 //               into a 3-stage ring (a stage is released after dK_i, since
 //               dQ_i reads neither Q nor dO)
 //   warp 1      tcgen05 issuer, TMEM owner
-//   warps 2..9  softmax gradient, two warps per TMEM lane quadrant (one per
+//   warps 2, 3  idle (they complete the first warpgroup)
+//   warps 4..11 softmax gradient, two warps per TMEM lane quadrant (one per
 //               64-query half): per key row (TMEM lane) P^T = exp2(S^T - lse),
 //               dS^T = P^T (dP^T - Delta); P^T to TMEM (bf16), dS^T to shared
 //               memory (bf16, double buffered); final dK (first half) and dV
 //               (second half) epilogue
-//   warps 10..13 dQ drain: TMEM -> swizzled shared staging -> TMA reduce-add
+//   warps 12..15 dQ drain: TMEM -> swizzled shared staging -> TMA reduce-add
+// The block launches with 512 x 128 registers (the whole register file);
+// setmaxnreg then gives the first warpgroup 56, the drain warpgroup 104 and
+// the two softmax-gradient warpgroups 176 each (56 + 104 + 2 x 176 = 4 x 128),
+// so the elementwise warps keep their 32-element chunks in flight without
+// spilling.  The launch checks the build has exactly 128 registers per thread.
 //
 // Per query tile the issuer runs S^T = K Q^T and dP^T = V dO^T (M = key rows),
 // then, once the softmax gradient of that tile is ready, dV += P^T dO (A from
@@ -61,8 +67,15 @@ namespace {
 using namespace sm100;
 
 constexpr int kBT = 128;          // rows per tile (keys and queries)
-constexpr int kThreads = 448;     // 14 warps
-constexpr int kEwThreads = 256;   // softmax-gradient threads (warps 2..9)
+constexpr int kThreads = 512;     // 16 warps (four warpgroups)
+constexpr int kEwThreads = 256;   // softmax-gradient threads (warps 4..11)
+constexpr int kEwWarp0 = 4;       // first softmax-gradient warp
+constexpr int kDrainWarp0 = 12;   // first dQ-drain warp
+constexpr int kRegsLaunch = 128;  // registers per thread at launch
+constexpr int kRegsIssue = 56;    // producer / MMA warpgroup after the hand-over
+constexpr int kRegsEw = 176;      // softmax-gradient warpgroups
+constexpr int kRegsDrain = 104;   // drain warpgroup
+static_assert(kRegsIssue + kRegsDrain + 2 * kRegsEw == 4 * kRegsLaunch, "the register split must add up");
 constexpr int kQStages = 3;       // Q / dO / lse / Delta ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -217,6 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D, tdQ = tmem + 256 + 2 * D;
     const uint32_t tP = tmem + 256 + 3 * D;
 
+    if (warp < kEwWarp0) {
+    // ==================================================== first warpgroup
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIssue));
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (whole warp,
         // one elected lane issues)
@@ -312,10 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit_e(&sm.acc_done);
         mma_commit_e(&sm.drain);
         mbar_wait_warp(&sm.drain, 0, err, abort);
-    } else if (warp < 10) {
+    }
+    } else if (warp < kDrainWarp0) {
+    // ==================================================== softmax-gradient warpgroups
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEw));
+    {
         // ------------------------------------------------ softmax gradient
         const int quad = warp & 3;
-        const int half = (warp - 2) >> 2;               // query columns [64 half, 64 half + 64)
+        const int half = (warp - kEwWarp0) >> 2;        // query columns [64 half, 64 half + 64)
         const int kr = quad * 32 + lane;                // key row within the tile (TMEM lane)
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t sw = (uint32_t)(kr & 7);
@@ -439,12 +459,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+    }
     } else {
+    // ==================================================== drain warpgroup
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
+    {
         // ------------------------------------------------ dQ drain
         const int quad = warp & 3;
         const int qr = quad * 32 + lane;                // query row within the tile
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const bool leader = (warp == 10 && lane == 0);
+        const bool leader = (warp == kDrainWarp0 && lane == 0);
         const uint32_t sw = (uint32_t)(qr & 7);
         for (int idx = 0; idx < n_q; ++idx) {
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, (uint32_t)idx & 1u, err, abort));
@@ -476,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (leader) bulk_wait_all();
+    }
     }
 
     tc_fence_before();
@@ -531,6 +556,17 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     li.kernels += 1;
 
     const size_t smem = sizeof(BwdSmem<D>) + 1024;
+    {
+        // The setmaxnreg hand-over assumes the block holds 512 x 128
+        // registers; any other build would make the increases wait forever.
+        static int checked = 0;  // 0 unknown, 1 good, -1 bad
+        if (checked == 0) {
+            cudaFuncAttributes fa;
+            if ((e = cudaFuncGetAttributes(&fa, bwd_main_kernel<D, Causal, Drop>)) != cudaSuccess) return e;
+            checked = (fa.numRegs == kRegsLaunch) ? 1 : -1;
+        }
+        if (checked < 0) return cudaErrorInvalidConfiguration;
+    }
     if ((e = cudaFuncSetAttribute(bwd_main_kernel<D, Causal, Drop>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
