@@ -76,7 +76,7 @@ constexpr int kRegsIssue = 56;    // producer / MMA warpgroup after the hand-ove
 constexpr int kRegsEw = 176;      // softmax-gradient warpgroups
 constexpr int kRegsDrain = 104;   // drain warpgroup
 static_assert(kRegsIssue + kRegsDrain + 2 * kRegsEw == 4 * kRegsLaunch, "the register split must add up");
-constexpr int kQStages = 3;       // Q / dO / lse / Delta ring depth
+constexpr int kQStages = 2;       // Q / dO / lse / Delta ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -85,17 +85,17 @@ struct BwdSmem {
     static constexpr int kTileBytes = kBT * D * 2;
     alignas(1024) __nv_bfloat16 q[kQStages][kBT * D];
     alignas(1024) __nv_bfloat16 dO[kQStages][kBT * D];
-    alignas(1024) __nv_bfloat16 k[kBT * D];
-    alignas(1024) __nv_bfloat16 v[kBT * D];
+    alignas(1024) __nv_bfloat16 k[2][kBT * D];   // double buffered across work items
+    alignas(1024) __nv_bfloat16 v[2][kBT * D];
     // dS^T, [buffer][query half][key row][64 queries], 128-byte swizzled rows
     alignas(1024) __nv_bfloat16 ds[2][2][kBT * 64];
     // dQ staging for the TMA reduce: one 32-column box [row][32 floats], swizzled
     alignas(1024) float stage[kBT * 32];
     alignas(16) float lse2[kQStages][kBT];
     alignas(16) float delta[kQStages][kBT];
-    uint64_t kv_full, qdo_full[kQStages], qdo_empty[kQStages];
+    uint64_t kv_full[2], kv_empty[2], qdo_full[kQStages], qdo_empty[kQStages];
     uint64_t sdp_full, sdp_free, p_ready[2], ds_ready[2], p_free, ds_free[2];
-    uint64_t dq_full, dq_free, acc_done, drain;
+    uint64_t dq_full, dq_free, acc_done, acc_free, drain;
     uint32_t tmem_slot;
     int abort;
 };
@@ -174,6 +174,13 @@ __global__ void bwd_post_kernel(const float4 *__restrict__ acc, __nv_bfloat16 *_
 
 // ------------------------------------------------------------------ main
 
+// The n-th work item of CTA c in a grid of G CTAs over W items ordered
+// heaviest first (snake order: c, 2G - 1 - c, 2G + c, ...), or -1.
+__device__ __forceinline__ int item_of(int c, int n, int G, int W) {
+    const long long w = (long long)n * G + ((n & 1) ? (G - 1 - c) : c);
+    return w < W ? (int)w : -1;
+}
+
 template <int D, bool Causal, bool Drop>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -194,14 +201,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort = &sm.abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kt = (int)(blockIdx.x / BH);  // key tile; tile 0 sees the most query tiles
-    const int bh = (int)(blockIdx.x % BH);
-    const int hh = bh % H, bb = bh / H;
-    const int q_first = Causal ? kt : 0;    // query tiles q_first .. nt-1
-    const int n_q = nt - q_first;
+    const int G = (int)gridDim.x, cta = (int)blockIdx.x;
+    const int W = nt * BH;  // work items; item w is key tile w / BH (tile 0 heaviest) of head w % BH
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+        }
         for (int s = 0; s < kQStages; ++s) {
             mbar_init(&sm.qdo_full[s], 1);
             mbar_init(&sm.qdo_empty[s], 1);
@@ -217,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sm.dq_full, 1);
         mbar_init(&sm.dq_free, kBT);
         mbar_init(&sm.acc_done, 1);
+        mbar_init(&sm.acc_free, kEwThreads);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -235,7 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIssue));
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (whole warp,
-        // one elected lane issues)
+        // one elected lane issues): per item, K and V into buffer n & 1 (once
+        // the MMAs of item n - 2 released it), then Q, dO, lse, Delta of its
+        // query tiles through the ring (g counts the CTA's tiles).
         if (lane == 0) {
             prefetch_tensormap(&tq);
             prefetch_tensormap(&tk);
@@ -243,89 +253,117 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tdo);
         }
         __syncwarp();
-        mbar_arrive_expect_tx_e(&sm.kv_full, 2 * Smem::kTileBytes);
-        tma_load_4d_e(sm.k, &tk, &sm.kv_full, 0, kt * kBT, hh, bb);
-        tma_load_4d_e(sm.v, &tv, &sm.kv_full, 0, kt * kBT, hh, bb);
-        int issued = 0;
-        for (int idx = 0; idx < n_q; ++idx) {
-            const int st = idx % kQStages;
-            const int i = q_first + idx;
-            if (!mbar_wait_warp(&sm.qdo_empty[st], (uint32_t)((idx / kQStages) & 1) ^ 1u, err, abort)) break;
-            mbar_arrive_expect_tx_e(&sm.qdo_full[st], 2 * Smem::kTileBytes + 2 * kBT * 4);
-            tma_load_4d_e(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, hh, bb);
-            tma_load_4d_e(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, hh, bb);
-            const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
-            bulk_load_e(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
-            bulk_load_e(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
-            issued = idx + 1;
+        int g = 0, n_items = 0;
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            const int w = item_of(cta, n, G, W);
+            if (w < 0) break;
+            const int kt = w / BH, bh = w % BH, hh = bh % H, bb = bh / H;
+            const int q_first = Causal ? kt : 0;
+            const int kb = n & 1;
+            if (n >= 2 && !(ok = mbar_wait_warp(&sm.kv_empty[kb], (uint32_t)((n >> 1) - 1) & 1u, err, abort)))
+                break;
+            mbar_arrive_expect_tx_e(&sm.kv_full[kb], 2 * Smem::kTileBytes);
+            tma_load_4d_e(sm.k[kb], &tk, &sm.kv_full[kb], 0, kt * kBT, hh, bb);
+            tma_load_4d_e(sm.v[kb], &tv, &sm.kv_full[kb], 0, kt * kBT, hh, bb);
+            n_items = n + 1;
+            for (int i = q_first; i < nt; ++i, ++g) {
+                const int st = g % kQStages;
+                if (!(ok = mbar_wait_warp(&sm.qdo_empty[st], (uint32_t)((g / kQStages) & 1) ^ 1u, err, abort))) break;
+                mbar_arrive_expect_tx_e(&sm.qdo_full[st], 2 * Smem::kTileBytes + 2 * kBT * 4);
+                tma_load_4d_e(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, hh, bb);
+                tma_load_4d_e(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, hh, bb);
+                const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
+                bulk_load_e(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
+                bulk_load_e(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
+            }
         }
-        for (int idx = (issued > kQStages ? issued - kQStages : 0); idx < issued; ++idx)
-            for (uint32_t n = 0; n < kWaitLimit && !mbar_try_wait(&sm.qdo_full[idx % kQStages], (uint32_t)(idx / kQStages) & 1u); ++n) {}
-        mbar_wait_warp(&sm.kv_full, 0, err, abort);
+        // The last loads issued have landed before the CTA leaves.
+        for (int x = (g > kQStages ? g - kQStages : 0); x < g; ++x)
+            for (uint32_t m = 0; m < kWaitLimit && !mbar_try_wait(&sm.qdo_full[x % kQStages], (uint32_t)(x / kQStages) & 1u); ++m) {}
+        for (int n = (n_items > 2 ? n_items - 2 : 0); n < n_items; ++n)
+            for (uint32_t m = 0; m < kWaitLimit && !mbar_try_wait(&sm.kv_full[n & 1], (uint32_t)(n >> 1) & 1u); ++m) {}
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (whole warp,
         // one elected lane issues)
         constexpr uint32_t idS = idesc_bf16(kBT, kBT, 0, 0);  // S^T, dP^T: both K-major
         constexpr uint32_t idKV = idesc_bf16(kBT, D, 0, 1);   // dV, dK: A K-major/TMEM, B MN-major
         constexpr uint32_t idQ = idesc_bf16(kBT, D, 1, 1);    // dQ: A (dS) and B (K) MN-major
-        // K and V as K-major operands (S^T, dP^T) and K as the MN-major B of dQ.
-        const uint64_t kd_k = smem_desc(smem_u32(sm.k), 16, kAtom, kSwz);
-        const uint64_t vd_k = smem_desc(smem_u32(sm.v), 16, kAtom, kSwz);
-        const uint64_t kd_mn = smem_desc(smem_u32(sm.k), kBT * kRowBytes, kAtom, kSwz);
-        bool ok = mbar_wait_warp(&sm.kv_full, 0, err, abort);
-        for (int idx = 0; ok && idx <= n_q; ++idx) {
-            if (idx < n_q) {
-                const int st = idx % kQStages;
-                if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(idx / kQStages) & 1u, err, abort))) break;
-                if (idx >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(idx - 1) & 1u, err, abort))) break;
-                tc_fence_after();
-                // S^T = K Q^T and dP^T = V dO^T: D / 16 MMAs each, all operands
-                // K-major (32 bytes per step).
-                const uint64_t qd = smem_desc(smem_u32(sm.q[st]), 16, kAtom, kSwz);
-                const uint64_t dod = smem_desc(smem_u32(sm.dO[st]), 16, kAtom, kSwz);
-                if constexpr (D == 64) {
-                    mma_ss_x4<2, 2>(tS, kd_k, qd, idS, 0u);
-                    mma_ss_x4<2, 2>(tdP, vd_k, dod, idS, 0u);
-                } else {
-                    mma_ss_x2<2, 2>(tS, kd_k, qd, idS, 0u);
-                    mma_ss_x2<2, 2>(tdP, vd_k, dod, idS, 0u);
+        int g0 = 0;  // the CTA's tiles before this item
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            const int w = item_of(cta, n, G, W);
+            if (w < 0) break;
+            const int kt = w / BH;
+            const int n_q = nt - (Causal ? kt : 0);
+            const int kb = n & 1;
+            // K and V as K-major operands (S^T, dP^T) and K as the MN-major B of dQ.
+            const uint64_t kd_k = smem_desc(smem_u32(sm.k[kb]), 16, kAtom, kSwz);
+            const uint64_t vd_k = smem_desc(smem_u32(sm.v[kb]), 16, kAtom, kSwz);
+            const uint64_t kd_mn = smem_desc(smem_u32(sm.k[kb]), kBT * kRowBytes, kAtom, kSwz);
+            if (!(ok = mbar_wait_warp(&sm.kv_full[kb], (uint32_t)(n >> 1) & 1u, err, abort))) break;
+            for (int idx = 0; ok && idx <= n_q; ++idx) {
+                if (idx < n_q) {
+                    const int g = g0 + idx, st = g % kQStages;
+                    if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(g / kQStages) & 1u, err, abort))) break;
+                    if (g >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(g - 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    // S^T = K Q^T and dP^T = V dO^T: D / 16 MMAs each, all operands
+                    // K-major (32 bytes per step).
+                    const uint64_t qd = smem_desc(smem_u32(sm.q[st]), 16, kAtom, kSwz);
+                    const uint64_t dod = smem_desc(smem_u32(sm.dO[st]), 16, kAtom, kSwz);
+                    if constexpr (D == 64) {
+                        mma_ss_x4<2, 2>(tS, kd_k, qd, idS, 0u);
+                        mma_ss_x4<2, 2>(tdP, vd_k, dod, idS, 0u);
+                    } else {
+                        mma_ss_x2<2, 2>(tS, kd_k, qd, idS, 0u);
+                        mma_ss_x2<2, 2>(tdP, vd_k, dod, idS, 0u);
+                    }
+                    mma_commit_e(&sm.sdp_full);
                 }
-                mma_commit_e(&sm.sdp_full);
+                if (idx >= 1) {
+                    const int p = idx - 1;  // the item's tile whose gradients are now issued
+                    const int gp = g0 + p, st = gp % kQStages, b = gp & 1;
+                    // MN-major views (16 rows = kRowBytes 16-byte units per K step).
+                    const uint64_t qd_mn = smem_desc(smem_u32(sm.q[st]), kBT * kRowBytes, kAtom, kSwz);
+                    const uint64_t dod_mn = smem_desc(smem_u32(sm.dO[st]), kBT * kRowBytes, kAtom, kSwz);
+                    const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
+                    // dS^T read K-major for dK (32 bytes per step within a 64-query
+                    // half, the second half kHalf further) and MN-major for dQ (16 key
+                    // rows of 128 bytes per step, the two query halves kHalf apart).
+                    const uint64_t dsd_k = smem_desc(ds_addr, 16, 1024, kSwizzle128B);
+                    const uint64_t dsd_mn = smem_desc(ds_addr, kHalf, 1024, kSwizzle128B);
+                    if (!(ok = mbar_wait_warp(&sm.p_ready[b], (uint32_t)(gp >> 1) & 1u, err, abort))) break;
+                    // The item's first dV / dK overwrite the accumulators: the
+                    // previous item's epilogue must have read them.
+                    if (p == 0 && n >= 1 &&
+                        !(ok = mbar_wait_warp(&sm.acc_free, (uint32_t)(n - 1) & 1u, err, abort)))
+                        break;
+                    tc_fence_after();
+                    // dV += P^T dO: 8 MMAs of K = 16 queries, A from TMEM.
+                    mma_ts_x4<kRowBytes>(tdV, tP, dod_mn, idKV, p > 0 ? 1u : 0u);
+                    mma_ts_x4<kRowBytes>(tdV, tP + 32, dod_mn + 4 * kRowBytes, idKV, 1u);
+                    mma_commit_e(&sm.p_free);
+                    if (!(ok = mbar_wait_warp(&sm.ds_ready[b], (uint32_t)(gp >> 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    // dK += dS^T Q: 8 MMAs of K = 16 queries.
+                    mma_ss_x4<2, kRowBytes>(tdK, dsd_k, qd_mn, idKV, p > 0 ? 1u : 0u);
+                    mma_ss_x4<2, kRowBytes>(tdK, dsd_k + (kHalf >> 4), qd_mn + 4 * kRowBytes, idKV, 1u);
+                    mma_commit_e(&sm.qdo_empty[st]);  // Q, dO, lse, Delta of this tile are consumed
+                    if (gp >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(gp - 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    // dQ_i = dS K: 8 MMAs of K = 16 keys, both operands MN-major.
+                    mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn, kd_mn, idQ, 0u);
+                    mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn + 4 * 128, kd_mn + 4 * kRowBytes, idQ, 1u);
+                    mma_commit_e(&sm.dq_full);
+                    mma_commit_e(&sm.ds_free[b]);
+                }
             }
-            if (idx >= 1) {
-                const int p = idx - 1;  // the tile whose gradients are now issued
-                const int st = p % kQStages, b = p & 1;
-                // MN-major views (16 rows = kRowBytes 16-byte units per K step).
-                const uint64_t qd_mn = smem_desc(smem_u32(sm.q[st]), kBT * kRowBytes, kAtom, kSwz);
-                const uint64_t dod_mn = smem_desc(smem_u32(sm.dO[st]), kBT * kRowBytes, kAtom, kSwz);
-                const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
-                // dS^T read K-major for dK (32 bytes per step within a 64-query
-                // half, the second half kHalf further) and MN-major for dQ (16 key
-                // rows of 128 bytes per step, the two query halves kHalf apart).
-                const uint64_t dsd_k = smem_desc(ds_addr, 16, 1024, kSwizzle128B);
-                const uint64_t dsd_mn = smem_desc(ds_addr, kHalf, 1024, kSwizzle128B);
-                if (!(ok = mbar_wait_warp(&sm.p_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
-                tc_fence_after();
-                // dV += P^T dO: 8 MMAs of K = 16 queries, A from TMEM.
-                mma_ts_x4<kRowBytes>(tdV, tP, dod_mn, idKV, p > 0 ? 1u : 0u);
-                mma_ts_x4<kRowBytes>(tdV, tP + 32, dod_mn + 4 * kRowBytes, idKV, 1u);
-                mma_commit_e(&sm.p_free);
-                if (!(ok = mbar_wait_warp(&sm.ds_ready[b], (uint32_t)(p >> 1) & 1u, err, abort))) break;
-                tc_fence_after();
-                // dK += dS^T Q: 8 MMAs of K = 16 queries.
-                mma_ss_x4<2, kRowBytes>(tdK, dsd_k, qd_mn, idKV, p > 0 ? 1u : 0u);
-                mma_ss_x4<2, kRowBytes>(tdK, dsd_k + (kHalf >> 4), qd_mn + 4 * kRowBytes, idKV, 1u);
-                mma_commit_e(&sm.qdo_empty[st]);  // Q, dO, lse, Delta of this tile are consumed
-                if (p >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(p - 1) & 1u, err, abort))) break;
-                tc_fence_after();
-                // dQ_i = dS K: 8 MMAs of K = 16 keys, both operands MN-major.
-                mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn, kd_mn, idQ, 0u);
-                mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn + 4 * 128, kd_mn + 4 * kRowBytes, idQ, 1u);
-                mma_commit_e(&sm.dq_full);
-                mma_commit_e(&sm.ds_free[b]);
-            }
+            if (!ok) break;
+            mma_commit_e(&sm.acc_done);     // this item's dK, dV are complete
+            mma_commit_e(&sm.kv_empty[kb]);  // and its K, V are no longer read
+            g0 += n_q;
         }
-        mma_commit_e(&sm.acc_done);
         mma_commit_e(&sm.drain);
         mbar_wait_warp(&sm.drain, 0, err, abort);
     }
@@ -340,9 +378,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t sw = (uint32_t)(kr & 7);
         bool ok = true;
+        int g0 = 0;  // the CTA's tiles before this item
+        for (int n = 0; ok; ++n) {
+        const int w = item_of(cta, n, G, W);
+        if (w < 0) break;
+        const int kt = w / BH, bh = w % BH, hh = bh % H, bb = bh / H;
+        const int q_first = Causal ? kt : 0;
+        const int n_q = nt - q_first;
         for (int idx = 0; idx < n_q; ++idx) {
-            const int st = idx % kQStages, b = idx & 1;
-            ok = mbar_wait_warp(&sm.sdp_full, (uint32_t)idx & 1u, err, abort);
+            const int g = g0 + idx;
+            const int st = g % kQStages, b = g & 1;
+            ok = mbar_wait_warp(&sm.sdp_full, (uint32_t)g & 1u, err, abort);
             if (!ok) break;
             tc_fence_after();
             const bool diag = Causal && (idx == 0);
@@ -407,10 +453,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (c == 0) {
                     // P^T in TMEM is free once dV of the previous tile completed;
                     // this dS^T buffer once dK/dQ of two tiles ago completed.
-                    bool w = true;
-                    if (idx >= 1) w = mbar_wait(&sm.p_free, (uint32_t)(idx - 1) & 1u, err, abort);
-                    w = w && mbar_wait(&sm.ds_free[b], (uint32_t)((idx >> 1) & 1) ^ 1u, err, abort);
-                    ok = __all_sync(0xffffffffu, w);
+                    bool wt = true;
+                    if (g >= 1) wt = mbar_wait(&sm.p_free, (uint32_t)(g - 1) & 1u, err, abort);
+                    wt = wt && mbar_wait(&sm.ds_free[b], (uint32_t)((g >> 1) & 1) ^ 1u, err, abort);
+                    ok = __all_sync(0xffffffffu, wt);
                     if (!ok) break;
                     tc_fence_after();
                 }
@@ -429,8 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&sm.p_ready[b]);
             mbar_arrive(&sm.ds_ready[b]);
         }
-        // ---- epilogue: dK (times scale) from the first half's warps, dV from the second's
-        if (ok) ok = mbar_wait_warp(&sm.acc_done, 0, err, abort);
+        // ---- epilogue of the item: dK (times scale) from the first half's
+        // warps, dV from the second's; then the accumulators are free
+        if (ok) ok = mbar_wait_warp(&sm.acc_done, (uint32_t)n & 1u, err, abort);
         if (ok) {
             tc_fence_after();
             const int t = kt * kBT + kr;
@@ -458,6 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&sm.acc_free);
+        }
+        g0 += n_q;
         }
     }
     } else {
@@ -470,8 +521,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const bool leader = (warp == kDrainWarp0 && lane == 0);
         const uint32_t sw = (uint32_t)(qr & 7);
-        for (int idx = 0; idx < n_q; ++idx) {
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, (uint32_t)idx & 1u, err, abort));
+        int g = 0;
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+        const int w = item_of(cta, n, G, W);
+        if (w < 0) break;
+        const int kt = w / BH, bh = w % BH;
+        const int q_first = Causal ? kt : 0;
+        for (int idx = 0; idx < nt - q_first; ++idx, ++g) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.dq_full, (uint32_t)g & 1u, err, abort));
             if (!ok) break;
             tc_fence_after();
             uint32_t r[D / 32][32];
@@ -498,6 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_commit();
                 }
             }
+        }
         }
         if (leader) bulk_wait_all();
     }
@@ -538,7 +597,13 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     const int BH = s.B * s.H;
     const int nt = (s.T + kBT - 1) / kBT;
     const int Tpad = nt * kBT;
-    const long long blocks = (long long)nt * BH;
+    const long long items = (long long)nt * BH;
+    int dev = 0, sms = 0;
+    cudaError_t e0;
+    if ((e0 = cudaGetDevice(&dev)) != cudaSuccess) return e0;
+    if ((e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e0;
+    // Persistent grid: one CTA per SM over the (key tile, head) items.
+    const long long blocks = items < sms ? items : sms;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     CUtensorMap mq, mk, mv, mdo, mdq;
     cudaError_t e;
