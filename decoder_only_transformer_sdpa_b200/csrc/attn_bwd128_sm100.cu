@@ -111,6 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    grid_dep_wait();
+    grid_dep_launch();
     const uint32_t tmem = sm.tmem_slot;
     const uint32_t tS = tmem, tdP = tmem + 64, tdV = tmem + 128, tdK = tmem + 256;
     const uint32_t tdQ = tmem + 384, tP = tmem + 448;
@@ -433,10 +435,10 @@ cudaError_t launch128(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
         return e;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    bwd128_main_kernel<Causal, Drop><<<(unsigned)blocks, kThreads, smem, st>>>(
-        mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, str.dk, str.dv, s.T, Tpad, s.H, BH, nqt,
-        s.scale * kLog2e, s.scale, s.drop, err);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(bwd128_main_kernel<Causal, Drop>, dim3((unsigned)blocks), dim3(kThreads), smem,
+                        st, mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, str.dk, str.dv, s.T, Tpad, s.H,
+                        BH, nqt, s.scale * kLog2e, s.scale, s.drop, err)) != cudaSuccess)
+        return e;
     li.kernels += 1;
     return mark_main_end(li, st);
 }

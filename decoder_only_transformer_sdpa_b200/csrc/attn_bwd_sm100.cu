@@ -116,6 +116,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
                                                        long long prows, int H, TStrides so,
                                                        TStrides sdo) {
     constexpr int kTpr = D / 8;  // threads per row (a power of two dividing 32)
+    grid_dep_wait();
+    grid_dep_launch();
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long prow = gid / kTpr;
     const int c = (int)(gid - prow * kTpr);
@@ -156,6 +158,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
 __global__ void bwd_post_kernel(const float4 *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
                                 long long n8, float scale, int T, int H, int D, TStrides sdq) {
     const int cpr = D / 8;  // 8-element chunks per row
+    grid_dep_wait();
+    grid_dep_launch();
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
          i += (long long)gridDim.x * blockDim.x) {
         const long long row = i / cpr;
@@ -233,6 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    grid_dep_wait();
+    grid_dep_launch();
     const uint32_t tmem = sm.tmem_slot;
     const uint32_t tS = tmem, tdP = tmem + 128;
     const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D, tdQ = tmem + 256 + 2 * D;
@@ -615,9 +621,10 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
 
     const long long prows = (long long)BH * Tpad;
     const long long prep_threads = prows * (D / 8);
-    bwd_prep_kernel<D><<<(unsigned)((prep_threads + 255) / 256), 256, 0, st>>>(
-        o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows, s.H, str.o, str.dO);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(bwd_prep_kernel<D>, dim3((unsigned)((prep_threads + 255) / 256)), dim3(256), 0,
+                        st, o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows, s.H, str.o, str.dO)) !=
+        cudaSuccess)
+        return e;
     li.kernels += 1;
 
     const size_t smem = sizeof(BwdSmem<D>) + 1024;
@@ -636,19 +643,20 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
                                   (int)smem)) != cudaSuccess)
         return e;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    bwd_main_kernel<D, Causal, Drop><<<(unsigned)blocks, kThreads, smem, st>>>(
-        mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, str.dk, str.dv, s.T, Tpad, s.H, BH, nt,
-        s.scale * kLog2e, s.scale, s.drop, err);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(bwd_main_kernel<D, Causal, Drop>, dim3((unsigned)blocks), dim3(kThreads), smem, st,
+                        mq, mk, mv, mdo, mdq, lse2, delta, dk, dv, str.dk, str.dv, s.T, Tpad, s.H, BH,
+                        nt, s.scale * kLog2e, s.scale, s.drop, err)) != cudaSuccess)
+        return e;
     li.kernels += 1;
     if ((e = mark_main_end(li, st)) != cudaSuccess) return e;
 
     const long long n8 = (long long)BH * s.T * D / 8;
     const long long want = (n8 + 255) / 256;
     const int post_blocks = (int)(want < 148 * 16 ? want : 148 * 16);
-    bwd_post_kernel<<<post_blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc), dq, n8,
-                                                  s.scale, s.T, s.H, D, str.dq);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(bwd_post_kernel, dim3(post_blocks), dim3(256), 0, st,
+                        reinterpret_cast<const float4 *>(dq_acc), dq, n8, s.scale, s.T, s.H, D,
+                        str.dq)) != cudaSuccess)
+        return e;
     li.kernels += 1;
     return cudaSuccess;
 }
@@ -665,10 +673,11 @@ cudaError_t launch_bwd128(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const 
     const int Tpad = (s.T + kBT - 1) / kBT * kBT;
     const long long prows = (long long)BH * Tpad;
     const long long prep_threads = prows * (D / 8);
-    bwd_prep_kernel<D><<<(unsigned)((prep_threads + 255) / 256), 256, 0, st>>>(
-        o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows, s.H, str.o, str.dO);
     cudaError_t e;
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(bwd_prep_kernel<D>, dim3((unsigned)((prep_threads + 255) / 256)), dim3(256), 0,
+                        st, o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows, s.H, str.o, str.dO)) !=
+        cudaSuccess)
+        return e;
     li.kernels += 1;
     if ((e = sm100_bwd128_main(q, k, v, dO, dk, dv, dq_acc, lse2, delta, s, str, err, st, li)) !=
         cudaSuccess)
@@ -676,9 +685,10 @@ cudaError_t launch_bwd128(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const 
     const long long n8 = (long long)BH * s.T * D / 8;
     const long long want = (n8 + 255) / 256;
     const int post_blocks = (int)(want < 148 * 16 ? want : 148 * 16);
-    bwd_post_kernel<<<post_blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc), dq, n8,
-                                                  s.scale, s.T, s.H, D, str.dq);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(bwd_post_kernel, dim3(post_blocks), dim3(256), 0, st,
+                        reinterpret_cast<const float4 *>(dq_acc), dq, n8, s.scale, s.T, s.H, D,
+                        str.dq)) != cudaSuccess)
+        return e;
     li.kernels += 1;
     return cudaSuccess;
 }

@@ -112,9 +112,13 @@ __global__ void __launch_bounds__(kThreads)
         }
         sm.abort = 0;
         fence_mbar_init();
-        // The first tiles start streaming before anything else happens.
         prefetch_tensormap(&tk);
         prefetch_tensormap(&tv);
+    }
+    grid_dep_wait();
+    grid_dep_launch();
+    if (tid == 0) {
+        // The first tiles start streaming before anything else happens.
         for (int n = 0; n < kStages && n < my_tiles; ++n) {
             const int tile = rank + n * cs;
             mbar_arrive_expect_tx(&sm.full[n], 2 * Smem::kTileBytes);
@@ -381,13 +385,17 @@ cudaError_t launch_decode(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const 
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // Programmatic stream serialisation: the kernel's prologue may overlap the
+    // previous grid's tail (it calls grid_dep_wait before touching memory).
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const float qscale = s.scale * kLog2e;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     e = cudaLaunchKernelEx(&cfg, decode_kernel<D, NQ>, mk, mv, q, str.q, o, str.o, lse, s.H, s.Tq,

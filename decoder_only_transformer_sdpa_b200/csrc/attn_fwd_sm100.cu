@@ -135,6 +135,8 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    grid_dep_wait();
+    grid_dep_launch();
     const uint32_t tmem = sm.tmem_slot;
     const uint32_t tS = tmem;
     const uint32_t tP = tmem + 128;
@@ -523,9 +525,10 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     }
     const float scale_log2 = s.scale * 1.4426950408889634f;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
-    fwd_kernel<D, Causal, Drop><<<(unsigned)grid, kThreads, smem, st>>>(
-        mq, mk, mv, o, str.o, lse, s.T, s.H, BH, ntiles, scale_log2, s.drop, err);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(fwd_kernel<D, Causal, Drop>, dim3((unsigned)grid), dim3(kThreads), smem, st,
+                        mq, mk, mv, o, str.o, lse, s.T, s.H, BH, ntiles, scale_log2, s.drop, err)) !=
+        cudaSuccess)
+        return e;
     li.kernels += 1;
     return mark_main_end(li, st);
 }

@@ -57,6 +57,26 @@ struct LaunchInfo {
     cudaEvent_t main_end = nullptr;
 };
 
+// Launches `kernel` with programmatic stream serialisation: its CTAs may be
+// scheduled, and run their prologue (barrier init, TMEM allocation), while the
+// previous grid in the stream drains.  Every kernel launched this way calls
+// grid_dep_wait() before touching global memory.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 // Records li.main_start / li.main_end (when armed) around a main kernel.
 inline cudaError_t mark_main_start(const LaunchInfo &li, cudaStream_t st) {
     return li.main_start ? cudaEventRecord(li.main_start, st) : cudaSuccess;

@@ -127,6 +127,21 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ------------------------------------------------ programmatic dependent launch
+
+// Blocks until every grid this one depends on has completed and its memory
+// writes are visible (returns at once when the launch carried no programmatic
+// dependency).  Each kernel calls it before its first global-memory access,
+// read or write, so that it stays ordered after whatever ran before it.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next grid in the stream begin launching; it still waits for this
+// grid's completion in its own grid_dep_wait.  Called after grid_dep_wait, so
+// at most two grids of the stream are ever resident together.
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- TMEM
 
 // Allocates `ncols` TMEM columns (power of two >= 32); whole warp executes.
