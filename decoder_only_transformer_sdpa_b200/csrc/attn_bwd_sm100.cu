@@ -33,9 +33,10 @@
 //   warps 4..11 softmax gradient, two warps per TMEM lane quadrant (one per
 //               64-query half): per key row (TMEM lane) P^T = exp2(S^T - lse),
 //               dS^T = P^T (dP^T - Delta); P^T to TMEM (bf16), dS^T to shared
-//               memory (bf16, double buffered); final dK (first half) and dV
-//               (second half) epilogue
-//   warps 12..15 dQ drain: TMEM -> swizzled shared staging -> TMA reduce-add
+//               memory (bf16, double buffered)
+//   warps 12..15 dQ drain: TMEM -> swizzled shared staging -> TMA reduce-add;
+//               at the end of each item the dK and dV epilogue, so that the
+//               softmax-gradient warps go straight on to the next item
 // The block launches with 512 x 128 registers (the whole register file);
 // setmaxnreg then gives the first warpgroup 56, the drain warpgroup 104 and
 // the two softmax-gradient warpgroups 176 each (56 + 104 + 2 x 176 = 4 x 128),
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sm.dq_full, 1);
         mbar_init(&sm.dq_free, kBT);
         mbar_init(&sm.acc_done, 1);
-        mbar_init(&sm.acc_free, kEwThreads);
+        mbar_init(&sm.acc_free, kBT);  // the drain warpgroup
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -295,80 +296,95 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idS = idesc_bf16(kBT, kBT, 0, 0);  // S^T, dP^T: both K-major
         constexpr uint32_t idKV = idesc_bf16(kBT, D, 0, 1);   // dV, dK: A K-major/TMEM, B MN-major
         constexpr uint32_t idQ = idesc_bf16(kBT, D, 1, 1);    // dQ: A (dS) and B (K) MN-major
-        int g0 = 0;  // the CTA's tiles before this item
+        // One pass over the CTA's tiles g = 0, 1, ... (all items in order): step
+        // g issues S^T / dP^T of tile g, then the gradients of tile g - 1, so
+        // the first scores of an item go out ahead of the previous item's last
+        // gradients exactly as within an item.  The two items involved keep
+        // their own K/V buffers (kb).
+        int sn = 0, s_idx = 0, s_nq = 0, s_kb = 0;  // item and position of the next S^T tile
+        int pn = -1, p_idx = 0, p_nq = 0, p_kb = 0;  // item and position of the pending gradients
+        bool s_valid = item_of(cta, 0, G, W) >= 0;
         bool ok = true;
-        for (int n = 0; ok; ++n) {
-            const int w = item_of(cta, n, G, W);
-            if (w < 0) break;
-            const int kt = w / BH;
-            const int n_q = nt - (Causal ? kt : 0);
-            const int kb = n & 1;
-            // K and V as K-major operands (S^T, dP^T) and K as the MN-major B of dQ.
-            const uint64_t kd_k = smem_desc(smem_u32(sm.k[kb]), 16, kAtom, kSwz);
-            const uint64_t vd_k = smem_desc(smem_u32(sm.v[kb]), 16, kAtom, kSwz);
-            const uint64_t kd_mn = smem_desc(smem_u32(sm.k[kb]), kBT * kRowBytes, kAtom, kSwz);
-            if (!(ok = mbar_wait_warp(&sm.kv_full[kb], (uint32_t)(n >> 1) & 1u, err, abort))) break;
-            for (int idx = 0; ok && idx <= n_q; ++idx) {
-                if (idx < n_q) {
-                    const int g = g0 + idx, st = g % kQStages;
-                    if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(g / kQStages) & 1u, err, abort))) break;
-                    if (g >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(g - 1) & 1u, err, abort))) break;
-                    tc_fence_after();
-                    // S^T = K Q^T and dP^T = V dO^T: D / 16 MMAs each, all operands
-                    // K-major (32 bytes per step).
-                    const uint64_t qd = smem_desc(smem_u32(sm.q[st]), 16, kAtom, kSwz);
-                    const uint64_t dod = smem_desc(smem_u32(sm.dO[st]), 16, kAtom, kSwz);
-                    if constexpr (D == 64) {
-                        mma_ss_x4<2, 2>(tS, kd_k, qd, idS, 0u);
-                        mma_ss_x4<2, 2>(tdP, vd_k, dod, idS, 0u);
-                    } else {
-                        mma_ss_x2<2, 2>(tS, kd_k, qd, idS, 0u);
-                        mma_ss_x2<2, 2>(tdP, vd_k, dod, idS, 0u);
-                    }
-                    mma_commit_e(&sm.sdp_full);
+        for (int g = 0; ok; ++g) {
+            if (s_valid) {
+                if (s_idx == 0) {
+                    const int kt = item_of(cta, sn, G, W) / BH;
+                    s_nq = nt - (Causal ? kt : 0);
+                    s_kb = sn & 1;
+                    if (!(ok = mbar_wait_warp(&sm.kv_full[s_kb], (uint32_t)(sn >> 1) & 1u, err, abort))) break;
                 }
-                if (idx >= 1) {
-                    const int p = idx - 1;  // the item's tile whose gradients are now issued
-                    const int gp = g0 + p, st = gp % kQStages, b = gp & 1;
-                    // MN-major views (16 rows = kRowBytes 16-byte units per K step).
-                    const uint64_t qd_mn = smem_desc(smem_u32(sm.q[st]), kBT * kRowBytes, kAtom, kSwz);
-                    const uint64_t dod_mn = smem_desc(smem_u32(sm.dO[st]), kBT * kRowBytes, kAtom, kSwz);
-                    const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
-                    // dS^T read K-major for dK (32 bytes per step within a 64-query
-                    // half, the second half kHalf further) and MN-major for dQ (16 key
-                    // rows of 128 bytes per step, the two query halves kHalf apart).
-                    const uint64_t dsd_k = smem_desc(ds_addr, 16, 1024, kSwizzle128B);
-                    const uint64_t dsd_mn = smem_desc(ds_addr, kHalf, 1024, kSwizzle128B);
-                    if (!(ok = mbar_wait_warp(&sm.p_ready[b], (uint32_t)(gp >> 1) & 1u, err, abort))) break;
-                    // The item's first dV / dK overwrite the accumulators: the
-                    // previous item's epilogue must have read them.
-                    if (p == 0 && n >= 1 &&
-                        !(ok = mbar_wait_warp(&sm.acc_free, (uint32_t)(n - 1) & 1u, err, abort)))
-                        break;
-                    tc_fence_after();
-                    // dV += P^T dO: 8 MMAs of K = 16 queries, A from TMEM.
-                    mma_ts_x4<kRowBytes>(tdV, tP, dod_mn, idKV, p > 0 ? 1u : 0u);
-                    mma_ts_x4<kRowBytes>(tdV, tP + 32, dod_mn + 4 * kRowBytes, idKV, 1u);
-                    mma_commit_e(&sm.p_free);
-                    if (!(ok = mbar_wait_warp(&sm.ds_ready[b], (uint32_t)(gp >> 1) & 1u, err, abort))) break;
-                    tc_fence_after();
-                    // dK += dS^T Q: 8 MMAs of K = 16 queries.
-                    mma_ss_x4<2, kRowBytes>(tdK, dsd_k, qd_mn, idKV, p > 0 ? 1u : 0u);
-                    mma_ss_x4<2, kRowBytes>(tdK, dsd_k + (kHalf >> 4), qd_mn + 4 * kRowBytes, idKV, 1u);
-                    mma_commit_e(&sm.qdo_empty[st]);  // Q, dO, lse, Delta of this tile are consumed
-                    if (gp >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(gp - 1) & 1u, err, abort))) break;
-                    tc_fence_after();
-                    // dQ_i = dS K: 8 MMAs of K = 16 keys, both operands MN-major.
-                    mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn, kd_mn, idQ, 0u);
-                    mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn + 4 * 128, kd_mn + 4 * kRowBytes, idQ, 1u);
-                    mma_commit_e(&sm.dq_full);
-                    mma_commit_e(&sm.ds_free[b]);
+                const int st = g % kQStages;
+                if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(g / kQStages) & 1u, err, abort))) break;
+                if (g >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(g - 1) & 1u, err, abort))) break;
+                tc_fence_after();
+                // S^T = K Q^T and dP^T = V dO^T: D / 16 MMAs each, all operands
+                // K-major (32 bytes per step).
+                const uint64_t s_kd_k = smem_desc(smem_u32(sm.k[s_kb]), 16, kAtom, kSwz);
+                const uint64_t s_vd_k = smem_desc(smem_u32(sm.v[s_kb]), 16, kAtom, kSwz);
+                const uint64_t qd = smem_desc(smem_u32(sm.q[st]), 16, kAtom, kSwz);
+                const uint64_t dod = smem_desc(smem_u32(sm.dO[st]), 16, kAtom, kSwz);
+                if constexpr (D == 64) {
+                    mma_ss_x4<2, 2>(tS, s_kd_k, qd, idS, 0u);
+                    mma_ss_x4<2, 2>(tdP, s_vd_k, dod, idS, 0u);
+                } else {
+                    mma_ss_x2<2, 2>(tS, s_kd_k, qd, idS, 0u);
+                    mma_ss_x2<2, 2>(tdP, s_vd_k, dod, idS, 0u);
+                }
+                mma_commit_e(&sm.sdp_full);
+            }
+            if (pn >= 0) {
+                const int p = p_idx;  // the item's tile whose gradients are now issued
+                const int gp = g - 1, st = gp % kQStages, b = gp & 1;
+                // MN-major views (16 rows = kRowBytes 16-byte units per K step).
+                const uint64_t qd_mn = smem_desc(smem_u32(sm.q[st]), kBT * kRowBytes, kAtom, kSwz);
+                const uint64_t dod_mn = smem_desc(smem_u32(sm.dO[st]), kBT * kRowBytes, kAtom, kSwz);
+                const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
+                // K as the MN-major B operand of dQ.
+                const uint64_t p_kd_mn = smem_desc(smem_u32(sm.k[p_kb]), kBT * kRowBytes, kAtom, kSwz);
+                // dS^T read K-major for dK (32 bytes per step within a 64-query
+                // half, the second half kHalf further) and MN-major for dQ (16 key
+                // rows of 128 bytes per step, the two query halves kHalf apart).
+                const uint64_t dsd_k = smem_desc(ds_addr, 16, 1024, kSwizzle128B);
+                const uint64_t dsd_mn = smem_desc(ds_addr, kHalf, 1024, kSwizzle128B);
+                if (!(ok = mbar_wait_warp(&sm.p_ready[b], (uint32_t)(gp >> 1) & 1u, err, abort))) break;
+                // The item's first dV / dK overwrite the accumulators: the
+                // previous item's epilogue must have read them.
+                if (p == 0 && pn >= 1 &&
+                    !(ok = mbar_wait_warp(&sm.acc_free, (uint32_t)(pn - 1) & 1u, err, abort)))
+                    break;
+                tc_fence_after();
+                // dV += P^T dO: 8 MMAs of K = 16 queries, A from TMEM.
+                mma_ts_x4<kRowBytes>(tdV, tP, dod_mn, idKV, p > 0 ? 1u : 0u);
+                mma_ts_x4<kRowBytes>(tdV, tP + 32, dod_mn + 4 * kRowBytes, idKV, 1u);
+                mma_commit_e(&sm.p_free);
+                if (!(ok = mbar_wait_warp(&sm.ds_ready[b], (uint32_t)(gp >> 1) & 1u, err, abort))) break;
+                tc_fence_after();
+                // dK += dS^T Q: 8 MMAs of K = 16 queries.
+                mma_ss_x4<2, kRowBytes>(tdK, dsd_k, qd_mn, idKV, p > 0 ? 1u : 0u);
+                mma_ss_x4<2, kRowBytes>(tdK, dsd_k + (kHalf >> 4), qd_mn + 4 * kRowBytes, idKV, 1u);
+                mma_commit_e(&sm.qdo_empty[st]);  // Q, dO, lse, Delta of this tile are consumed
+                if (gp >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(gp - 1) & 1u, err, abort))) break;
+                tc_fence_after();
+                // dQ_i = dS K: 8 MMAs of K = 16 keys, both operands MN-major.
+                mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn, p_kd_mn, idQ, 0u);
+                mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn + 4 * 128, p_kd_mn + 4 * kRowBytes, idQ, 1u);
+                mma_commit_e(&sm.dq_full);
+                mma_commit_e(&sm.ds_free[b]);
+                if (p == p_nq - 1) {
+                    mma_commit_e(&sm.acc_done);        // this item's dK, dV are complete
+                    mma_commit_e(&sm.kv_empty[p_kb]);  // and its K, V are no longer read
                 }
             }
-            if (!ok) break;
-            mma_commit_e(&sm.acc_done);     // this item's dK, dV are complete
-            mma_commit_e(&sm.kv_empty[kb]);  // and its K, V are no longer read
-            g0 += n_q;
+            if (!s_valid) break;
+            // Tile g's gradients are issued at the next step.
+            pn = sn;
+            p_idx = s_idx;
+            p_nq = s_nq;
+            p_kb = s_kb;
+            if (++s_idx == s_nq) {
+                s_idx = 0;
+                s_valid = item_of(cta, ++sn, G, W) >= 0;
+            }
         }
         mma_commit_e(&sm.drain);
         mbar_wait_warp(&sm.drain, 0, err, abort);
@@ -388,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int n = 0; ok; ++n) {
         const int w = item_of(cta, n, G, W);
         if (w < 0) break;
-        const int kt = w / BH, bh = w % BH, hh = bh % H, bb = bh / H;
+        const int kt = w / BH, bh = w % BH;
         const int q_first = Causal ? kt : 0;
         const int n_q = nt - q_first;
         for (int idx = 0; idx < n_q; ++idx) {
@@ -481,39 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&sm.p_ready[b]);
             mbar_arrive(&sm.ds_ready[b]);
         }
-        // ---- epilogue of the item: dK (times scale) from the first half's
-        // warps, dV from the second's; then the accumulators are free
-        if (ok) ok = mbar_wait_warp(&sm.acc_done, (uint32_t)n & 1u, err, abort);
-        if (ok) {
-            tc_fence_after();
-            const int t = kt * kBT + kr;
-            const uint32_t src = half == 0 ? tdK : tdV;
-            const float mul = half == 0 ? scale : (Drop ? dp.keep_scale : 1.f);
-            const TStrides so = half == 0 ? sdk : sdv;
-            __nv_bfloat16 *out = (half == 0 ? dk : dv) + (long long)bb * so.b + (long long)hh * so.h +
-                                 (long long)t * so.t;
-#pragma unroll
-            for (int c = 0; c < D; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(src + lane_off + c, r);
-                tmem_wait_ld();
-                reg_fence32(r);
-                if (t < T) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + c);
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        uint4 w4;
-                        w4.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * mul, __uint_as_float(r[8 * x + 1]) * mul);
-                        w4.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * mul, __uint_as_float(r[8 * x + 3]) * mul);
-                        w4.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * mul, __uint_as_float(r[8 * x + 5]) * mul);
-                        w4.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * mul, __uint_as_float(r[8 * x + 7]) * mul);
-                        dst[x] = w4;
-                    }
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&sm.acc_free);
-        }
         g0 += n_q;
         }
     }
@@ -563,6 +546,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        if (!ok) break;
+        // ---- epilogue of the item: dK (times scale) and dV (times the keep
+        // scale) leave TMEM as bf16 rows (TMEM lane = key row); then the
+        // accumulators are free for the next item's first dV / dK MMAs
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_done, (uint32_t)n & 1u, err, abort));
+        if (!ok) break;
+        tc_fence_after();
+        {
+            const int hh = bh % H, bb = bh / H;
+            const int t = kt * kBT + qr;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t src = which == 0 ? tdK : tdV;
+                const float mul = which == 0 ? scale : (Drop ? dp.keep_scale : 1.f);
+                const TStrides so = which == 0 ? sdk : sdv;
+                __nv_bfloat16 *out = (which == 0 ? dk : dv) + (long long)bb * so.b +
+                                     (long long)hh * so.h + (long long)t * so.t;
+                uint32_t r[D / 32][32];
+#pragma unroll
+                for (int h = 0; h < D / 32; ++h) tmem_ld32(src + lane_off + 32 * h, r[h]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < D / 32; ++h) reg_fence32(r[h]);
+                if (t < T) {
+#pragma unroll
+                    for (int h = 0; h < D / 32; ++h) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(out + 32 * h);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            uint4 w4;
+                            w4.x = pack_bf16x2(__uint_as_float(r[h][8 * x + 0]) * mul, __uint_as_float(r[h][8 * x + 1]) * mul);
+                            w4.y = pack_bf16x2(__uint_as_float(r[h][8 * x + 2]) * mul, __uint_as_float(r[h][8 * x + 3]) * mul);
+                            w4.z = pack_bf16x2(__uint_as_float(r[h][8 * x + 4]) * mul, __uint_as_float(r[h][8 * x + 5]) * mul);
+                            w4.w = pack_bf16x2(__uint_as_float(r[h][8 * x + 6]) * mul, __uint_as_float(r[h][8 * x + 7]) * mul);
+                            dst[x] = w4;
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(&sm.acc_free);
         }
         if (leader) bulk_wait_all();
     }
