@@ -28,8 +28,9 @@
 //   warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, Delta_i per tile
 //               into a 3-stage ring (a stage is released after dK_i, since
 //               dQ_i reads neither Q nor dO)
-//   warp 1      tcgen05 issuer, TMEM owner
-//   warps 2, 3  idle (they complete the first warpgroup)
+//   warp 1      tcgen05 issuer of S^T and dP^T, TMEM owner
+//   warp 2      idle (it completes the first warpgroup)
+//   warp 3      tcgen05 issuer of dV, dK and dQ
 //   warps 4..11 softmax gradient, two warps per TMEM lane quadrant (one per
 //               64-query half): per key row (TMEM lane) P^T = exp2(S^T - lse),
 //               dS^T = P^T (dP^T - Delta); P^T to TMEM (bf16), dS^T to shared
@@ -43,11 +44,14 @@
 // so the elementwise warps keep their 32-element chunks in flight without
 // spilling.  The launch checks the build has exactly 128 registers per thread.
 //
-// Per query tile the issuer runs S^T = K Q^T and dP^T = V dO^T (M = key rows),
-// then, once the softmax gradient of that tile is ready, dV += P^T dO (A from
-// TMEM), dK += dS^T Q and dQ_i = dS K (A read MN-major from the same shared
-// dS^T tile).  The next tile's S^T / dP^T are issued as soon as the current
-// ones have been read out of TMEM, so they overlap the elementwise work.
+// Per query tile the score issuer runs S^T = K Q^T and dP^T = V dO^T (M = key
+// rows); once the softmax gradient of that tile is ready, the gradient issuer
+// runs dV += P^T dO (A from TMEM), dK += dS^T Q and dQ_i = dS K (A read
+// MN-major from the same shared dS^T tile).  The next tile's S^T / dP^T are
+// issued as soon as the current ones have been read out of TMEM, so they
+// overlap the elementwise work; across items the score issuer runs ahead into
+// the next item's K/V buffer while the gradients of the last tile are still
+// being issued.
 //
 // With attention dropout (Drop) the keep bit of (query i, key j) is the one
 // the forward drew (philox.cuh): the eight lanes holding keys 8g .. 8g+7 each
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.kv_empty[s], 2);  // one commit from each tcgen05 stream
         }
         for (int s = 0; s < kQStages; ++s) {
             mbar_init(&sm.qdo_full[s], 1);
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sm.dq_free, kBT);
         mbar_init(&sm.acc_done, 1);
         mbar_init(&sm.acc_free, kBT);  // the drain warpgroup
-        mbar_init(&sm.drain, 1);
+        mbar_init(&sm.drain, 2);  // both tcgen05 streams
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -290,100 +294,99 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (uint32_t m = 0; m < kWaitLimit && !mbar_try_wait(&sm.qdo_full[x % kQStages], (uint32_t)(x / kQStages) & 1u); ++m) {}
         for (int n = (n_items > 2 ? n_items - 2 : 0); n < n_items; ++n)
             for (uint32_t m = 0; m < kWaitLimit && !mbar_try_wait(&sm.kv_full[n & 1], (uint32_t)(n >> 1) & 1u); ++m) {}
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer (whole warp,
-        // one elected lane issues)
+    } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------ tcgen05 issuers (whole
+        // warp, one elected lane issues).  Two independent streams share the
+        // tensor core, so that each warp's waits and bookkeeping overlap the
+        // other's MMAs: warp 1 issues S^T / dP^T of every tile, warp 3 the
+        // gradients dV, dK, dQ.  They touch disjoint TMEM regions, and each
+        // barrier is committed by the stream whose MMAs it tracks (a commit
+        // covers only its own thread's MMAs); the K/V buffer of an item is
+        // released once both streams have committed.
         constexpr uint32_t idS = idesc_bf16(kBT, kBT, 0, 0);  // S^T, dP^T: both K-major
         constexpr uint32_t idKV = idesc_bf16(kBT, D, 0, 1);   // dV, dK: A K-major/TMEM, B MN-major
         constexpr uint32_t idQ = idesc_bf16(kBT, D, 1, 1);    // dQ: A (dS) and B (K) MN-major
-        // One pass over the CTA's tiles g = 0, 1, ... (all items in order): step
-        // g issues S^T / dP^T of tile g, then the gradients of tile g - 1, so
-        // the first scores of an item go out ahead of the previous item's last
-        // gradients exactly as within an item.  The two items involved keep
-        // their own K/V buffers (kb).
-        int sn = 0, s_idx = 0, s_nq = 0, s_kb = 0;  // item and position of the next S^T tile
-        int pn = -1, p_idx = 0, p_nq = 0, p_kb = 0;  // item and position of the pending gradients
-        bool s_valid = item_of(cta, 0, G, W) >= 0;
         bool ok = true;
-        for (int g = 0; ok; ++g) {
-            if (s_valid) {
-                if (s_idx == 0) {
-                    const int kt = item_of(cta, sn, G, W) / BH;
-                    s_nq = nt - (Causal ? kt : 0);
-                    s_kb = sn & 1;
-                    if (!(ok = mbar_wait_warp(&sm.kv_full[s_kb], (uint32_t)(sn >> 1) & 1u, err, abort))) break;
+        int g = 0;  // the CTA's tiles so far
+        for (int n = 0; ok; ++n) {
+            const int w = item_of(cta, n, G, W);
+            if (w < 0) break;
+            const int kt = w / BH;
+            const int n_q = nt - (Causal ? kt : 0);
+            const int kb = n & 1;
+            if (warp == 1) {
+                // ---- score stream
+                if (!(ok = mbar_wait_warp(&sm.kv_full[kb], (uint32_t)(n >> 1) & 1u, err, abort))) break;
+                // K and V as K-major operands.
+                const uint64_t kd_k = smem_desc(smem_u32(sm.k[kb]), 16, kAtom, kSwz);
+                const uint64_t vd_k = smem_desc(smem_u32(sm.v[kb]), 16, kAtom, kSwz);
+                for (int idx = 0; idx < n_q; ++idx, ++g) {
+                    const int st = g % kQStages;
+                    if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(g / kQStages) & 1u, err, abort))) break;
+                    if (g >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(g - 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    // S^T = K Q^T and dP^T = V dO^T: D / 16 MMAs each, all
+                    // operands K-major (32 bytes per step).
+                    const uint64_t qd = smem_desc(smem_u32(sm.q[st]), 16, kAtom, kSwz);
+                    const uint64_t dod = smem_desc(smem_u32(sm.dO[st]), 16, kAtom, kSwz);
+                    if constexpr (D == 64) {
+                        mma_ss_x4<2, 2>(tS, kd_k, qd, idS, 0u);
+                        mma_ss_x4<2, 2>(tdP, vd_k, dod, idS, 0u);
+                    } else {
+                        mma_ss_x2<2, 2>(tS, kd_k, qd, idS, 0u);
+                        mma_ss_x2<2, 2>(tdP, vd_k, dod, idS, 0u);
+                    }
+                    mma_commit_e(&sm.sdp_full);
                 }
-                const int st = g % kQStages;
-                if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(g / kQStages) & 1u, err, abort))) break;
-                if (g >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(g - 1) & 1u, err, abort))) break;
-                tc_fence_after();
-                // S^T = K Q^T and dP^T = V dO^T: D / 16 MMAs each, all operands
-                // K-major (32 bytes per step).
-                const uint64_t s_kd_k = smem_desc(smem_u32(sm.k[s_kb]), 16, kAtom, kSwz);
-                const uint64_t s_vd_k = smem_desc(smem_u32(sm.v[s_kb]), 16, kAtom, kSwz);
-                const uint64_t qd = smem_desc(smem_u32(sm.q[st]), 16, kAtom, kSwz);
-                const uint64_t dod = smem_desc(smem_u32(sm.dO[st]), 16, kAtom, kSwz);
-                if constexpr (D == 64) {
-                    mma_ss_x4<2, 2>(tS, s_kd_k, qd, idS, 0u);
-                    mma_ss_x4<2, 2>(tdP, s_vd_k, dod, idS, 0u);
-                } else {
-                    mma_ss_x2<2, 2>(tS, s_kd_k, qd, idS, 0u);
-                    mma_ss_x2<2, 2>(tdP, s_vd_k, dod, idS, 0u);
+                if (!ok) break;
+                mma_commit_e(&sm.kv_empty[kb]);  // this stream's reads of the item's K, V
+            } else {
+                // ---- gradient stream.  K needs no wait of its own: the first
+                // tile's dS^T exists only after that tile's S^T, which waited
+                // for K and V.
+                const uint64_t kd_mn = smem_desc(smem_u32(sm.k[kb]), kBT * kRowBytes, kAtom, kSwz);
+                for (int p = 0; p < n_q; ++p, ++g) {
+                    const int st = g % kQStages, b = g & 1;
+                    // MN-major views (16 rows = kRowBytes 16-byte units per K step).
+                    const uint64_t qd_mn = smem_desc(smem_u32(sm.q[st]), kBT * kRowBytes, kAtom, kSwz);
+                    const uint64_t dod_mn = smem_desc(smem_u32(sm.dO[st]), kBT * kRowBytes, kAtom, kSwz);
+                    const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
+                    // dS^T read K-major for dK (32 bytes per step within a 64-query
+                    // half, the second half kHalf further) and MN-major for dQ (16
+                    // key rows of 128 bytes per step, the two query halves kHalf
+                    // apart).
+                    const uint64_t dsd_k = smem_desc(ds_addr, 16, 1024, kSwizzle128B);
+                    const uint64_t dsd_mn = smem_desc(ds_addr, kHalf, 1024, kSwizzle128B);
+                    if (!(ok = mbar_wait_warp(&sm.p_ready[b], (uint32_t)(g >> 1) & 1u, err, abort))) break;
+                    // The item's first dV / dK overwrite the accumulators: the
+                    // previous item's epilogue must have read them.
+                    if (p == 0 && n >= 1 &&
+                        !(ok = mbar_wait_warp(&sm.acc_free, (uint32_t)(n - 1) & 1u, err, abort)))
+                        break;
+                    tc_fence_after();
+                    // dV += P^T dO: 8 MMAs of K = 16 queries, A from TMEM.
+                    mma_ts_x4<kRowBytes>(tdV, tP, dod_mn, idKV, p > 0 ? 1u : 0u);
+                    mma_ts_x4<kRowBytes>(tdV, tP + 32, dod_mn + 4 * kRowBytes, idKV, 1u);
+                    mma_commit_e(&sm.p_free);
+                    if (!(ok = mbar_wait_warp(&sm.ds_ready[b], (uint32_t)(g >> 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    // dK += dS^T Q: 8 MMAs of K = 16 queries.
+                    mma_ss_x4<2, kRowBytes>(tdK, dsd_k, qd_mn, idKV, p > 0 ? 1u : 0u);
+                    mma_ss_x4<2, kRowBytes>(tdK, dsd_k + (kHalf >> 4), qd_mn + 4 * kRowBytes, idKV, 1u);
+                    // Q, dO, lse, Delta of this tile are consumed (its S^T / dP^T
+                    // completed before its dS^T existed).
+                    mma_commit_e(&sm.qdo_empty[st]);
+                    if (g >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(g - 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    // dQ_i = dS K: 8 MMAs of K = 16 keys, both operands MN-major.
+                    mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn, kd_mn, idQ, 0u);
+                    mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn + 4 * 128, kd_mn + 4 * kRowBytes, idQ, 1u);
+                    mma_commit_e(&sm.dq_full);
+                    mma_commit_e(&sm.ds_free[b]);
                 }
-                mma_commit_e(&sm.sdp_full);
-            }
-            if (pn >= 0) {
-                const int p = p_idx;  // the item's tile whose gradients are now issued
-                const int gp = g - 1, st = gp % kQStages, b = gp & 1;
-                // MN-major views (16 rows = kRowBytes 16-byte units per K step).
-                const uint64_t qd_mn = smem_desc(smem_u32(sm.q[st]), kBT * kRowBytes, kAtom, kSwz);
-                const uint64_t dod_mn = smem_desc(smem_u32(sm.dO[st]), kBT * kRowBytes, kAtom, kSwz);
-                const uint32_t ds_addr = smem_u32(sm.ds[b][0]);
-                // K as the MN-major B operand of dQ.
-                const uint64_t p_kd_mn = smem_desc(smem_u32(sm.k[p_kb]), kBT * kRowBytes, kAtom, kSwz);
-                // dS^T read K-major for dK (32 bytes per step within a 64-query
-                // half, the second half kHalf further) and MN-major for dQ (16 key
-                // rows of 128 bytes per step, the two query halves kHalf apart).
-                const uint64_t dsd_k = smem_desc(ds_addr, 16, 1024, kSwizzle128B);
-                const uint64_t dsd_mn = smem_desc(ds_addr, kHalf, 1024, kSwizzle128B);
-                if (!(ok = mbar_wait_warp(&sm.p_ready[b], (uint32_t)(gp >> 1) & 1u, err, abort))) break;
-                // The item's first dV / dK overwrite the accumulators: the
-                // previous item's epilogue must have read them.
-                if (p == 0 && pn >= 1 &&
-                    !(ok = mbar_wait_warp(&sm.acc_free, (uint32_t)(pn - 1) & 1u, err, abort)))
-                    break;
-                tc_fence_after();
-                // dV += P^T dO: 8 MMAs of K = 16 queries, A from TMEM.
-                mma_ts_x4<kRowBytes>(tdV, tP, dod_mn, idKV, p > 0 ? 1u : 0u);
-                mma_ts_x4<kRowBytes>(tdV, tP + 32, dod_mn + 4 * kRowBytes, idKV, 1u);
-                mma_commit_e(&sm.p_free);
-                if (!(ok = mbar_wait_warp(&sm.ds_ready[b], (uint32_t)(gp >> 1) & 1u, err, abort))) break;
-                tc_fence_after();
-                // dK += dS^T Q: 8 MMAs of K = 16 queries.
-                mma_ss_x4<2, kRowBytes>(tdK, dsd_k, qd_mn, idKV, p > 0 ? 1u : 0u);
-                mma_ss_x4<2, kRowBytes>(tdK, dsd_k + (kHalf >> 4), qd_mn + 4 * kRowBytes, idKV, 1u);
-                mma_commit_e(&sm.qdo_empty[st]);  // Q, dO, lse, Delta of this tile are consumed
-                if (gp >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(gp - 1) & 1u, err, abort))) break;
-                tc_fence_after();
-                // dQ_i = dS K: 8 MMAs of K = 16 keys, both operands MN-major.
-                mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn, p_kd_mn, idQ, 0u);
-                mma_ss_x4<128, kRowBytes>(tdQ, dsd_mn + 4 * 128, p_kd_mn + 4 * kRowBytes, idQ, 1u);
-                mma_commit_e(&sm.dq_full);
-                mma_commit_e(&sm.ds_free[b]);
-                if (p == p_nq - 1) {
-                    mma_commit_e(&sm.acc_done);        // this item's dK, dV are complete
-                    mma_commit_e(&sm.kv_empty[p_kb]);  // and its K, V are no longer read
-                }
-            }
-            if (!s_valid) break;
-            // Tile g's gradients are issued at the next step.
-            pn = sn;
-            p_idx = s_idx;
-            p_nq = s_nq;
-            p_kb = s_kb;
-            if (++s_idx == s_nq) {
-                s_idx = 0;
-                s_valid = item_of(cta, ++sn, G, W) >= 0;
+                if (!ok) break;
+                mma_commit_e(&sm.acc_done);      // this item's dK, dV are complete
+                mma_commit_e(&sm.kv_empty[kb]);  // and this stream's reads of its K
             }
         }
         mma_commit_e(&sm.drain);
