@@ -22,10 +22,11 @@
 // Eight warps in two warpgroups:
 //   warp 0      TMA producer: Q of each item into a 2-buffer ring, K_j / V_j
 //               tiles into a 2-stage ring
-//   warp 1      tcgen05 issuer: S = Q K_j^T into TMEM, O += P_j V_j with P_j
-//               read from TMEM; owns the TMEM allocation.  S of the next tile
-//               is issued as soon as the softmax has read the current one.
-//   warps 2, 3  idle (they complete the first warpgroup)
+//   warp 1      tcgen05 issuer of S = Q K_j^T into TMEM; owns the TMEM
+//               allocation.  S of the next tile is issued as soon as the
+//               softmax has read the current one.
+//   warp 2      idle (it completes the first warpgroup)
+//   warp 3      tcgen05 issuer of O += P_j V_j with P_j read from TMEM
 //   warps 4..7  softmax: one query row per thread (TMEM lane), online max and
 //               sum in registers, P_j written to TMEM as bf16, lazy rescale of
 //               the O accumulator, final O / l and lse per item.
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.o_final, 1);
         mbar_init(&sm.o_free, kBM);
-        mbar_init(&sm.drain, 1);
+        mbar_init(&sm.drain, 2);  // both tcgen05 streams
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -201,76 +202,73 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
         }
         for (int n = (nq > 2 ? nq - 2 : 0); n < nq; ++n)
             for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.q_full[n & 1], (uint32_t)(n >> 1) & 1u); ++i) {}
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer (whole warp,
-        // one elected lane issues).  Global tile g runs S_g, then PV_{g-1}: the
-        // S of a tile is in flight while the softmax of the previous one runs,
-        // also across item boundaries.
+    } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------ tcgen05 issuers (whole
+        // warp, one elected lane issues).  Two independent streams share the
+        // tensor core so that each warp's waits overlap the other's MMAs: warp
+        // 1 issues S_g = Q K_g^T for every key tile (S_{g+1} is in flight while
+        // the softmax of g runs, also across items), warp 3 issues O += P_g V_g
+        // once the softmax has written P_g.  Each barrier is committed by the
+        // stream whose MMAs it tracks.
         constexpr uint32_t idS = idesc_bf16(kBM, kBN, 0, 0);  // Q, K both K-major
         constexpr uint32_t idO = idesc_bf16(kBM, D, 0, 1);    // P from TMEM, V MN-major
-        // The pending PV (of the previous tile): its global index, item, key
-        // tile index within the item and whether it is the item's last.
-        int pv_g = -1, pv_n = 0, pv_j = 0;
-        bool pv_last = false;
         bool ok = true;
-        auto issue_pv = [&]() -> bool {
-            const int s = pv_g % kStages;
-            if (!mbar_wait_warp(&sm.p_full, (uint32_t)pv_g & 1u, err, abort)) return false;
-            if (!mbar_wait_warp(&sm.v_full[s], (uint32_t)(pv_g / kStages) & 1u, err, abort)) return false;
-            // The first PV of an item overwrites O: the previous item's O must
-            // have been read out by the softmax warps.
-            if (pv_j == 0 && pv_n >= 1 &&
-                !mbar_wait_warp(&sm.o_free, (uint32_t)(pv_n - 1) & 1u, err, abort))
-                return false;
-            tc_fence_after();
-            // 8 MMAs of K = 16 keys: P from TMEM (8 columns per step), V MN-major
-            // (16 rows = kRowBytes 16-byte units per step).
-            // (The LBO is the slab stride: N = 128 spans two slabs at D = 128.)
-            const uint64_t vd = smem_desc(smem_u32(sm.v[s]), kSlabBytes, kAtom, kSwz);
-            mma_ts_x4<kRowBytes>(tO, tP, vd, idO, pv_j > 0 ? 1u : 0u);
-            mma_ts_x4<kRowBytes>(tO, tP + 32, vd + 4 * kRowBytes, idO, 1u);
-            mma_commit_e(&sm.o_done);  // PV complete: O stable, P region free
-            mma_commit_e(&sm.v_empty[s]);
-            if (pv_last) mma_commit_e(&sm.o_final);
-            return true;
-        };
         int gt = 0;
         for (int n = 0; ok; ++n) {
             const int w = item_of(cta, n, G, W);
             if (w < 0) break;
             const int qt = ntiles - 1 - w / BH;
             const int qb = n & 1;
-            if (!(ok = mbar_wait_warp(&sm.q_full[qb], (uint32_t)(n >> 1) & 1u, err, abort))) break;
-            const uint64_t qd = smem_desc(smem_u32(sm.q[qb]), 16, kAtom, kSwz);
             const int nk = Causal ? qt + 1 : ntiles;
-            for (int j = 0; j < nk; ++j, ++gt) {
-                // S_g = Q K_j^T, once the softmax has read S_{g-1} out of TMEM.
-                const int s = gt % kStages;
-                if (!(ok = mbar_wait_warp(&sm.k_full[s], (uint32_t)(gt / kStages) & 1u, err, abort))) break;
-                if (gt >= 1 && !(ok = mbar_wait_warp(&sm.s_free, (uint32_t)(gt - 1) & 1u, err, abort))) break;
-                tc_fence_after();
-                // D / 16 MMAs of K = 16: Q and K both K-major (32 bytes per step).
-                const uint64_t kd = smem_desc(smem_u32(sm.k[s]), 16, kAtom, kSwz);
-                if constexpr (D == 128) {
-                    mma_ss_x4<2, 2>(tS, qd, kd, idS, 0u);
-                    mma_ss_x4<2, 2>(tS, qd + (kSlabBytes >> 4), kd + (kSlabBytes >> 4), idS, 1u);
-                } else if constexpr (D == 64) {
-                    mma_ss_x4<2, 2>(tS, qd, kd, idS, 0u);
-                } else {
-                    mma_ss_x2<2, 2>(tS, qd, kd, idS, 0u);
+            if (warp == 1) {
+                // ---- score stream
+                if (!(ok = mbar_wait_warp(&sm.q_full[qb], (uint32_t)(n >> 1) & 1u, err, abort))) break;
+                const uint64_t qd = smem_desc(smem_u32(sm.q[qb]), 16, kAtom, kSwz);
+                for (int j = 0; j < nk; ++j, ++gt) {
+                    // S_g = Q K_j^T, once the softmax has read S_{g-1} out of TMEM.
+                    const int s = gt % kStages;
+                    if (!(ok = mbar_wait_warp(&sm.k_full[s], (uint32_t)(gt / kStages) & 1u, err, abort))) break;
+                    if (gt >= 1 && !(ok = mbar_wait_warp(&sm.s_free, (uint32_t)(gt - 1) & 1u, err, abort))) break;
+                    tc_fence_after();
+                    // D / 16 MMAs of K = 16: Q and K both K-major (32 bytes per step).
+                    const uint64_t kd = smem_desc(smem_u32(sm.k[s]), 16, kAtom, kSwz);
+                    if constexpr (D == 128) {
+                        mma_ss_x4<2, 2>(tS, qd, kd, idS, 0u);
+                        mma_ss_x4<2, 2>(tS, qd + (kSlabBytes >> 4), kd + (kSlabBytes >> 4), idS, 1u);
+                    } else if constexpr (D == 64) {
+                        mma_ss_x4<2, 2>(tS, qd, kd, idS, 0u);
+                    } else {
+                        mma_ss_x2<2, 2>(tS, qd, kd, idS, 0u);
+                    }
+                    mma_commit_e(&sm.s_full);
+                    mma_commit_e(&sm.k_empty[s]);
+                    if (j == nk - 1) mma_commit_e(&sm.q_empty[qb]);  // this item's Q no longer read
                 }
-                mma_commit_e(&sm.s_full);
-                mma_commit_e(&sm.k_empty[s]);
-                if (j == nk - 1) mma_commit_e(&sm.q_empty[qb]);  // this item's Q no longer read
-                if (pv_g >= 0 && !(ok = issue_pv())) break;
-                pv_g = gt;
-                pv_n = n;
-                pv_j = j;
-                pv_last = (j == nk - 1);
+            } else {
+                // ---- PV stream
+                for (int j = 0; j < nk; ++j, ++gt) {
+                    const int s = gt % kStages;
+                    if (!(ok = mbar_wait_warp(&sm.p_full, (uint32_t)gt & 1u, err, abort))) break;
+                    if (!(ok = mbar_wait_warp(&sm.v_full[s], (uint32_t)(gt / kStages) & 1u, err, abort))) break;
+                    // The first PV of an item overwrites O: the previous item's O
+                    // must have been read out by the softmax warps.
+                    if (j == 0 && n >= 1 &&
+                        !(ok = mbar_wait_warp(&sm.o_free, (uint32_t)(n - 1) & 1u, err, abort)))
+                        break;
+                    tc_fence_after();
+                    // 8 MMAs of K = 16 keys: P from TMEM (8 columns per step), V
+                    // MN-major (16 rows = kRowBytes 16-byte units per step).
+                    // (The LBO is the slab stride: N = 128 spans two slabs at D = 128.)
+                    const uint64_t vd = smem_desc(smem_u32(sm.v[s]), kSlabBytes, kAtom, kSwz);
+                    mma_ts_x4<kRowBytes>(tO, tP, vd, idO, j > 0 ? 1u : 0u);
+                    mma_ts_x4<kRowBytes>(tO, tP + 32, vd + 4 * kRowBytes, idO, 1u);
+                    mma_commit_e(&sm.o_done);  // PV complete: O stable, P region free
+                    mma_commit_e(&sm.v_empty[s]);
+                    if (j == nk - 1) mma_commit_e(&sm.o_final);
+                }
             }
         }
-        if (ok && pv_g >= 0) ok = issue_pv();
-        // All MMAs this warp issued are complete once `drain` fires.
+        // All MMAs of both streams are complete once `drain` fires.
         mma_commit_e(&sm.drain);
         mbar_wait_warp(&sm.drain, 0, err, abort);
     }
