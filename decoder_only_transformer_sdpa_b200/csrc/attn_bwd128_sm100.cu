@@ -13,15 +13,17 @@
 //   * the drain warps transpose dQ^T through a swizzled shared staging tile
 //     and add it into the float32 accumulator with TMA reduce-add.
 //
-// One CTA per (128-row key tile, head), 14 warps:
+// One CTA per (128-row key tile, head), 15 warps:
 //   warp 0      TMA producer: K_j, V_j once (two 64-column slabs each); Q_i,
 //               dO_i (64 rows, two slabs each), lse_i, Delta_i per sub-tile
 //               into a 2-stage ring
-//   warp 1      tcgen05 issuer, TMEM owner
+//   warp 1      tcgen05 issuer of S^T and dP^T, TMEM owner
 //   warps 2..9  softmax gradient: two warps per TMEM lane quadrant (32 key
 //               rows), one per 32-query half of the sub-tile; P^T to TMEM
 //               (bf16), dS^T to shared memory (bf16, double buffered)
 //   warps 10..13 dQ drain: TMEM lane d holds column d of dQ^T
+//   warp 14     tcgen05 issuer of dV, dK and dQ^T (a second stream, so that
+//               each issuer's waits overlap the other's MMAs)
 //
 // TMEM columns: S^T [0,64), dP^T [64,128), dV [128,256), dK [256,384),
 // dQ^T [384,448), P^T (bf16 pairs) [448,480).
@@ -38,7 +40,7 @@ using namespace sm100;
 constexpr int D = 128;
 constexpr int kBK = 128;          // key rows per CTA
 constexpr int kBQ = 64;           // query rows per sub-tile
-constexpr int kThreads = 448;     // 14 warps
+constexpr int kThreads = 480;     // 15 warps
 constexpr int kEwThreads = 256;   // softmax-gradient threads (warps 2..9)
 constexpr int kQStages = 2;       // Q / dO / lse / Delta ring depth
 constexpr uint32_t kTmemCols = 512;
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sm.dq_full, 1);
         mbar_init(&sm.dq_free, 128);
         mbar_init(&sm.acc_done, 1);
-        mbar_init(&sm.drain, 1);
+        mbar_init(&sm.drain, 2);  // both tcgen05 streams
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -149,20 +151,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int idx = (issued > kQStages ? issued - kQStages : 0); idx < issued; ++idx)
             for (uint32_t n = 0; n < kWaitLimit && !mbar_try_wait(&sm.qdo_full[idx % kQStages], (uint32_t)(idx / kQStages) & 1u); ++n) {}
         mbar_wait_warp(&sm.kv_full, 0, err, abort);
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 14) {
+        // ------------------------------------------------ tcgen05 issuers: warp 1
+        // the scores, warp 14 the gradients.  They touch disjoint TMEM, and each
+        // barrier is committed by the stream whose MMAs it tracks (a commit
+        // covers only its own thread's MMAs).
         constexpr uint32_t idS = idesc_bf16(kBK, kBQ, 0, 0);  // S^T, dP^T: M = 128 keys, N = 64 queries
         constexpr uint32_t idKV = idesc_bf16(kBK, D, 0, 1);   // dV, dK: N = 128 columns (B MN-major)
         constexpr uint32_t idQ = idesc_bf16(D, kBQ, 1, 1);    // dQ^T: M = 128 columns, both MN-major
-        // K and V K-major (A of S^T / dP^T; 32 bytes per K step, second slab
-        // kKSlab further) and K MN-major as the A of dQ^T (M = 128 spans the
-        // two slabs: LBO = slab stride; 16 keys = 2048 bytes per K step).
-        const uint64_t kd_k = smem_desc(smem_u32(sm.k[0]), 16, kAtom, kSwizzle128B);
-        const uint64_t vd_k = smem_desc(smem_u32(sm.v[0]), 16, kAtom, kSwizzle128B);
-        const uint64_t kd_mn = smem_desc(smem_u32(sm.k[0]), kKSlab, kAtom, kSwizzle128B);
-        bool ok = mbar_wait_warp(&sm.kv_full, 0, err, abort);
-        for (int idx = 0; ok && idx <= n_q; ++idx) {
-            if (idx < n_q) {
+        bool ok = true;
+        if (warp == 1) {
+            // K and V K-major (A of S^T / dP^T; 32 bytes per K step, second slab
+            // kKSlab further).
+            const uint64_t kd_k = smem_desc(smem_u32(sm.k[0]), 16, kAtom, kSwizzle128B);
+            const uint64_t vd_k = smem_desc(smem_u32(sm.v[0]), 16, kAtom, kSwizzle128B);
+            ok = mbar_wait_warp(&sm.kv_full, 0, err, abort);
+            for (int idx = 0; ok && idx < n_q; ++idx) {
                 const int st = idx % kQStages;
                 if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(idx / kQStages) & 1u, err, abort))) break;
                 if (idx >= 1 && !(ok = mbar_wait_warp(&sm.sdp_free, (uint32_t)(idx - 1) & 1u, err, abort))) break;
@@ -176,8 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_ss_x4<2, 2>(tdP, vd_k + (kKSlab >> 4), dod + (kQSlab >> 4), idS, 1u);
                 mma_commit_e(&sm.sdp_full);
             }
-            if (idx >= 1) {
-                const int p = idx - 1;
+        } else {
+            // K MN-major as the A of dQ^T (M = 128 spans the two slabs: LBO =
+            // slab stride; 16 keys = 2048 bytes per K step).  It needs no wait
+            // of its own: the first dS^T exists only after the first S^T, which
+            // waited for K and V.
+            const uint64_t kd_mn = smem_desc(smem_u32(sm.k[0]), kKSlab, kAtom, kSwizzle128B);
+            for (int p = 0; ok && p < n_q; ++p) {
                 const int st = p % kQStages, b = p & 1;
                 // Q and dO MN-major as B of dK / dV (N = 128 spans two slabs:
                 // LBO = slab stride; 16 queries = 2048 bytes per K step).
@@ -197,7 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 // dK += dS^T Q: 4 MMAs of K = 16 queries.
                 mma_ss_x4<2, 128>(tdK, dsd_k, qd_mn, idKV, p > 0 ? 1u : 0u);
-                mma_commit_e(&sm.qdo_empty[st]);  // Q, dO, lse, Delta of this sub-tile are consumed
+                // Q, dO, lse, Delta of this sub-tile are consumed (its S^T /
+                // dP^T completed before its dS^T existed).
+                mma_commit_e(&sm.qdo_empty[st]);
                 if (p >= 1 && !(ok = mbar_wait_warp(&sm.dq_free, (uint32_t)(p - 1) & 1u, err, abort))) break;
                 tc_fence_after();
                 // dQ^T = K^T dS^T: 8 MMAs of K = 16 keys.
@@ -206,8 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit_e(&sm.dq_full);
                 mma_commit_e(&sm.ds_free[b]);
             }
+            mma_commit_e(&sm.acc_done);
         }
-        mma_commit_e(&sm.acc_done);
         mma_commit_e(&sm.drain);
         mbar_wait_warp(&sm.drain, 0, err, abort);
     } else if (warp < 10) {
