@@ -27,6 +27,13 @@
  *  - All pointers are device pointers owned by the caller.  The library
  *    allocates no device memory, never synchronises the stream and only
  *    enqueues work on `stream` (NULL = the legacy default stream).
+ *  - Stream order is the ordinary one.  The bf16 kernels are launched with
+ *    programmatic stream serialisation, so a kernel's set-up may overlap the
+ *    end of the work before it in the stream.  But each kernel waits for that
+ *    work to complete before it reads or writes any memory, so work enqueued
+ *    earlier (a producer of q, k, v, a reader of the workspace) is fully
+ *    ordered before it.  The calls may be captured into CUDA graphs (after
+ *    one call outside the capture on the device).
  *  - bf16 entry points take __nv_bfloat16 data through `void *`; every tensor
  *    pointer must be 16-byte aligned (TMA requirement).  float32 entry points
  *    need 4-byte alignment.
