@@ -81,6 +81,17 @@ struct FwdSmem {
     int abort;
 };
 
+// Stores a 4-D tile from shared memory through a tensor map (rows past the
+// map's extent are not written); one thread issues, bulk-group tracked.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group"
+        " [%0, {%1, %2, %3, %4}], [%5];" ::"l"(reinterpret_cast<uint64_t>(map)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(src))
+        : "memory");
+}
+
 // The n-th work item of CTA c in a grid of G CTAs over W items (snake order),
 // or -1 when the CTA has no n-th item.
 __device__ __forceinline__ int item_of(int c, int n, int G, int W) {
@@ -91,8 +102,8 @@ __device__ __forceinline__ int item_of(int c, int n, int G, int W) {
 template <int D, bool Causal, bool Drop>
 __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-               const __grid_constant__ CUtensorMap tv, __nv_bfloat16 *__restrict__ o,
-               const TStrides so, float *__restrict__ lse, int T, int H, int BH, int ntiles,
+               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+               float *__restrict__ lse, int T, int H, int BH, int ntiles,
                float scale_log2, const DropoutParams dp, int *err) {
     using Smem = FwdSmem<D>;
     constexpr int kSlabCols = D > 64 ? 64 : D;            // columns per swizzle slab
@@ -242,7 +253,8 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                     }
                     mma_commit_e(&sm.s_full);
                     mma_commit_e(&sm.k_empty[s]);
-                    if (j == nk - 1) mma_commit_e(&sm.q_empty[qb]);  // this item's Q no longer read
+                    // (this item's Q buffer is released by the softmax warps,
+                    // which stage the item's O in it for the TMA store)
                 }
             } else {
                 // ---- PV stream
@@ -430,30 +442,51 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
             tc_fence_before();
             mbar_arrive(&sm.o_free);
             const int t = qt * kBM + row;
-            if (t < T) {
+            // O / l as bf16 into this item's Q buffer, in the swizzled layout
+            // of a TMA tile (every S MMA of the item has completed: the
+            // softmax consumed the last S before the last PV), then one TMA
+            // store per slab; rows past T are not written by the store.
+            {
                 const float inv = (Drop ? dp.keep_scale : 1.f) / l;
-                const size_t grow = (size_t)bh * T + t;
-                __nv_bfloat16 *orow = o + (long long)(bh / H) * so.b + (long long)(bh % H) * so.h +
-                                      (long long)t * so.t;
+                uint8_t *qbuf = reinterpret_cast<uint8_t *>(sm.q[n & 1]);
+                constexpr int kChunks = kRowBytes / 16;  // 16-byte chunks per slab row
+                const uint32_t swz = kRowBytes == 128 ? (uint32_t)(row & 7) : (uint32_t)((row >> 1) & 3);
 #pragma unroll
-                for (int h = 0; h < D / 32; ++h) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * h);
+                for (int sl = 0; sl < kSlabs; ++sl) {
+                    const uint32_t base = smem_u32(qbuf + sl * kSlabBytes) + (uint32_t)row * kRowBytes;
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        uint4 w4;
-                        w4.x = pack_bf16x2(__uint_as_float(r[h][8 * x + 0]) * inv, __uint_as_float(r[h][8 * x + 1]) * inv);
-                        w4.y = pack_bf16x2(__uint_as_float(r[h][8 * x + 2]) * inv, __uint_as_float(r[h][8 * x + 3]) * inv);
-                        w4.z = pack_bf16x2(__uint_as_float(r[h][8 * x + 4]) * inv, __uint_as_float(r[h][8 * x + 5]) * inv);
-                        w4.w = pack_bf16x2(__uint_as_float(r[h][8 * x + 6]) * inv, __uint_as_float(r[h][8 * x + 7]) * inv);
-                        dst[x] = w4;
+                    for (int c = 0; c < kChunks; ++c) {
+                        const int col = sl * kSlabCols + 8 * c;  // first of the chunk's 8 columns
+                        const uint32_t *v = &r[col / 32][col % 32];
+                        st_shared_v4(base + ((c ^ swz) << 4),
+                                     pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
+                                     pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
+                                     pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
+                                     pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
                     }
                 }
+                fence_proxy_async_smem();
+                named_bar_sync(1, kBM);
+                if (warp == kSoftmaxWarp0 && lane == 0) {
+#pragma unroll
+                    for (int sl = 0; sl < kSlabs; ++sl)
+                        tma_store_4d(&to, qbuf + sl * kSlabBytes, sl * kSlabCols, qt * kBM, bh % H, bh / H);
+                    bulk_commit();
+                    // Once the store has read the tile, the buffer takes item n + 2's Q.
+                    bulk_wait_read_all();
+                    mbar_arrive(&sm.q_empty[n & 1]);
+                }
+            }
+            if (t < T) {
+                const size_t grow = (size_t)bh * T + t;
                 lse[grow] = (m_used + log2f(l)) * 0.69314718055994531f;
             }
         }
     }
     }
 
+    // The O stores issued by the first softmax thread have completed.
+    if (warp == kSoftmaxWarp0 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -501,11 +534,12 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     // work items.
     const long long per_sm = D > 64 ? 1 : 2;
     const long long grid = items < per_sm * sms ? items : per_sm * sms;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     cudaError_t e;
     if ((e = make_map_bf16(&mq, q, s, str.q)) != cudaSuccess) return e;
     if ((e = make_map_bf16(&mk, k, s, str.k)) != cudaSuccess) return e;
     if ((e = make_map_bf16(&mv, v, s, str.v)) != cudaSuccess) return e;
+    if ((e = make_map_bf16(&mo, o, s, str.o)) != cudaSuccess) return e;
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
     if ((e = cudaFuncSetAttribute(fwd_kernel<D, Causal, Drop>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
@@ -524,7 +558,7 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     const float scale_log2 = s.scale * 1.4426950408889634f;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     if ((e = launch_pdl(fwd_kernel<D, Causal, Drop>, dim3((unsigned)grid), dim3(kThreads), smem, st,
-                        mq, mk, mv, o, str.o, lse, s.T, s.H, BH, ntiles, scale_log2, s.drop, err)) !=
+                        mq, mk, mv, mo, lse, s.T, s.H, BH, ntiles, scale_log2, s.drop, err)) !=
         cudaSuccess)
         return e;
     li.kernels += 1;
