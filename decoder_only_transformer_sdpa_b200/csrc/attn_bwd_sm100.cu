@@ -26,7 +26,7 @@
 //
 // Main kernel, sixteen warps in four warpgroups:
 //   warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, Delta_i per tile
-//               into a 3-stage ring (a stage is released after dK_i, since
+//               into a 2-stage ring (a stage is released after dK_i, since
 //               dQ_i reads neither Q nor dO)
 //   warp 1      tcgen05 issuer of S^T and dP^T, TMEM owner
 //   warp 2      idle (it completes the first warpgroup)
