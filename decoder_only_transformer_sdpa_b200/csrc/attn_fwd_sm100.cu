@@ -29,7 +29,10 @@
 //   warp 3      tcgen05 issuer of O += P_j V_j with P_j read from TMEM
 //   warps 4..7  softmax: one query row per thread (TMEM lane), online max and
 //               sum in registers, P_j written to TMEM as bf16, lazy rescale of
-//               the O accumulator, final O / l and lse per item.
+//               the O accumulator, final O / l and lse per item (O / l is
+//               staged in the item's Q buffer, no longer read by then, and
+//               written by one TMA store; the buffer then goes back to the
+//               producer).
 // At D <= 64 (two CTAs per SM, 128 registers per thread at launch) the first
 // warpgroup hands registers to the softmax warpgroup with setmaxnreg: 56 and
 // 200 per thread, 128 x 56 + 128 x 200 = the block's 256 x 128; the launch
