@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.q_full[b], 1);
-            mbar_init(&sm.q_empty[b], 1);
+            mbar_init(&sm.q_empty[b], 1);  // the first softmax thread, after the O store read it
         }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
