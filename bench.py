@@ -59,6 +59,8 @@ def parse_args():
                    help="skip the secondary measurement of decode attention")
     p.add_argument("--no-d128", action="store_true",
                    help="skip the secondary measurement at head_dim 128")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the per-workload measurements (char GPT, small-head, GPT-2 XL, tiny fp32)")
     p.add_argument("--layers", type=int, default=None,
                    help="layer instances per step (default: the workload's 12); fewer only for profiling")
     return p.parse_args()
@@ -277,6 +279,99 @@ def run_reference(args, w):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ------------------------------------------------------- per-workload legs
+
+def min_hbm_bytes(w) -> int:
+    """Fewest HBM bytes one forward + backward can move: the forward reads Q,
+    K, V and writes O and lse; the backward reads Q, K, V, O, dO, lse and
+    writes dQ, dK, dV."""
+    n = w.B * w.H * w.T * w.D
+    es = 4 if w.dtype == "f32" else 2
+    return 12 * n * es + 2 * w.B * w.H * w.T * 4
+
+
+def config_leg(A, torch, name, args, rank, world, dev, stream, peaks):
+    """One forward + backward per iteration of the named workload, through the
+    plain entry points, cycling over enough independent input sets that their
+    buffers (outputs and workspace included) exceed twice the L2: no set is
+    still cache-resident when its turn comes again.  Reports fwd+bwd TFLOP/s
+    (causal count), HBM GB/s against the fewest bytes the pass can move, and
+    each main kernel's time from events recorded around it."""
+    from workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[name]
+    f32 = w.dtype == "f32"
+    es = 4 if f32 else 2
+    n = w.B * w.H * w.T * w.D
+    ws_bytes = (A.attn_bwd_f32_workspace_bytes if f32 else A.attn_bwd_workspace_bytes)(w.B, w.H, w.T, w.D)
+    per_set = 8 * n * es + 2 * w.B * w.H * w.T * 4 + ws_bytes
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_sets = max(4, math.ceil(2 * l2 / per_set))
+    sets = []
+    for i in range(n_sets):
+        inp = make_inputs(w, seed=args.seed + 7919 * rank, layer=i)
+        b = {k: inp[k].to(dev) for k in ("q", "k", "v", "do")}
+        b["o"], b["dq"], b["dk"], b["dv"] = (torch.empty_like(b["q"]) for _ in range(4))
+        b["lse"] = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=dev)
+        b["ws"] = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        sets.append(b)
+    fwd = A.attn_fwd_f32 if f32 else A.attn_fwd
+    bwd = A.attn_bwd_f32 if f32 else A.attn_bwd
+    n_it = max(4 * n_sets, min(args.steps, 200))
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [((mk(), mk()), (mk(), mk())) for _ in range(n_it)]
+    for e in evs:
+        for pair in e:
+            for x in pair:
+                x.record(stream)
+
+    def one(i, ev=None):
+        b = sets[i % n_sets]
+        if ev is not None:
+            A.attn_profile_next_call(*ev[0])
+        fwd(b["q"], b["k"], b["v"], b["o"], b["lse"])
+        if ev is not None:
+            A.attn_profile_next_call(*ev[1])
+        bwd(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"], b["dv"], workspace=b["ws"])
+
+    for i in range(max(3, n_sets)):
+        one(i)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    s0, s1 = mk(), mk()
+    s0.record(stream)
+    for i in range(n_it):
+        one(i, evs[i])
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    if A.attn_device_error() != 0:
+        raise RuntimeError(f"a bounded in-kernel wait timed out in the {name} leg")
+    ms = reduce_max(s0.elapsed_time(s1), world, dev) / n_it
+    fm = statistics.mean(e[0][0].elapsed_time(e[0][1]) for e in evs)
+    bm = statistics.mean(e[1][0].elapsed_time(e[1][1]) for e in evs)
+    peak = float(peaks.get("bf16_tflops"))
+    hbm = float(peaks.get("hbm_gbs"))
+    tf = lambda fl, t: fl / (t * 1e-3) / 1e12
+    hb = min_hbm_bytes(w)
+    out = {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} D={w.D} {w.dtype}, causal fwd+bwd",
+           "sets": n_sets, "iterations": n_it,
+           "l2": f"{n_sets} input sets of {per_set / 1e6:.1f} MB rotated (> 2x the {l2 / 1e6:.0f} MB L2)",
+           "ms_per_fwd_bwd": ms, "us_per_fwd_bwd": 1e3 * ms,
+           "tflops": world * tf(w.flops(), ms),
+           "hbm_min_bytes": hb, "gbs": world * hb / (ms * 1e-3) / 1e9,
+           "fwd_main": {"avg_launch_ms": fm, "tflops": tf(w.fwd_flops(), fm)},
+           "bwd_main": {"avg_launch_ms": bm, "tflops": tf(8 * w.D * w.causal_pairs(), bm)}}
+    if not f32:
+        out["frac_of_bf16_peak"] = out["tflops"] / world / peak
+        out["hbm_frac"] = out["gbs"] / world / hbm
+        out["fwd_main"]["frac"] = out["fwd_main"]["tflops"] / peak
+        out["bwd_main"]["frac"] = out["bwd_main"]["tflops"] / peak
+    else:
+        out["bound"] = "launch latency (50 KB of data): reported in microseconds"
+    return out
 
 
 # ------------------------------------------------------------------ GPU leg
@@ -682,6 +777,11 @@ def run_ours(args, w):
                              "frac": tf(8 * D2 * pairs_w, nb) / peak}}
         del wl
 
+    configs = None
+    if not args.no_configs:
+        configs = {name: config_leg(A, torch, name, args, rank, world, dev, stream, peaks)
+                   for name in ("char_gpt", "small_head", "gpt2_xl", "tiny_f32")}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.seed)
@@ -698,7 +798,7 @@ def run_ours(args, w):
                             "datasheet_2250": value / world / 2250.0},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "strided_io": strided,
             "noncausal": noncausal, "dropout": dropout, "decode": decode, "d128": d128,
-            "gpu_launches": launches, "clocks": clocks,
+            "configs": configs, "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -218,10 +218,10 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     return finish(e, li);
 }
 
-int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
-             const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D, float scale,
-             const Opts &op, const BwdStrides &str, void *workspace, size_t workspace_bytes,
-             cudaStream_t stream, LaunchInfo &li) {
+// Pointer, shape, head_dim, scale and alignment checks of the bf16 backward,
+// in the order its status codes are reported.
+int bwd_args(const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D, float scale) {
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 128);
     if (st != ATTN_OK) return st;
@@ -231,6 +231,15 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     for (const void *p : ptrs)
         if (!aligned(p, 16)) return ATTN_ERR_ALIGN;
     if (!aligned(lse, 4)) return ATTN_ERR_ALIGN;
+    return ATTN_OK;
+}
+
+int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D, float scale,
+             const Opts &op, const BwdStrides &str, void *workspace, size_t workspace_bytes,
+             cudaStream_t stream, LaunchInfo &li) {
+    int st = bwd_args(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale);
+    if (st != ATTN_OK) return st;
     const size_t need = attn_bwd_workspace_bytes(B, H, T, D);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
     int *err = nullptr;
@@ -433,6 +442,14 @@ ATTN_API int attn_selftest_wait_timeout(uint32_t polls, cudaStream_t stream) {
 }
 
 namespace attn {
+int bwd_arg_check(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D,
+                  float scale) {
+    return bwd_args(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale);
+}
+
+int device_check() { return device_setup(nullptr); }
+
 void *tensor_map_encoder() {
     static void *fn = nullptr;
     static std::once_flag once;

@@ -45,8 +45,10 @@ int scratch_on_current_device(void **out) {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
     if (g_scratch_ptr[dev] == nullptr) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();  // leave no stale error for a later launch check to find
             return ATTN_ERR_CUDA;
+        }
         g_scratch_ptr[dev] = p;
     }
     *out = g_scratch_ptr[dev];
@@ -59,15 +61,16 @@ int scratch_on_current_device(void **out) {
 ATTN_API int attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
                               const float *lse, const void *dO, void *dq, void *dk, void *dv,
                               int B, int H, int T, int D, float scale, cudaStream_t stream) {
-    const size_t need = attn_bwd_workspace_bytes(B, H, T, D);
-    if (need == 0) {
-        // Bad shape or head_dim: let attn_bwd report the precise status.
-        return attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, nullptr, 0, stream);
-    }
-    if (need > (size_t)ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
-    void *scratch = nullptr;
-    const int st = attn::scratch_on_current_device(&scratch);
+    // The statuses and their order are attn_bwd's: argument errors, then the
+    // scratch size (attn_bwd's workspace check), then the device; the scratch
+    // address is looked up only on a supported device.
+    int st = attn::bwd_arg_check(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale);
     if (st != ATTN_OK) return st;
+    const size_t need = attn_bwd_workspace_bytes(B, H, T, D);
+    if (need == 0 || need > (size_t)ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
+    if ((st = attn::device_check()) != ATTN_OK) return st;
+    void *scratch = nullptr;
+    if ((st = attn::scratch_on_current_device(&scratch)) != ATTN_OK) return st;
     return attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, scratch,
                     (size_t)ATTN_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -145,6 +145,17 @@ inline BwdWorkspace bwd_workspace_layout(int B, int H, int T, int D) {
 // most `polls` times, so the timeout path can be exercised without a fault.
 cudaError_t selftest_wait_timeout(uint32_t polls, int *err, cudaStream_t st);
 
+// The argument checks attn_bwd runs before it looks at its workspace
+// (pointers, shape, head_dim, scale, alignment, in that order): ATTN_OK or the
+// status attn_bwd returns for these arguments.
+int bwd_arg_check(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D,
+                  float scale);
+// The device check attn_bwd runs after its workspace check: ATTN_OK on an
+// sm_100 device, ATTN_ERR_DEVICE on another, ATTN_ERR_CUDA when the runtime
+// cannot say.
+int device_check();
+
 // Driver entry point for cuTensorMapEncodeTiled, resolved once at run time
 // through the runtime (so the library does not link libcuda directly).
 void *tensor_map_encoder();

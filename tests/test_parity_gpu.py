@@ -136,3 +136,34 @@ def test_bf16_guard_bands_and_determinism():
             torch.testing.assert_close(a.float(), b.float(), rtol=0, atol=1e-3)
         else:
             assert torch.equal(a, b), f"{name} differs between identical runs"
+
+
+def test_bf16_o_error_by_magnitude_band():
+    """bf16 O against the oracle, broken out by |O| band (< 1, 1-4, >= 4), on
+    the GPT-2 XL workload, whose outlier keys (1% of K rows x8) concentrate a
+    row's attention on single value rows so that |O| reaches the range where
+    bf16's own half-ulp (2^-7 on [2, 4), 2^-6 on [4, 8)) takes most of the
+    2e-2 budget.  Each band must meet the bound; and beyond the unavoidable
+    rounding of the output itself, the error of the computation (GPU O against
+    the oracle's O rounded to bf16) must stay within 1e-2 in every band."""
+    w = WORKLOADS["gpt2_xl"]
+    inp = make_inputs(w, seed=0)
+    got = parity.run_gpu(inp)
+    heads = parity.sample_heads(w.B, w.H, 10, seed=5)
+    ref = parity.run_oracle(inp, heads=heads)
+    o = parity.select_heads(got, heads, w.B, w.H)["o"]
+    r = ref["o"]
+    r_bf16 = torch.from_numpy(r).to(torch.bfloat16).double().numpy()
+    report = []
+    for lo, hi in ((0.0, 1.0), (1.0, 4.0), (4.0, np.inf)):
+        m = (np.abs(r) >= lo) & (np.abs(r) < hi)
+        if not m.any():
+            report.append(f"[{lo},{hi}): empty")
+            continue
+        err = float(np.max(np.abs(o - r)[m]))
+        comp = float(np.max(np.abs(o - r_bf16)[m]))
+        report.append(f"[{lo},{hi}): n={int(m.sum())} max-abs {err:.3e} (headroom {2e-2 - err:.3e}), "
+                      f"beyond output rounding {comp:.3e}")
+        assert err <= parity.BF16_TOL["max_abs"], report[-1]
+        assert comp <= 1e-2, report[-1]
+    print("O error by |O| band (gpt2_xl):", "; ".join(report))
