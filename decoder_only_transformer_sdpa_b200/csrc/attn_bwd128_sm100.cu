@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit_e(&sm.acc_done);
         }
         mma_commit_e(&sm.drain);
-        mbar_wait_warp(&sm.drain, 0, err, abort);
+        mbar_wait_drain(&sm.drain, 0);
     } else if (warp < 10) {
         // ------------------------------------------------ softmax gradient
         const int quad = warp & 3;

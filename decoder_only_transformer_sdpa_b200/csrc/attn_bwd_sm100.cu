@@ -110,7 +110,9 @@ struct BwdSmem {
 // One thread per (tile-padded row, 16-byte chunk of the row): D/8 threads per
 // row read O and dO with coalesced 16-byte loads, Delta_i is reduced across
 // them with shuffles, and the same threads zero their part of the dQ
-// accumulator row.
+// accumulator row.  Grid: x over blocks of 256 / (D/8) tokens, y over heads
+// (striding when there are more heads than grid rows), so a thread finds its
+// token and head without integer division.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o,
                                                        const __nv_bfloat16 *__restrict__ dO,
@@ -118,67 +120,78 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
                                                        float *__restrict__ lse2,
                                                        float *__restrict__ delta,
                                                        float *__restrict__ dq_acc, int T, int Tpad,
-                                                       long long prows, int H, TStrides so,
-                                                       TStrides sdo) {
-    constexpr int kTpr = D / 8;  // threads per row (a power of two dividing 32)
+                                                       int BH, int H, TStrides so, TStrides sdo) {
+    constexpr int kTpr = D / 8;           // threads per row (a power of two dividing 32)
+    constexpr int kRows = 256 / kTpr;     // rows per block
     grid_dep_wait();
     grid_dep_launch();
-    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long prow = gid / kTpr;
-    const int c = (int)(gid - prow * kTpr);
-    const bool valid = prow < prows;
-    const long long bh = valid ? prow / Tpad : 0;
-    const int t = valid ? (int)(prow - bh * Tpad) : 0;
-    const bool live = valid && t < T;
-    const size_t row = (size_t)bh * T + t;
-    float acc = 0.f;
-    if (live) {
-        const long long hb = bh / H, hh = bh % H;
-        const uint4 a = reinterpret_cast<const uint4 *>(o + hb * so.b + hh * so.h + (long long)t * so.t)[c];
-        const uint4 g = reinterpret_cast<const uint4 *>(dO + hb * sdo.b + hh * sdo.h + (long long)t * sdo.t)[c];
-        const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
-        const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&g);
+    const int c = (int)threadIdx.x % kTpr;
+    const int t = (int)blockIdx.x * kRows + (int)threadIdx.x / kTpr;
+    if (t >= Tpad) return;  // whole rows leave together: the shuffle groups stay complete
+    const bool live = t < T;
+    for (int bh = (int)blockIdx.y; bh < BH; bh += (int)gridDim.y) {
+        const size_t row = (size_t)bh * T + t;
+        float acc = 0.f;
+        if (live) {
+            const long long hb = bh / H, hh = bh % H;
+            const uint4 a = reinterpret_cast<const uint4 *>(o + hb * so.b + hh * so.h + (long long)t * so.t)[c];
+            const uint4 g = reinterpret_cast<const uint4 *>(dO + hb * sdo.b + hh * sdo.h + (long long)t * sdo.t)[c];
+            const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
+            const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&g);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const float2 fa = __bfloat1622float2(a2[x]), fg = __bfloat1622float2(g2[x]);
-            acc = fmaf(fa.x, fg.x, acc);
-            acc = fmaf(fa.y, fg.y, acc);
+            for (int x = 0; x < 4; ++x) {
+                const float2 fa = __bfloat1622float2(a2[x]), fg = __bfloat1622float2(g2[x]);
+                acc = fmaf(fa.x, fg.x, acc);
+                acc = fmaf(fa.y, fg.y, acc);
+            }
+            float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D + 8 * c);
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D + 8 * c);
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
 #pragma unroll
-    for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (valid && c == 0) {
-        delta[prow] = live ? acc : 0.f;
-        lse2[prow] = live ? lse[row] * kLog2e : INFINITY;
+        for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (c == 0) {
+            const size_t prow = (size_t)bh * Tpad + t;
+            delta[prow] = live ? acc : 0.f;
+            lse2[prow] = live ? lse[row] * kLog2e : INFINITY;
+        }
     }
 }
 
 // ------------------------------------------------------------------ post
 
-// dQ = scale * accumulator, 8 elements per thread (two 16-byte loads, one
-// 16-byte store into the strided dQ view).
-__global__ void bwd_post_kernel(const float4 *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
-                                long long n8, float scale, int T, int H, int D, TStrides sdq) {
-    const int cpr = D / 8;  // 8-element chunks per row
+// dQ = scale * accumulator: 8 elements per thread (two 16-byte loads, one
+// 16-byte store into the strided dQ view).  Grid as the prep kernel's: x over
+// blocks of 256 / (D/8) tokens, y over heads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float4 *__restrict__ acc,
+                                                       __nv_bfloat16 *__restrict__ dq, float scale,
+                                                       int T, int BH, int H, TStrides sdq) {
+    constexpr int kCpr = D / 8;           // 8-element chunks per row
+    constexpr int kRows = 256 / kCpr;
     grid_dep_wait();
     grid_dep_launch();
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
-         i += (long long)gridDim.x * blockDim.x) {
-        const long long row = i / cpr;
-        const int c = (int)(i - row * cpr);
-        const long long bh = row / T;
-        const long long t = row - bh * T;
+    const int c = (int)threadIdx.x % kCpr;
+    const int t = (int)blockIdx.x * kRows + (int)threadIdx.x / kCpr;
+    if (t >= T) return;
+    for (int bh = (int)blockIdx.y; bh < BH; bh += (int)gridDim.y) {
+        const size_t i = ((size_t)bh * T + t) * kCpr + c;
         const float4 a = acc[2 * i], b = acc[2 * i + 1];
         uint4 r;
         r.x = pack_bf16x2(a.x * scale, a.y * scale);
         r.y = pack_bf16x2(a.z * scale, a.w * scale);
         r.z = pack_bf16x2(b.x * scale, b.y * scale);
         r.w = pack_bf16x2(b.z * scale, b.w * scale);
-        *reinterpret_cast<uint4 *>(dq + (bh / H) * sdq.b + (bh % H) * sdq.h + t * sdq.t + 8 * c) = r;
+        const long long hb = bh / H, hh = bh % H;
+        *reinterpret_cast<uint4 *>(dq + hb * sdq.b + hh * sdq.h + (long long)t * sdq.t + 8 * c) = r;
     }
+}
+
+// The (token blocks, heads) grid of the prep and post kernels.
+template <int D>
+dim3 rows_grid(int rows, int BH) {
+    constexpr int kRows = 256 / (D / 8);
+    return dim3((unsigned)((rows + kRows - 1) / kRows), (unsigned)(BH < 65535 ? BH : 65535));
 }
 
 // ------------------------------------------------------------------ main
@@ -390,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         mma_commit_e(&sm.drain);
-        mbar_wait_warp(&sm.drain, 0, err, abort);
+        mbar_wait_drain(&sm.drain, 0);
     }
     } else if (warp < kDrainWarp0) {
     // ==================================================== softmax-gradient warpgroups
@@ -626,8 +639,8 @@ template <int D, bool Causal, bool Drop>
 cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                        const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                        __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
-                       float *lse2, float *delta, Shape s, const BwdStrides &str, int *err,
-                       cudaStream_t st, LaunchInfo &li) {
+                       float *lse2, float *delta, Shape s, const BwdStrides &str,
+                       int *err, cudaStream_t st, LaunchInfo &li) {
     const int BH = s.B * s.H;
     const int nt = (s.T + kBT - 1) / kBT;
     const int Tpad = nt * kBT;
@@ -647,11 +660,8 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if ((e = make_map_bf16(&mdo, dO, s, str.dO)) != cudaSuccess) return e;
     if ((e = make_map(&mdq, dq_acc, BH, s.T, D, true, 32)) != cudaSuccess) return e;
 
-    const long long prows = (long long)BH * Tpad;
-    const long long prep_threads = prows * (D / 8);
-    if ((e = launch_pdl(bwd_prep_kernel<D>, dim3((unsigned)((prep_threads + 255) / 256)), dim3(256), 0,
-                        st, o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows, s.H, str.o, str.dO)) !=
-        cudaSuccess)
+    if ((e = launch_pdl(bwd_prep_kernel<D>, rows_grid<D>(Tpad, BH), dim3(256), 0, st, o, dO, lse, lse2,
+                        delta, dq_acc, s.T, Tpad, BH, s.H, str.o, str.dO)) != cudaSuccess)
         return e;
     li.kernels += 1;
 
@@ -678,12 +688,9 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     li.kernels += 1;
     if ((e = mark_main_end(li, st)) != cudaSuccess) return e;
 
-    const long long n8 = (long long)BH * s.T * D / 8;
-    const long long want = (n8 + 255) / 256;
-    const int post_blocks = (int)(want < 148 * 16 ? want : 148 * 16);
-    if ((e = launch_pdl(bwd_post_kernel, dim3(post_blocks), dim3(256), 0, st,
-                        reinterpret_cast<const float4 *>(dq_acc), dq, n8, s.scale, s.T, s.H, D,
-                        str.dq)) != cudaSuccess)
+    if ((e = launch_pdl(bwd_post_kernel<D>, rows_grid<D>(s.T, BH), dim3(256), 0, st,
+                        reinterpret_cast<const float4 *>(dq_acc), dq, s.scale, s.T, BH, s.H, str.dq)) !=
+        cudaSuccess)
         return e;
     li.kernels += 1;
     return cudaSuccess;
@@ -694,28 +701,22 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
 cudaError_t launch_bwd128(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                           const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                           __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
-                          float *lse2, float *delta, Shape s, const BwdStrides &str, int *err,
-                          cudaStream_t st, LaunchInfo &li) {
+                          float *lse2, float *delta, Shape s, const BwdStrides &str,
+                          int *err, cudaStream_t st, LaunchInfo &li) {
     constexpr int D = 128;
     const int BH = s.B * s.H;
     const int Tpad = (s.T + kBT - 1) / kBT * kBT;
-    const long long prows = (long long)BH * Tpad;
-    const long long prep_threads = prows * (D / 8);
     cudaError_t e;
-    if ((e = launch_pdl(bwd_prep_kernel<D>, dim3((unsigned)((prep_threads + 255) / 256)), dim3(256), 0,
-                        st, o, dO, lse, lse2, delta, dq_acc, s.T, Tpad, prows, s.H, str.o, str.dO)) !=
-        cudaSuccess)
+    if ((e = launch_pdl(bwd_prep_kernel<D>, rows_grid<D>(Tpad, BH), dim3(256), 0, st, o, dO, lse, lse2,
+                        delta, dq_acc, s.T, Tpad, BH, s.H, str.o, str.dO)) != cudaSuccess)
         return e;
     li.kernels += 1;
     if ((e = sm100_bwd128_main(q, k, v, dO, dk, dv, dq_acc, lse2, delta, s, str, err, st, li)) !=
         cudaSuccess)
         return e;
-    const long long n8 = (long long)BH * s.T * D / 8;
-    const long long want = (n8 + 255) / 256;
-    const int post_blocks = (int)(want < 148 * 16 ? want : 148 * 16);
-    if ((e = launch_pdl(bwd_post_kernel, dim3(post_blocks), dim3(256), 0, st,
-                        reinterpret_cast<const float4 *>(dq_acc), dq, n8, s.scale, s.T, s.H, D,
-                        str.dq)) != cudaSuccess)
+    if ((e = launch_pdl(bwd_post_kernel<D>, rows_grid<D>(s.T, BH), dim3(256), 0, st,
+                        reinterpret_cast<const float4 *>(dq_acc), dq, s.scale, s.T, BH, s.H, str.dq)) !=
+        cudaSuccess)
         return e;
     li.kernels += 1;
     return cudaSuccess;
@@ -726,12 +727,12 @@ cudaError_t launch_bwd128(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const 
 cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const __nv_bfloat16 *o, const float *lse, const __nv_bfloat16 *dO,
                       __nv_bfloat16 *dq, __nv_bfloat16 *dk, __nv_bfloat16 *dv, float *dq_acc,
-                      float *lse2, float *delta, Shape s, const BwdStrides &str, int *err,
-                      cudaStream_t st, LaunchInfo &li) {
-#define ATTN_BWD_CASE(DD, C, R)                                                          \
-    if (s.D == DD && (s.causal != 0) == C && s.dropout == R)                             \
-        return launch_bwd<DD, C, R>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, \
-                                    str, err, st, li);
+                      float *lse2, float *delta, Shape s, const BwdStrides &str,
+                      int *err, cudaStream_t st, LaunchInfo &li) {
+#define ATTN_BWD_CASE(DD, C, R)                                                                    \
+    if (s.D == DD && (s.causal != 0) == C && s.dropout == R)                                       \
+        return launch_bwd<DD, C, R>(q, k, v, o, lse, dO, dq, dk, dv, dq_acc, lse2, delta, s, str, err, \
+                                    st, li);
     ATTN_BWD_CASE(64, true, false)
     ATTN_BWD_CASE(64, false, false)
     ATTN_BWD_CASE(64, true, true)

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
         }
         // All MMAs of both streams are complete once `drain` fires.
         mma_commit_e(&sm.drain);
-        mbar_wait_warp(&sm.drain, 0, err, abort);
+        mbar_wait_drain(&sm.drain, 0);
     }
     } else {
     // ==================================================== softmax warpgroup

@@ -67,6 +67,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     return false;
 }
 
+// Waits for async work this thread (or warp) itself issued, e.g. the last
+// TMA loads or MMAs before the CTA exits: polls at most kWaitLimit times and
+// does not give up early when another thread has aborted, since the work in
+// flight must land before its shared memory or TMEM is released.  Returns
+// whether the phase completed.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0,

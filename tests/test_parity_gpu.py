@@ -142,10 +142,12 @@ def test_bf16_o_error_by_magnitude_band():
     """bf16 O against the oracle, broken out by |O| band (< 1, 1-4, >= 4), on
     the GPT-2 XL workload, whose outlier keys (1% of K rows x8) concentrate a
     row's attention on single value rows so that |O| reaches the range where
-    bf16's own half-ulp (2^-7 on [2, 4), 2^-6 on [4, 8)) takes most of the
-    2e-2 budget.  Each band must meet the bound; and beyond the unavoidable
-    rounding of the output itself, the error of the computation (GPU O against
-    the oracle's O rounded to bf16) must stay within 1e-2 in every band."""
+    bf16's own half-ulp (2^-7 on [2, 4), 2^-6 on [4, 8)) takes much of the 2e-2
+    budget.  Every band must meet the bound, and every element must be within
+    the error the bf16 path can have: half an ulp of its exact value (the final
+    rounding) plus the rounding of the weights P to bf16 before P V, which moves
+    O by at most 2^-9 max|v| (2^-8 max|v| is allowed, which also covers the
+    float32 normalisation).  The band table is printed as the headroom report."""
     w = WORKLOADS["gpt2_xl"]
     inp = make_inputs(w, seed=0)
     got = parity.run_gpu(inp)
@@ -153,17 +155,23 @@ def test_bf16_o_error_by_magnitude_band():
     ref = parity.run_oracle(inp, heads=heads)
     o = parity.select_heads(got, heads, w.B, w.H)["o"]
     r = ref["o"]
-    r_bf16 = torch.from_numpy(r).to(torch.bfloat16).double().numpy()
-    report = []
+    v = inp["v"].to(torch.float64).numpy().reshape(w.B * w.H, w.T, w.D)[heads][None]
+    vmax = np.max(np.abs(v), axis=(2, 3), keepdims=True)          # per head
+    a = np.abs(r)
+    half_ulp = np.where(a > 0, np.exp2(np.floor(np.log2(np.maximum(a, 1e-30))) - 8), 0.0)
+    bound = half_ulp + 2.0 ** -8 * vmax
+    err = np.abs(o - r)
+    report, failures = [], []
     for lo, hi in ((0.0, 1.0), (1.0, 4.0), (4.0, np.inf)):
-        m = (np.abs(r) >= lo) & (np.abs(r) < hi)
+        m = (a >= lo) & (a < hi)
         if not m.any():
-            report.append(f"[{lo},{hi}): empty")
+            report.append(f"|O| in [{lo},{hi}): empty")
             continue
-        err = float(np.max(np.abs(o - r)[m]))
-        comp = float(np.max(np.abs(o - r_bf16)[m]))
-        report.append(f"[{lo},{hi}): n={int(m.sum())} max-abs {err:.3e} (headroom {2e-2 - err:.3e}), "
-                      f"beyond output rounding {comp:.3e}")
-        assert err <= parity.BF16_TOL["max_abs"], report[-1]
-        assert comp <= 1e-2, report[-1]
-    print("O error by |O| band (gpt2_xl):", "; ".join(report))
+        ma = float(np.max(err[m]))
+        slack = float(np.min((bound - err)[m]))
+        report.append(f"|O| in [{lo},{hi}): n={int(m.sum())} max-abs {ma:.3e} (headroom to 2e-2: "
+                      f"{2e-2 - ma:.3e}; smallest slack to the bf16 bound: {slack:.3e})")
+        if ma > parity.BF16_TOL["max_abs"] or slack < 0:
+            failures.append(report[-1])
+    print("O error by |O| band (gpt2_xl):\n  " + "\n  ".join(report))
+    assert not failures, failures
