@@ -371,6 +371,39 @@ def config_leg(A, torch, name, args, rank, world, dev, stream, peaks):
         out["bwd_main"]["frac"] = out["bwd_main"]["tflops"] / peak
     else:
         out["bound"] = "launch latency (50 KB of data): reported in microseconds"
+    # The same iterations replayed from a CUDA graph (one pass over every input
+    # set per replay): the device time without the host's per-call cost, which
+    # is comparable to the kernels' time at these small shapes.
+    try:
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(stream)
+        with torch.cuda.stream(gs):
+            for i in range(n_sets):
+                one(i)
+        stream.wait_stream(gs)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n_sets):
+                one(i)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        n_rep = max(3, n_it // n_sets)
+        s0.record(stream)
+        for _ in range(n_rep):
+            g.replay()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        if A.attn_device_error() != 0:
+            raise RuntimeError(f"a bounded in-kernel wait timed out in the {name} graph leg")
+        gms = reduce_max(s0.elapsed_time(s1), world, dev) / (n_rep * n_sets)
+        out["graph"] = {"us_per_fwd_bwd": 1e3 * gms, "tflops": world * tf(w.flops(), gms),
+                        "gbs": world * hb / (gms * 1e-3) / 1e9, "replays": n_rep}
+        if not f32:
+            out["graph"]["frac_of_bf16_peak"] = out["graph"]["tflops"] / world / peak
+            out["graph"]["hbm_frac"] = out["graph"]["gbs"] / world / hbm
+        del g
+    except RuntimeError as exc:  # capture unsupported here: report, do not fail the bench
+        out["graph"] = {"unavailable": str(exc).splitlines()[0][:200]}
     return out
 
 
