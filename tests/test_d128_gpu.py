@@ -89,3 +89,15 @@ def test_d128_packed_layout():
     cpu = lambda t: t.detach().to("cpu", torch.float64).contiguous().numpy()
     got = dict(o=cpu(o), lse=cpu(lse), dq=cpu(dq), dk=cpu(dk), dv=cpu(dv))
     parity.assert_close(got, parity.run_oracle(inp), torch.bfloat16, "D=128 packed")
+
+
+@pytest.mark.parametrize("causal,dropout_p", [(True, 0.0), (False, 0.0), (True, 0.1)])
+def test_d128_many_items_per_cta(causal, dropout_p):
+    """768 (key tile, head) items, about five waves of CTAs on 148 SMs, with
+    every head checked."""
+    B, H, T = 16, 24, 130
+    inp = random_qkv(4242 + int(causal), B, H, T, D, dtype=torch.bfloat16, do_std=1e-2)
+    kw = dict(dropout_p=dropout_p, seed=5, offset=0) if dropout_p else {}
+    got = parity.run_gpu(inp, causal=causal, **kw)
+    parity.assert_close(got, parity.run_oracle(inp, causal=causal, **kw), torch.bfloat16,
+                        f"D=128 B={B} H={H} T={T} causal={causal} p={dropout_p}")
