@@ -25,14 +25,20 @@
 //   warp 1      tcgen05 issuer of S = Q K_j^T into TMEM; owns the TMEM
 //               allocation.  S of the next tile is issued as soon as the
 //               softmax has read the current one.
-//   warp 2      idle (it completes the first warpgroup)
+//   warp 2      at D = 128 without dropout, the O store stream: stores each
+//               item's O / l, staged by the softmax warps in the item's Q
+//               buffer, with TMA and hands the buffer back to the producer
+//               once the store has read it; otherwise idle, and the first
+//               softmax thread does this
 //   warp 3      tcgen05 issuer of O += P_j V_j with P_j read from TMEM
 //   warps 4..7  softmax: one query row per thread (TMEM lane), online max and
 //               sum in registers, P_j written to TMEM as bf16, lazy rescale of
-//               the O accumulator, final O / l and lse per item (O / l is
-//               staged in the item's Q buffer, no longer read by then, and
-//               written by one TMA store; the buffer then goes back to the
-//               producer).
+//               the O accumulator, final O / l and lse per item.  At D = 128
+//               without dropout an item's epilogue runs inside the next
+//               item's first tile, after its exponentials, so the item's last
+//               PV completes behind them instead of stalling the warps at the
+//               item boundary.  O / l is staged in the item's Q buffer, no
+//               longer read by then.
 // At D <= 64 (two CTAs per SM, 128 registers per thread at launch) the first
 // warpgroup hands registers to the softmax warpgroup with setmaxnreg: 56 and
 // 200 per thread, 128 x 56 + 128 x 200 = the block's 256 x 128; the launch
@@ -79,7 +85,7 @@ struct FwdSmem {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
     uint64_t s_full, s_free, p_full;
-    uint64_t o_done, o_final, o_free, drain;
+    uint64_t o_done, o_final, o_free, o_staged, drain;
     uint32_t tmem_slot;
     int abort;
 };
@@ -116,6 +122,13 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
     constexpr uint32_t kAtom = 8 * kRowBytes;             // 8-row swizzle atom
     constexpr uint32_t kSlabBytes = 128 * kRowBytes;      // one 128-row slab
     constexpr uint32_t kTmemCols = tmem_cols<D>();
+    // With one CTA per SM (D = 128) nothing else fills the item boundary, so an
+    // item's epilogue moves into the next item's first tile and warp 2 issues
+    // its O store; with two CTAs per SM the other CTA's softmax fills the
+    // boundary, and the epilogue stays at the end of the item (measured: the
+    // deferred form is slower there).  Not with dropout, whose generator state
+    // leaves no registers for the deferred epilogue's.
+    constexpr bool kDeferEpilogue = D > 64 && !Drop;
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                          ~uintptr_t(1023));
@@ -128,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.q_full[b], 1);
-            mbar_init(&sm.q_empty[b], 1);  // the first softmax thread, after the O store read it
+            mbar_init(&sm.q_empty[b], 1);  // the O store's issuer, once the store has read the buffer
         }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.k_full[s], 1);
@@ -142,6 +155,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.o_final, 1);
         mbar_init(&sm.o_free, kBM);
+        mbar_init(&sm.o_staged, kBM);
         mbar_init(&sm.drain, 2);  // both tcgen05 streams
         sm.abort = 0;
         fence_mbar_init();
@@ -216,6 +230,29 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
         }
         for (int n = (nq > 2 ? nq - 2 : 0); n < nq; ++n)
             for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.q_full[n & 1], (uint32_t)(n >> 1) & 1u); ++i) {}
+    } else if (kDeferEpilogue && warp == 2) {
+        // ------------------------------------------------ O store stream: once
+        // the softmax warps have staged an item's O / l in its Q buffer, one
+        // lane stores it with the tensor map and, when the store has read the
+        // buffer, hands it back to the producer.
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            const int w = item_of(cta, n, G, W);
+            if (w < 0) break;
+            const int qt = ntiles - 1 - w / BH, bh = w % BH;
+            if (!(ok = mbar_wait_warp(&sm.o_staged, (uint32_t)n & 1u, err, abort))) break;
+            if (lane == 0) {
+                const uint8_t *qbuf = reinterpret_cast<const uint8_t *>(sm.q[n & 1]);
+#pragma unroll
+                for (int sl = 0; sl < kSlabs; ++sl)
+                    tma_store_4d(&to, qbuf + sl * kSlabBytes, sl * kSlabCols, qt * kBM, bh % H, bh / H);
+                bulk_commit();
+                bulk_wait_read_all();
+                mbar_arrive(&sm.q_empty[n & 1]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) bulk_wait_all();  // the O stores have completed
     } else if (warp == 1 || warp == 3) {
         // ------------------------------------------------ tcgen05 issuers (whole
         // warp, one elected lane issues).  Two independent streams share the
@@ -294,7 +331,69 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
         const int row = quad * 32 + lane;          // row within the query tile
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        // Epilogue of item pn (row max pm in log2 units, row sum pl): once its
+        // last PV has completed, O / l goes as bf16 into the item's Q buffer
+        // (every S MMA of the item has completed by then) in the swizzled
+        // layout of a TMA tile, for warp 2 to store; O's TMEM is released as
+        // soon as it is in registers; the row's lse goes to global memory.
+        auto epilogue = [&](int pn, float pm, float pl, int pqt, int pbh) -> bool {
+            if (!mbar_wait_warp(&sm.o_final, (uint32_t)pn & 1u, err, abort)) return false;
+            tc_fence_after();
+            const float inv = (Drop ? dp.keep_scale : 1.f) / pl;
+            uint8_t *qbuf = reinterpret_cast<uint8_t *>(sm.q[pn & 1]);
+            const uint32_t swz = kRowBytes == 128 ? (uint32_t)(row & 7) : (uint32_t)((row >> 1) & 3);
+            constexpr int kPerRound = D > 64 ? 2 : D / 32;  // 32-column TMEM loads in flight at once
+#pragma unroll
+            for (int h0 = 0; h0 < D / 32; h0 += kPerRound) {
+                uint32_t r[kPerRound][32];
+#pragma unroll
+                for (int h = 0; h < kPerRound; ++h) tmem_ld32(tO + lane_off + 32 * (h0 + h), r[h]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < kPerRound; ++h) reg_fence32(r[h]);
+                if (h0 + kPerRound == D / 32) {
+                    tc_fence_before();
+                    mbar_arrive(&sm.o_free);
+                }
+#pragma unroll
+                for (int h = 0; h < kPerRound; ++h) {
+                    const int col0 = 32 * (h0 + h);  // first column of this load
+                    const int sl = col0 / kSlabCols;
+                    const uint32_t base = smem_u32(qbuf + sl * kSlabBytes) + (uint32_t)row * kRowBytes;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {  // 16-byte chunks of 8 columns
+                        const uint32_t chunk = (uint32_t)((col0 % kSlabCols) / 8 + c);
+                        const uint32_t *v = &r[h][8 * c];
+                        st_shared_v4(base + ((chunk ^ swz) << 4),
+                                     pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
+                                     pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
+                                     pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
+                                     pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            if constexpr (kDeferEpilogue) {
+                mbar_arrive(&sm.o_staged);
+            } else {
+                named_bar_sync(1, kBM);
+                if (warp == kSoftmaxWarp0 && lane == 0) {
+#pragma unroll
+                    for (int sl = 0; sl < kSlabs; ++sl)
+                        tma_store_4d(&to, qbuf + sl * kSlabBytes, sl * kSlabCols, pqt * kBM, pbh % H, pbh / H);
+                    bulk_commit();
+                    // Once the store has read the tile, the buffer takes item pn + 2's Q.
+                    bulk_wait_read_all();
+                    mbar_arrive(&sm.q_empty[pn & 1]);
+                }
+            }
+            const int t = pqt * kBM + row;
+            if (t < T) lse[(size_t)pbh * T + t] = (pm + log2f(pl)) * 0.69314718055994531f;
+            return true;
+        };
         int gt = 0;  // global key-tile counter (barrier phases)
+        int pn = -1, pqt = 0, pbh = 0;  // the item whose epilogue is still to run
+        float pm = 0.f, pl = 1.f;
         bool ok = true;
         for (int n = 0; ok; ++n) {
             const int w = item_of(cta, n, G, W);
@@ -418,7 +517,13 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                     }
                 }
                 l += la + lb;
-                if (!pv_done) {
+                if (kDeferEpilogue && j == 0 && pn >= 0) {
+                    // The previous item's epilogue, off the item boundary: its
+                    // last PV has had this tile's exponentials to complete (its
+                    // completion also frees the P region).
+                    if (!(ok = epilogue(pn, pm, pl, pqt, pbh))) break;
+                    pn = -1;
+                } else if (!pv_done) {
                     ok = mbar_wait_warp(&sm.o_done, (uint32_t)(gt - 1) & 1u, err, abort);
                     if (!ok) break;
                     tc_fence_after();
@@ -431,65 +536,22 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 mbar_arrive(&sm.p_full);
             }
             if (!ok) break;
-            // ---- epilogue of the item: O / l and lse; O's TMEM is released as
-            // soon as it is in registers so the next item's PV can start.
-            ok = mbar_wait_warp(&sm.o_final, (uint32_t)n & 1u, err, abort);
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t r[D / 32][32];
-#pragma unroll
-            for (int h = 0; h < D / 32; ++h) tmem_ld32(tO + lane_off + 32 * h, r[h]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < D / 32; ++h) reg_fence32(r[h]);
-            tc_fence_before();
-            mbar_arrive(&sm.o_free);
-            const int t = qt * kBM + row;
-            // O / l as bf16 into this item's Q buffer, in the swizzled layout
-            // of a TMA tile (every S MMA of the item has completed: the
-            // softmax consumed the last S before the last PV), then one TMA
-            // store per slab; rows past T are not written by the store.
-            {
-                const float inv = (Drop ? dp.keep_scale : 1.f) / l;
-                uint8_t *qbuf = reinterpret_cast<uint8_t *>(sm.q[n & 1]);
-                constexpr int kChunks = kRowBytes / 16;  // 16-byte chunks per slab row
-                const uint32_t swz = kRowBytes == 128 ? (uint32_t)(row & 7) : (uint32_t)((row >> 1) & 3);
-#pragma unroll
-                for (int sl = 0; sl < kSlabs; ++sl) {
-                    const uint32_t base = smem_u32(qbuf + sl * kSlabBytes) + (uint32_t)row * kRowBytes;
-#pragma unroll
-                    for (int c = 0; c < kChunks; ++c) {
-                        const int col = sl * kSlabCols + 8 * c;  // first of the chunk's 8 columns
-                        const uint32_t *v = &r[col / 32][col % 32];
-                        st_shared_v4(base + ((c ^ swz) << 4),
-                                     pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
-                                     pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
-                                     pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
-                                     pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
-                    }
-                }
-                fence_proxy_async_smem();
-                named_bar_sync(1, kBM);
-                if (warp == kSoftmaxWarp0 && lane == 0) {
-#pragma unroll
-                    for (int sl = 0; sl < kSlabs; ++sl)
-                        tma_store_4d(&to, qbuf + sl * kSlabBytes, sl * kSlabCols, qt * kBM, bh % H, bh / H);
-                    bulk_commit();
-                    // Once the store has read the tile, the buffer takes item n + 2's Q.
-                    bulk_wait_read_all();
-                    mbar_arrive(&sm.q_empty[n & 1]);
-                }
-            }
-            if (t < T) {
-                const size_t grow = (size_t)bh * T + t;
-                lse[grow] = (m_used + log2f(l)) * 0.69314718055994531f;
+            if constexpr (kDeferEpilogue) {
+                pn = n;
+                pqt = qt;
+                pbh = bh;
+                pm = m_used;
+                pl = l;
+            } else if (!(ok = epilogue(n, m_used, l, qt, bh))) {
+                break;
             }
         }
+        if (kDeferEpilogue && ok && pn >= 0) epilogue(pn, pm, pl, pqt, pbh);  // the CTA's last item
+        // The O stores issued by the first softmax thread have completed.
+        if (!kDeferEpilogue && warp == kSoftmaxWarp0 && lane == 0) bulk_wait_all();
     }
     }
 
-    // The O stores issued by the first softmax thread have completed.
-    if (warp == kSoftmaxWarp0 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
