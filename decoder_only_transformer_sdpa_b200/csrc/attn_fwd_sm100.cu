@@ -21,7 +21,7 @@
 // stream in and its first S MMA issues while the current item drains.
 // Eight warps in two warpgroups:
 //   warp 0      TMA producer: Q of each item into a 2-buffer ring, K_j / V_j
-//               tiles into a 2-stage ring
+//               tiles into a 2-stage ring (at D <= 64, K one tile ahead of V)
 //   warp 1      tcgen05 issuer of S = Q K_j^T into TMEM; owns the TMEM
 //               allocation.  S of the next tile is issued as soon as the
 //               softmax has read the current one.
@@ -182,54 +182,117 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
             prefetch_tensormap(&tv);
         }
         __syncwarp();
-        int gt = 0;  // key tiles loaded so far (the K/V ring position)
-        int nq = 0;  // Q tiles loaded so far
-        bool ok = true;
-        for (int n = 0; ok; ++n) {
-            const int w = item_of(cta, n, G, W);
-            if (w < 0) break;
-            const int qt = ntiles - 1 - w / BH, bh = w % BH;
-            const int hh = bh % H, bb = bh / H;
-            const int qb = n & 1;
-            if (!(ok = mbar_wait_warp(&sm.q_empty[qb], (uint32_t)((n >> 1) & 1) ^ 1u, err, abort))) break;
-            mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
-#pragma unroll
-            for (int sl = 0; sl < kSlabs; ++sl)
-                tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.q[qb]) + sl * kSlabBytes, &tq,
-                              &sm.q_full[qb], sl * kSlabCols, qt * kBM, hh, bb);
-            nq = n + 1;
-            const int nk = Causal ? qt + 1 : ntiles;  // key tiles this item reads
-            for (int j = 0; j < nk; ++j, ++gt) {
-                const int s = gt % kStages;
-                const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
-                if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
-                mbar_arrive_expect_tx_e(&sm.k_full[s], Smem::kTileBytes);
-#pragma unroll
-                for (int sl = 0; sl < kSlabs; ++sl)
-                    tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.k[s]) + sl * kSlabBytes, &tk,
-                                  &sm.k_full[s], sl * kSlabCols, j * kBN, hh, bb);
-                if (!(ok = mbar_wait_warp(&sm.v_empty[s], ph ^ 1u, err, abort))) {
-                    // K of this tile is in flight: let it land before leaving.
-                    for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
-                    break;
-                }
+        if constexpr (D <= 64) {
+            // K runs one tile ahead of V: K_{g+1} is issued before V_g, so that
+            // the wait for V_g's ring slot (freed by PV_{g-2}) never holds up
+            // the K load the next S needs.
+            int gt = 0;  // K tiles loaded so far (the K/V ring position)
+            int gv = 0;  // V tiles loaded so far
+            int nq = 0;  // Q tiles loaded so far
+            int pv_j = 0, pv_hh = 0, pv_bb = 0;  // the V tile gv (pending while gv < gt)
+            bool ok = true;
+            auto load_v = [&]() -> bool {
+                const int s = gv % kStages;
+                const uint32_t ph = (uint32_t)(gv / kStages) & 1u;
+                if (!mbar_wait_warp(&sm.v_empty[s], ph ^ 1u, err, abort)) return false;
                 mbar_arrive_expect_tx_e(&sm.v_full[s], Smem::kTileBytes);
 #pragma unroll
                 for (int sl = 0; sl < kSlabs; ++sl)
                     tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.v[s]) + sl * kSlabBytes, &tv,
-                                  &sm.v_full[s], sl * kSlabCols, j * kBN, hh, bb);
+                                  &sm.v_full[s], sl * kSlabCols, pv_j * kBN, pv_hh, pv_bb);
+                ++gv;
+                return true;
+            };
+            for (int n = 0; ok; ++n) {
+                const int w = item_of(cta, n, G, W);
+                if (w < 0) break;
+                const int qt = ntiles - 1 - w / BH, bh = w % BH;
+                const int hh = bh % H, bb = bh / H;
+                const int qb = n & 1;
+                if (!(ok = mbar_wait_warp(&sm.q_empty[qb], (uint32_t)((n >> 1) & 1) ^ 1u, err, abort))) break;
+                mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
+#pragma unroll
+                for (int sl = 0; sl < kSlabs; ++sl)
+                    tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.q[qb]) + sl * kSlabBytes, &tq,
+                                  &sm.q_full[qb], sl * kSlabCols, qt * kBM, hh, bb);
+                nq = n + 1;
+                const int nk = Causal ? qt + 1 : ntiles;  // key tiles this item reads
+                for (int j = 0; j < nk; ++j, ++gt) {
+                    const int s = gt % kStages;
+                    const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
+                    if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
+                    mbar_arrive_expect_tx_e(&sm.k_full[s], Smem::kTileBytes);
+#pragma unroll
+                    for (int sl = 0; sl < kSlabs; ++sl)
+                        tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.k[s]) + sl * kSlabBytes, &tk,
+                                      &sm.k_full[s], sl * kSlabCols, j * kBN, hh, bb);
+                    if (gv < gt && !(ok = load_v())) break;  // the previous tile's V
+                    pv_j = j;
+                    pv_hh = hh;
+                    pv_bb = bb;
+                }
             }
+            if (ok && gv < gt) ok = load_v();  // the last V (K ahead)
+            // Drain: the last loads this warp issued have landed before exit (on the
+            // normal path the consumers waited on all of them already).
+            for (int g = (gt > kStages ? gt - kStages : 0); g < gt; ++g)
+                mbar_wait_drain(&sm.k_full[g % kStages], (uint32_t)(g / kStages) & 1u);
+            for (int g = (gv > kStages ? gv - kStages : 0); g < gv; ++g)
+                mbar_wait_drain(&sm.v_full[g % kStages], (uint32_t)(g / kStages) & 1u);
+            for (int n = (nq > 2 ? nq - 2 : 0); n < nq; ++n)
+                mbar_wait_drain(&sm.q_full[n & 1], (uint32_t)(n >> 1) & 1u);
+        } else {
+            // At D = 128 (one CTA per SM) K_j and V_j go in order: measured
+            // faster there than K ahead.
+            int gt = 0;  // key tiles loaded so far (the K/V ring position)
+            int nq = 0;  // Q tiles loaded so far
+            bool ok = true;
+            for (int n = 0; ok; ++n) {
+                const int w = item_of(cta, n, G, W);
+                if (w < 0) break;
+                const int qt = ntiles - 1 - w / BH, bh = w % BH;
+                const int hh = bh % H, bb = bh / H;
+                const int qb = n & 1;
+                if (!(ok = mbar_wait_warp(&sm.q_empty[qb], (uint32_t)((n >> 1) & 1) ^ 1u, err, abort))) break;
+                mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
+#pragma unroll
+                for (int sl = 0; sl < kSlabs; ++sl)
+                    tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.q[qb]) + sl * kSlabBytes, &tq,
+                                  &sm.q_full[qb], sl * kSlabCols, qt * kBM, hh, bb);
+                nq = n + 1;
+                const int nk = Causal ? qt + 1 : ntiles;  // key tiles this item reads
+                for (int j = 0; j < nk; ++j, ++gt) {
+                    const int s = gt % kStages;
+                    const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
+                    if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
+                    mbar_arrive_expect_tx_e(&sm.k_full[s], Smem::kTileBytes);
+#pragma unroll
+                    for (int sl = 0; sl < kSlabs; ++sl)
+                        tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.k[s]) + sl * kSlabBytes, &tk,
+                                      &sm.k_full[s], sl * kSlabCols, j * kBN, hh, bb);
+                    if (!(ok = mbar_wait_warp(&sm.v_empty[s], ph ^ 1u, err, abort))) {
+                        // K of this tile is in flight: let it land before leaving.
+                        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
+                        break;
+                    }
+                    mbar_arrive_expect_tx_e(&sm.v_full[s], Smem::kTileBytes);
+#pragma unroll
+                    for (int sl = 0; sl < kSlabs; ++sl)
+                        tma_load_4d_e(reinterpret_cast<uint8_t *>(sm.v[s]) + sl * kSlabBytes, &tv,
+                                      &sm.v_full[s], sl * kSlabCols, j * kBN, hh, bb);
+                }
+            }
+            // Drain: the last loads this warp issued have landed before exit (on the
+            // normal path the consumers waited on all of them already).
+            for (int g = (gt > kStages ? gt - kStages : 0); g < gt; ++g) {
+                const int s = g % kStages;
+                const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
+                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.v_full[s], ph); ++i) {}
+            }
+            for (int n = (nq > 2 ? nq - 2 : 0); n < nq; ++n)
+                for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.q_full[n & 1], (uint32_t)(n >> 1) & 1u); ++i) {}
         }
-        // Drain: the last loads this warp issued have landed before exit (on the
-        // normal path the consumers waited on all of them already).
-        for (int g = (gt > kStages ? gt - kStages : 0); g < gt; ++g) {
-            const int s = g % kStages;
-            const uint32_t ph = (uint32_t)(g / kStages) & 1u;
-            for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.k_full[s], ph); ++i) {}
-            for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.v_full[s], ph); ++i) {}
-        }
-        for (int n = (nq > 2 ? nq - 2 : 0); n < nq; ++n)
-            for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sm.q_full[n & 1], (uint32_t)(n >> 1) & 1u); ++i) {}
     } else if (kDeferEpilogue && warp == 2) {
         // ------------------------------------------------ O store stream: once
         // the softmax warps have staged an item's O / l in its Q buffer, one
