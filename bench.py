@@ -292,6 +292,15 @@ def min_hbm_bytes(w) -> int:
     return 12 * n * es + 2 * w.B * w.H * w.T * 4
 
 
+# Per-kernel timing inside a timed loop samples the launches: CUDA events go
+# around one layer of each step (the middle one), or one call in PROF_EVERY,
+# because an event recorded between two launches stops the second from
+# starting early (programmatic dependent launch) and events around every launch
+# measurably slow the loop they time (~6 us per bracketed launch on the GPT-2
+# step).
+PROF_EVERY = 4
+
+
 def config_leg(A, torch, name, args, rank, world, dev, stream, peaks):
     """One forward + backward per iteration of the named workload, through the
     plain entry points, cycling over enough independent input sets that their
@@ -320,7 +329,10 @@ def config_leg(A, torch, name, args, rank, world, dev, stream, peaks):
     bwd = A.attn_bwd_f32 if f32 else A.attn_bwd
     n_it = max(4 * n_sets, min(args.steps, 200))
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    evs = [((mk(), mk()), (mk(), mk())) for _ in range(n_it)]
+    # Kernel events on every PROF_EVERY-th iteration only: an event recorded
+    # between two launches stops the second from starting early (programmatic
+    # dependent launch), so events on every call would slow the timed loop.
+    evs = [((mk(), mk()), (mk(), mk())) for _ in range((n_it + PROF_EVERY - 1) // PROF_EVERY)]
     for e in evs:
         for pair in e:
             for x in pair:
@@ -344,7 +356,7 @@ def config_leg(A, torch, name, args, rank, world, dev, stream, peaks):
     s0, s1 = mk(), mk()
     s0.record(stream)
     for i in range(n_it):
-        one(i, evs[i])
+        one(i, evs[i // PROF_EVERY] if i % PROF_EVERY == 0 else None)
     s1.record(stream)
     torch.cuda.synchronize(dev)
     if A.attn_device_error() != 0:
@@ -439,17 +451,19 @@ def run_ours(args, w):
                            device=dev)))
     stream = torch.cuda.current_stream(dev)
 
+    PL = L // 2  # the layer whose kernels are bracketed by events
+
     def step(ev_fwd=None, ev_bwd=None):
         launches = 0
         for l, b in enumerate(layers):
-            if ev_fwd is not None:
-                A.attn_profile_next_call(*ev_fwd[l])
+            if ev_fwd is not None and l == PL:
+                A.attn_profile_next_call(*ev_fwd)
             A.attn_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"])
             launches += A.attn_last_launch_count()
         for l in range(L - 1, -1, -1):
             b = layers[l]
-            if ev_bwd is not None:
-                A.attn_profile_next_call(*ev_bwd[l])
+            if ev_bwd is not None and l == PL:
+                A.attn_profile_next_call(*ev_bwd)
             A.attn_bwd(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"], b["dv"],
                        workspace=b["ws"])
             launches += A.attn_last_launch_count()
@@ -468,9 +482,9 @@ def run_ours(args, w):
 
     # ---- timed region: K steps, events on the launching stream
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    ev = [([(mk(), mk()) for _ in range(L)], [(mk(), mk()) for _ in range(L)]) for _ in range(args.steps)]
+    ev = [((mk(), mk()), (mk(), mk())) for _ in range(args.steps)]
     for e in ev:  # torch creates the CUDA event on first record; the library re-records it
-        for pair in e[0] + e[1]:
+        for pair in e:
             for x in pair:
                 x.record(stream)
     sampler = ClockSampler(gpu_uuid(torch, dev))
@@ -490,8 +504,8 @@ def run_ours(args, w):
     if A.attn_device_error() != 0:
         raise RuntimeError("a bounded in-kernel wait timed out in the timed region")
 
-    fwd_ms = [a.elapsed_time(b) for e in ev for a, b in e[0]]
-    bwd_ms = [a.elapsed_time(b) for e in ev for a, b in e[1]]
+    fwd_ms = [e[0][0].elapsed_time(e[0][1]) for e in ev]
+    bwd_ms = [e[1][0].elapsed_time(e[1][1]) for e in ev]
     ms_max = reduce_max(ms, world, dev)
     flops_step = w.flops() * L
     value = whole_job_tflops(flops_step, world, args.steps, ms_max)
@@ -629,22 +643,22 @@ def run_ours(args, w):
     # per layer and step; the generator's work is not credited)
     def variant_leg(causal, dropout_p):
         n_v = max(3, min(args.steps, 30))
-        evn = [([(mk(), mk()) for _ in range(L)], [(mk(), mk()) for _ in range(L)]) for _ in range(n_v + 1)]
+        evn = [((mk(), mk()), (mk(), mk())) for _ in range(n_v + 1)]
         for e in evn:
-            for pair in e[0] + e[1]:
+            for pair in e:
                 for x in pair:
                     x.record(stream)
 
         def v_step(it, ev_fwd=None, ev_bwd=None):
             for l, b in enumerate(layers):
-                if ev_fwd is not None:
-                    A.attn_profile_next_call(*ev_fwd[l])
+                if ev_fwd is not None and l == PL:
+                    A.attn_profile_next_call(*ev_fwd)
                 A.attn_fwd_ex(b["q"], b["k"], b["v"], b["o"], b["lse"], causal=causal,
                               dropout_p=dropout_p, seed=args.seed + 1, offset=it * L + l)
             for l in range(L - 1, -1, -1):
                 b = layers[l]
-                if ev_bwd is not None:
-                    A.attn_profile_next_call(*ev_bwd[l])
+                if ev_bwd is not None and l == PL:
+                    A.attn_profile_next_call(*ev_bwd)
                 A.attn_bwd_ex(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"],
                               b["dv"], causal=causal, dropout_p=dropout_p, seed=args.seed + 1,
                               offset=it * L + l, workspace=b["ws"])
@@ -660,8 +674,8 @@ def run_ours(args, w):
             raise RuntimeError("a bounded in-kernel wait timed out in a secondary leg")
         v_ms = reduce_max(s0.elapsed_time(s1), world, dev)
         pairs_v = w.causal_pairs() if causal else w.B * w.H * w.T * w.T
-        nf = statistics.mean(a.elapsed_time(b) for e in evn[:n_v] for a, b in e[0])
-        nb = statistics.mean(a.elapsed_time(b) for e in evn[:n_v] for a, b in e[1])
+        nf = statistics.mean(e[0][0].elapsed_time(e[0][1]) for e in evn[:n_v])
+        nb = statistics.mean(e[1][0].elapsed_time(e[1][1]) for e in evn[:n_v])
         tf = lambda fl, ms_: fl / (ms_ * 1e-3) / 1e12
         return {"value": whole_job_tflops(12 * w.D * pairs_v * L, world, n_v, v_ms),
                 "unit": "TFLOP/s", "ms_per_step": v_ms / n_v, "steps": n_v,
@@ -690,16 +704,15 @@ def run_ours(args, w):
             dl[-1]["o"] = torch.empty_like(dl[-1]["q"])
             dl[-1]["lse"] = torch.empty((w.B, w.H, tq), dtype=torch.float32, device=dev)
         n_d = max(10, min(args.steps, 100))
-        evd = [[(mk(), mk()) for _ in range(L)] for _ in range(n_d)]
-        for e in evd:
-            for pair in e:
-                for x in pair:
-                    x.record(stream)
+        evd = [(mk(), mk()) for _ in range(n_d)]
+        for pair in evd:
+            for x in pair:
+                x.record(stream)
 
         def d_step(evs=None):
             for l, b in enumerate(dl):
-                if evs is not None:
-                    A.attn_profile_next_call(*evs[l])
+                if evs is not None and l == PL:
+                    A.attn_profile_next_call(*evs)
                 A.attn_decode(b["q"], b["k"], b["v"], b["o"], b["lse"])
         for _ in range(3):
             d_step()
@@ -711,7 +724,7 @@ def run_ours(args, w):
         s1.record(stream)
         barrier()
         d_ms = reduce_max(s0.elapsed_time(s1), world, dev) / n_d
-        k_ms = statistics.mean(a.elapsed_time(b) for e in evd for a, b in e)
+        k_ms = statistics.mean(a.elapsed_time(b) for a, b in evd)
         bytes_launch = w.B * w.H * (2 * w.T * w.D * 2 + 2 * tq * w.D * 2 + tq * 4)
         hbm_peak = float(peaks.get("hbm_gbs"))
         # the same step replayed from a CUDA graph (no per-launch host cost)
@@ -769,21 +782,21 @@ def run_ours(args, w):
                                   device=dev)
             wl.append(b)
         n_w = max(3, min(args.steps, 30))
-        evw = [([(mk(), mk()) for _ in range(L)], [(mk(), mk()) for _ in range(L)]) for _ in range(n_w)]
+        evw = [((mk(), mk()), (mk(), mk())) for _ in range(n_w)]
         for e in evw:
-            for pair in e[0] + e[1]:
+            for pair in e:
                 for x in pair:
                     x.record(stream)
 
         def w_step(ev_fwd=None, ev_bwd=None):
             for l, b in enumerate(wl):
-                if ev_fwd is not None:
-                    A.attn_profile_next_call(*ev_fwd[l])
+                if ev_fwd is not None and l == PL:
+                    A.attn_profile_next_call(*ev_fwd)
                 A.attn_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"])
             for l in range(L - 1, -1, -1):
                 b = wl[l]
-                if ev_bwd is not None:
-                    A.attn_profile_next_call(*ev_bwd[l])
+                if ev_bwd is not None and l == PL:
+                    A.attn_profile_next_call(*ev_bwd)
                 A.attn_bwd(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"],
                            b["dv"], workspace=b["ws"])
         w_step()
@@ -798,8 +811,8 @@ def run_ours(args, w):
             raise RuntimeError("a bounded in-kernel wait timed out in the head_dim 128 leg")
         w_ms = reduce_max(s0.elapsed_time(s1), world, dev)
         pairs_w = w.B * H2 * w.T * (w.T + 1) // 2
-        nf = statistics.mean(a.elapsed_time(b) for e in evw for a, b in e[0])
-        nb = statistics.mean(a.elapsed_time(b) for e in evw for a, b in e[1])
+        nf = statistics.mean(e[0][0].elapsed_time(e[0][1]) for e in evw)
+        nb = statistics.mean(e[1][0].elapsed_time(e[1][1]) for e in evw)
         tf = lambda fl, ms_: fl / (ms_ * 1e-3) / 1e12
         d128 = {"workload": f"B={w.B} H={H2} T={w.T} D={D2} (n_embd {H2 * D2}), {L} layers, causal",
                 "value": whole_job_tflops(12 * D2 * pairs_w * L, world, n_w, w_ms), "unit": "TFLOP/s",
