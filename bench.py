@@ -643,6 +643,9 @@ def run_ours(args, w):
     # per layer and step; the generator's work is not credited)
     def variant_leg(causal, dropout_p):
         n_v = max(3, min(args.steps, 30))
+        # with dropout, each layer's forward keeps its drawn mask for its backward
+        masks = [torch.empty(A.attn_dropout_mask_bytes(w.B, w.H, w.T), dtype=torch.uint8, device=dev)
+                 if dropout_p > 0 else None for _ in range(L)]
         evn = [((mk(), mk()), (mk(), mk())) for _ in range(n_v + 1)]
         for e in evn:
             for pair in e:
@@ -654,14 +657,15 @@ def run_ours(args, w):
                 if ev_fwd is not None and l == PL:
                     A.attn_profile_next_call(*ev_fwd)
                 A.attn_fwd_ex(b["q"], b["k"], b["v"], b["o"], b["lse"], causal=causal,
-                              dropout_p=dropout_p, seed=args.seed + 1, offset=it * L + l)
+                              dropout_p=dropout_p, seed=args.seed + 1, offset=it * L + l,
+                              dropout_mask=masks[l])
             for l in range(L - 1, -1, -1):
                 b = layers[l]
                 if ev_bwd is not None and l == PL:
                     A.attn_profile_next_call(*ev_bwd)
                 A.attn_bwd_ex(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["dq"], b["dk"],
                               b["dv"], causal=causal, dropout_p=dropout_p, seed=args.seed + 1,
-                              offset=it * L + l, workspace=b["ws"])
+                              offset=it * L + l, workspace=b["ws"], dropout_mask=masks[l])
         v_step(0)
         barrier()
         s0, s1 = mk(), mk()
@@ -677,9 +681,11 @@ def run_ours(args, w):
         nf = statistics.mean(e[0][0].elapsed_time(e[0][1]) for e in evn[:n_v])
         nb = statistics.mean(e[1][0].elapsed_time(e[1][1]) for e in evn[:n_v])
         tf = lambda fl, ms_: fl / (ms_ * 1e-3) / 1e12
+        del masks
         return {"value": whole_job_tflops(12 * w.D * pairs_v * L, world, n_v, v_ms),
                 "unit": "TFLOP/s", "ms_per_step": v_ms / n_v, "steps": n_v,
                 "causal": causal, "dropout_p": dropout_p,
+                "kept_mask": dropout_p > 0,
                 "flops_per_layer": 12 * w.D * pairs_v,
                 "fwd_main": {"avg_launch_ms": nf, "tflops": tf(4 * w.D * pairs_v, nf),
                              "frac": tf(4 * w.D * pairs_v, nf) / peak},

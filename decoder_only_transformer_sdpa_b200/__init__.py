@@ -55,7 +55,8 @@ class attn_options(ctypes.Structure):
     attention dropout."""
     _fields_ = [("causal", ctypes.c_int32), ("dropout_p", ctypes.c_float),
                 ("dropout_seed", ctypes.c_uint64), ("dropout_offset", ctypes.c_uint32),
-                ("reserved", ctypes.c_uint32)]
+                ("reserved", ctypes.c_uint32), ("dropout_mask", ctypes.c_void_p),
+                ("dropout_mask_bytes", ctypes.c_size_t)]
 
 
 _op = ctypes.POINTER(attn_options)
@@ -78,6 +79,8 @@ _lib.attn_bwd_f32_workspace_bytes.argtypes = [_i, _i, _i, _i]
 _lib.attn_bwd_f32_workspace_bytes.restype = _sz
 _lib.attn_bwd_f32.argtypes = [_fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _f, _vp, _sz, _vp]
 _lib.attn_bwd_f32.restype = _i
+_lib.attn_dropout_mask_bytes.argtypes = [_i, _i, _i]
+_lib.attn_dropout_mask_bytes.restype = _sz
 _lib.attn_device_error.argtypes = [_vp]
 _lib.attn_device_error.restype = _i
 _lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _vp]
@@ -90,7 +93,7 @@ EXPORTED = ("attn_status_string", "attn_version", "attn_last_launch_count", "att
             "attn_bwd_f32", "attn_device_error", "attn_profile_next_call",
             "attn_selftest_wait_timeout", "attn_bwd_noalloc", "attn_fwd_strided",
             "attn_bwd_strided", "attn_fwd_ex", "attn_bwd_ex", "attn_fwd_f32_ex", "attn_bwd_f32_ex",
-            "attn_decode")
+            "attn_decode", "attn_dropout_mask_bytes")
 
 
 class AttnError(RuntimeError):
@@ -344,9 +347,18 @@ def attn_bwd_strided(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Opti
     return dq, dk, dv
 
 
-def _options(causal: bool, dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+def attn_dropout_mask_bytes(B: int, H: int, T: int) -> int:
+    return int(_lib.attn_dropout_mask_bytes(B, H, T))
+
+
+def _options(causal: bool, dropout_p: float = 0.0, seed: int = 0, offset: int = 0, mask=None):
+    if mask is not None:
+        torch = _torch()
+        if mask.dtype != torch.uint8 or not mask.is_cuda or not mask.is_contiguous():
+            raise ValueError("dropout_mask must be a contiguous CUDA uint8 tensor")
     return attn_options(1 if causal else 0, float(dropout_p), int(seed) & (2**64 - 1),
-                        int(offset) & 0xFFFFFFFF, 0)
+                        int(offset) & 0xFFFFFFFF, 0, None if mask is None else mask.data_ptr(),
+                        0 if mask is None else mask.numel())
 
 
 def _all_contiguous(*tensors) -> bool:
@@ -354,12 +366,15 @@ def _all_contiguous(*tensors) -> bool:
 
 
 def attn_fwd_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = True,
-                dropout_p: float = 0.0, seed: int = 0, offset: int = 0, stream=None):
+                dropout_p: float = 0.0, seed: int = 0, offset: int = 0, stream=None,
+                dropout_mask=None):
     """bf16 forward with options: ``causal=False`` drops the mask (every query
     sees all T keys); ``dropout_p`` > 0 drops attention weights with the
-    Philox keep mask of (seed, offset).  Contiguous or strided [B, H, T, D]
-    views; O defaults to the layout of q (contiguous, else a [B, T, C]
-    buffer).  Returns (O, lse)."""
+    Philox keep mask of (seed, offset), and stores the drawn keep bits in
+    ``dropout_mask`` (a uint8 tensor of attn_dropout_mask_bytes(B, H, T)
+    bytes) when one is given, for attn_bwd_ex to reuse.  Contiguous or strided
+    [B, H, T, D] views; O defaults to the layout of q (contiguous, else a
+    [B, T, C] buffer).  Returns (O, lse)."""
     torch = _torch()
     B, H, T, D = _shape4(q)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -370,7 +385,7 @@ def attn_fwd_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal
             _check_view(v, "v", q.shape), _check_view(o, "o", q.shape),
             _check(lse, "lse", torch.float32, (B, H, T))]
     st = None if _all_contiguous(q, k, v, o) else _strides_of(q, k, v, o)
-    opts = _options(causal, dropout_p, seed, offset)
+    opts = _options(causal, dropout_p, seed, offset, dropout_mask)
     with torch.cuda.device(q.device):
         _raise(_lib.attn_fwd_ex(*ptrs, B, H, T, D, scale, st, ctypes.byref(opts),
                                 _stream_handle(stream)), "attn_fwd_ex")
@@ -379,10 +394,11 @@ def attn_fwd_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal
 
 def attn_bwd_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[float] = None,
                 causal: bool = True, dropout_p: float = 0.0, seed: int = 0, offset: int = 0,
-                workspace=None, stream=None):
+                workspace=None, stream=None, dropout_mask=None):
     """bf16 backward with options (the same ``causal``, ``dropout_p``, ``seed``
     and ``offset`` as given to attn_fwd_ex), on contiguous or strided views.
-    Returns (dQ, dK, dV)."""
+    ``dropout_mask``: the buffer the forward stored its keep bits in, read
+    instead of drawing the mask again.  Returns (dQ, dK, dV)."""
     torch = _torch()
     B, H, T, D = _shape4(q)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -401,7 +417,7 @@ def attn_bwd_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[
             _check_view(dv, "dv", q.shape)]
     views = (q, k, v, o, dO, dq, dk, dv)
     st = None if _all_contiguous(*views) else _strides_of(*views)
-    opts = _options(causal, dropout_p, seed, offset)
+    opts = _options(causal, dropout_p, seed, offset, dropout_mask)
     ws_bytes = workspace.numel() * workspace.element_size()
     with torch.cuda.device(q.device):
         _raise(_lib.attn_bwd_ex(*ptrs, B, H, T, D, scale, st, ctypes.byref(opts),

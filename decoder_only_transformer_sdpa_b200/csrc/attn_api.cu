@@ -142,6 +142,8 @@ struct Opts {
     int causal = 1;
     bool dropout = false;
     DropoutParams drop{};
+    uint8_t *mask = nullptr;  // a kept dropout mask (dropout only), not yet checked
+    size_t mask_bytes = 0;
 };
 
 // Reads the options (NULL = the decoder's defaults: causal, no dropout).
@@ -162,7 +164,29 @@ int read_options(const attn_options *opts, Opts &out) {
         out.drop.thr = (uint32_t)t;
         out.drop.offset = opts->dropout_offset;
         out.drop.keep_scale = (float)(65536.0 / (65536.0 - t));
+        out.mask = static_cast<uint8_t *>(opts->dropout_mask);
+        out.mask_bytes = opts->dropout_mask_bytes;
     }
+    return ATTN_OK;
+}
+
+size_t mask_bytes_for(int B, int H, int T) {
+    if (B < 1 || H < 1 || T < 1) return 0;
+    const size_t tp = ((size_t)T + 127) / 128 * 128;
+    const size_t heads = (size_t)B * (size_t)H;
+    if (heads > (SIZE_MAX / tp) / (tp / 8)) return 0;
+    return heads * (tp / 8) * tp;
+}
+
+// Hands a kept dropout mask to the kernels once its size is checked against
+// the shape (bf16 path; the float32 path draws the mask every time).
+int attach_mask(Opts &op, int B, int H, int T) {
+    if (!op.dropout || !op.mask) return ATTN_OK;
+    const size_t need = mask_bytes_for(B, H, T);
+    if (need == 0 || op.mask_bytes < need) return ATTN_ERR_OPTION;
+    if (!aligned(op.mask, 16)) return ATTN_ERR_ALIGN;
+    op.drop.mask = op.mask;
+    op.drop.mask_ld = (uint32_t)(((size_t)T + 127) / 128 * 128);
     return ATTN_OK;
 }
 
@@ -201,7 +225,7 @@ int bwd_strides(const attn_strides *strides, const Shape &s, BwdStrides &str) {
 }
 
 int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int T,
-             int D, float scale, const Opts &op, const FwdStrides &str, cudaStream_t stream,
+             int D, float scale, Opts op, const FwdStrides &str, cudaStream_t stream,
              LaunchInfo &li) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
     int st = check_shape(B, H, T, D, 128);
@@ -210,6 +234,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     if ((st = check_scale(scale)) != ATTN_OK) return st;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
         return ATTN_ERR_ALIGN;
+    if ((st = attach_mask(op, B, H, T)) != ATTN_OK) return st;
     int *err = nullptr;
     if ((st = device_setup(&err)) != ATTN_OK) return st;
     cudaError_t e = sm100_fwd(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
@@ -236,10 +261,11 @@ int bwd_args(const void *q, const void *k, const void *v, const void *o, const f
 
 int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
              const void *dO, void *dq, void *dk, void *dv, int B, int H, int T, int D, float scale,
-             const Opts &op, const BwdStrides &str, void *workspace, size_t workspace_bytes,
+             Opts op, const BwdStrides &str, void *workspace, size_t workspace_bytes,
              cudaStream_t stream, LaunchInfo &li) {
     int st = bwd_args(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale);
     if (st != ATTN_OK) return st;
+    if ((st = attach_mask(op, B, H, T)) != ATTN_OK) return st;
     const size_t need = attn_bwd_workspace_bytes(B, H, T, D);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
     int *err = nullptr;
@@ -380,6 +406,8 @@ ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float 
                           int B, int H, int T, int D, float scale, cudaStream_t stream) {
     return attn_fwd_f32_ex(q, k, v, o, lse, B, H, T, D, scale, nullptr, stream);
 }
+
+ATTN_API size_t attn_dropout_mask_bytes(int B, int H, int T) { return mask_bytes_for(B, H, T); }
 
 ATTN_API size_t attn_bwd_f32_workspace_bytes(int B, int H, int T, int D) {
     if (check_shape(B, H, T, D, 128) != ATTN_OK) return 0;

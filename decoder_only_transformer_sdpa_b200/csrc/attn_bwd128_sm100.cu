@@ -233,6 +233,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int idx = 0; idx < n_q; ++idx) {
             const int st = idx % kQStages, b = idx & 1;
             const int i = q_first + idx;
+            // With a kept dropout mask, this sub-tile's keep bytes are loaded
+            // before the wait for S^T (byte r: keys 8 jg .. +7 of query ib + 8 r).
+            uint32_t kept = 0u;
+            if constexpr (Drop) {
+                if (dp.mask) {
+                    const uint32_t jg = (uint32_t)((kt * kBK + quad * 32 + (lane & ~7)) >> 3);
+                    const uint32_t ib = (uint32_t)(i * kBQ + q0) + (lane & 7);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        kept |= (uint32_t)__ldg(dp.mask + philox::mask_at(dp, (uint32_t)bh, jg, ib + 8u * r))
+                                << (8 * r);
+                }
+            }
             ok = mbar_wait_warp(&sm.sdp_full, (uint32_t)idx & 1u, err, abort);
             if (!ok) break;
             tc_fence_after();
@@ -253,10 +266,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t sub = (uint32_t)(lane & 7);
                 const uint32_t jg = (uint32_t)((kt * kBK + quad * 32 + (lane & ~7)) >> 3);
                 const uint32_t ib = (uint32_t)(i * kBQ + q0) + sub;
-                uint32_t wbits = 0;
+                uint32_t wbits = kept;
+                if (!dp.mask) {
 #pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    wbits |= philox::keep_byte(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
+                    for (int r = 0; r < 4; ++r)
+                        wbits |= philox::keep_byte(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
+                }
                 keepm = 0;
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {

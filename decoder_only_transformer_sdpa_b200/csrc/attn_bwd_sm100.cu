@@ -426,6 +426,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int idx = 0; idx < n_q; ++idx) {
             const int g = g0 + idx;
             const int st = g % kQStages, b = g & 1;
+            // With a kept dropout mask, this tile's keep bytes are loaded
+            // before the wait for S^T, so their latency overlaps it: byte r of
+            // kept[c] is keys 8 jg .. +7 of query ib + 8 r (as drawn below).
+            uint32_t kept[2] = {0u, 0u};
+            if constexpr (Drop) {
+                if (dp.mask) {
+                    const uint32_t jg = (uint32_t)((kt * kBT + quad * 32 + (lane & ~7)) >> 3);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const uint32_t ib = (uint32_t)((q_first + idx) * kBT + 64 * half + 32 * c) + (lane & 7);
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+                            kept[c] |= (uint32_t)__ldg(dp.mask + philox::mask_at(dp, (uint32_t)bh, jg, ib + 8u * r))
+                                       << (8 * r);
+                    }
+                }
+            }
             ok = mbar_wait_warp(&sm.sdp_full, (uint32_t)g & 1u, err, abort);
             if (!ok) break;
             tc_fence_after();
@@ -451,10 +468,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sub = (uint32_t)(lane & 7);
                     const uint32_t jg = (uint32_t)((kt * kBT + quad * 32 + (lane & ~7)) >> 3);
                     const uint32_t ib = (uint32_t)((q_first + idx) * kBT + q0) + sub;
-                    uint32_t wbits = 0;  // byte r: keys 8 jg .. +7 of query ib + 8 r
+                    uint32_t wbits = kept[c];  // byte r: keys 8 jg .. +7 of query ib + 8 r
+                    if (!dp.mask) {
 #pragma unroll
-                    for (int r = 0; r < 4; ++r)
-                        wbits |= philox::keep_byte(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
+                        for (int r = 0; r < 4; ++r)
+                            wbits |= philox::keep_byte(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
+                    }
                     keepm = 0;
 #pragma unroll
                     for (int s = 0; s < 8; ++s) {

@@ -554,10 +554,20 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 if constexpr (Drop) {
                     // Keep bits of this row, eight keys per generator call.
                     const uint32_t ti = (uint32_t)(qt * kBM + row);
+                    uint32_t kw = 0u;  // keep bytes of four key groups, kept for the backward
+                    uint32_t *mrow = dp.mask ? reinterpret_cast<uint32_t *>(
+                                                   dp.mask + philox::mask_at(dp, (uint32_t)bh,
+                                                                             (uint32_t)(j * (kBN / 8)), ti))
+                                             : nullptr;
 #pragma unroll
                     for (int g = 0; g < kBN / 8; ++g) {
                         const uint32_t kb = philox::keep_byte(dp, ti, (uint32_t)(j * (kBN / 8) + g),
                                                               (uint32_t)bh);
+                        kw |= kb << (8 * (g & 3));
+                        if ((g & 3) == 3) {
+                            if (mrow) mrow[g >> 2] = kw;
+                            kw = 0u;
+                        }
 #pragma unroll
                         for (int y = 0; y < 4; ++y) {
                             const int x = 4 * g + y;

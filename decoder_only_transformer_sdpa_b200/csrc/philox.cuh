@@ -12,6 +12,13 @@
 // key = seed) is >= the threshold t = round(p * 65536); lane e is bits
 // 16 (e mod 2) .. +15 of output word e / 2.  Kept weights are scaled by
 // 65536 / (65536 - t).
+//
+// Optionally the bytes are kept in device memory (mask != NULL): the forward
+// stores every keep byte it draws, and the backward loads them instead of
+// drawing them again.  Byte (query i, key group g) of head bh sits at
+// (bh * mask_ld + i) * mask_ld / 8 + g, with mask_ld the tile-padded length:
+// a forward thread stores its row's keep bytes four key groups (one word) at a
+// time.
 #pragma once
 
 #include <stdint.h>
@@ -23,6 +30,8 @@ struct DropoutParams {
     uint32_t thr;        // drop threshold t (0 < t < 65536 when dropout is on)
     uint32_t offset;     // counter word 3
     float keep_scale;    // 65536 / (65536 - t)
+    uint32_t mask_ld;    // tile-padded T: bytes per key-group row of the kept mask
+    uint8_t *mask;       // the kept keep bytes, or NULL (draw them)
 };
 
 namespace philox {
@@ -62,6 +71,11 @@ __device__ __forceinline__ uint32_t keep_byte(const DropoutParams &dp, uint32_t 
         bits |= (u >= dp.thr ? 1u : 0u) << e;
     }
     return bits;
+}
+
+// Offset of the kept byte of query i, key group g, head bh.
+__device__ __forceinline__ size_t mask_at(const DropoutParams &dp, uint32_t bh, uint32_t g, uint32_t i) {
+    return ((size_t)bh * dp.mask_ld + i) * (dp.mask_ld >> 3) + g;
 }
 
 }  // namespace philox

@@ -188,6 +188,22 @@ int attn_bwd_strided(const void *q, const void *k, const void *v, const void *o,
  *   needs a fresh mask (each layer, each step).  0 <= dropout_p < 1 with
  *   t < 65536, else ATTN_ERR_OPTION; t = 0 (p < 1/131072) is no dropout.
  *
+ * dropout_mask, dropout_mask_bytes: optional device buffer of at least
+ *   attn_dropout_mask_bytes(B,H,T) bytes that keeps the drawn mask, so that
+ *   the backward does not draw it again (the generator's ten rounds per eight
+ *   weights otherwise cost the backward as much as the forward).  With
+ *   dropout on and dropout_mask != NULL, attn_fwd_ex stores the keep bits of
+ *   every weight it draws there, and attn_bwd_ex loads them instead of drawing
+ *   them; the buffer must then hold what the forward of the same q, k, shape
+ *   and options stored (the results equal those of drawing the mask again).
+ *   Layout, for the curious: byte (query i, key group g = j / 8) of head
+ *   b*H + h is at ((b*H + h) * Tp + i) * Tp/8 + g with Tp = T rounded up to a
+ *   multiple of 128, bit e = key 8 g + e, 1 = kept.  The buffer must be
+ *   16-byte aligned (ATTN_ERR_ALIGN otherwise); one smaller than required
+ *   gives ATTN_ERR_OPTION.  The float32 entry points and calls without
+ *   dropout ignore the two fields.  NULL / 0 (the default): the backward
+ *   draws the mask again.
+ *
  * reserved: must be 0 (ATTN_ERR_OPTION otherwise). */
 typedef struct {
     int32_t causal;
@@ -195,7 +211,13 @@ typedef struct {
     uint64_t dropout_seed;
     uint32_t dropout_offset;
     uint32_t reserved;
+    void *dropout_mask;
+    size_t dropout_mask_bytes;
 } attn_options;
+
+/* Bytes of a kept dropout mask for a [B, H, T] attention (see attn_options);
+ * 0 on a bad shape. */
+size_t attn_dropout_mask_bytes(int B, int H, int T);
 
 /* attn_fwd with options, on strided views.  strides: NULL for contiguous
  * [B, H, T, D] tensors, else strides[0..3] for q, k, v, o under the rules of

@@ -200,10 +200,12 @@ def test_options_reserved_must_be_zero():
 
 def test_options_struct_layout():
     """The ctypes mirror of attn_options matches the C layout: int32, float,
-    uint64 (8-aligned), uint32, uint32 = 24 bytes."""
-    assert ctypes.sizeof(lib_mod.attn_options) == 24
+    uint64 (8-aligned), uint32, uint32, pointer, size_t = 40 bytes."""
+    assert ctypes.sizeof(lib_mod.attn_options) == 40
     assert lib_mod.attn_options.dropout_seed.offset == 8
     assert lib_mod.attn_options.dropout_offset.offset == 16
+    assert lib_mod.attn_options.dropout_mask.offset == 24
+    assert lib_mod.attn_options.dropout_mask_bytes.offset == 32
 
 
 @pytest.mark.parametrize("p", [0.0, 1e-6, 0.1, 0.99999])
@@ -230,3 +232,22 @@ def test_decode_pointer_and_stride_errors():
     assert lib.attn_decode(P, P, P, P, P, 1, 1, 1, 8, 64, -1.0, None, None) == E_SCALE
     bad = _strides(4, t=12)
     assert lib.attn_decode(P, P, P, P, P, 1, 1, 1, 8, 64, 0.125, bad, None) == E_ALIGN
+
+
+def test_dropout_mask_bytes_and_rejection():
+    """The kept-mask size is (B*H) * Tp/8 * Tp bytes with Tp = T rounded up to
+    128; a buffer below it is rejected before any device work."""
+    assert lib_mod.attn_dropout_mask_bytes(1, 1, 1) == 16 * 128
+    assert lib_mod.attn_dropout_mask_bytes(2, 3, 129) == 6 * 32 * 256
+    assert lib_mod.attn_dropout_mask_bytes(12, 12, 1024) == 144 * 128 * 1024
+    assert lib_mod.attn_dropout_mask_bytes(0, 1, 8) == 0
+    lib = lib_mod.lib()
+    E_OPTION = -10
+    small = ctypes.byref(lib_mod.attn_options(1, 0.1, 7, 0, 0, P, 16 * 128 - 1))
+    assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 1, 64, 0.125, None, small, None) == E_OPTION
+    assert lib.attn_bwd_ex(*([P] * 9), 1, 1, 1, 64, 0.125, None, small, P, 1 << 30, None) == E_OPTION
+    odd = ctypes.byref(lib_mod.attn_options(1, 0.1, 7, 0, 0, P + 8, 1 << 20))
+    assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 1, 64, 0.125, None, odd, None) == E_ALIGN
+    # without dropout the mask fields are ignored: the ordinary checks decide
+    off = ctypes.byref(lib_mod.attn_options(1, 0.0, 7, 0, 0, P, 1))
+    assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 1, 48, 0.125, None, off, None) == E_D

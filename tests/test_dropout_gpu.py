@@ -137,3 +137,68 @@ def test_bf16_zero_threshold_is_plain():
     b = parity.run_gpu(inp)
     for n in ("o", "lse", "dk", "dv"):
         assert np.array_equal(a[n], b[n]), n
+
+
+def _unpack_kept_mask(buf, B, H, T):
+    """The [B, H, T, T] keep bits of a kept dropout mask buffer (layout of
+    include/attn.h: byte (query i, key group g) of head bh at
+    (bh * Tp + i) * Tp/8 + g, bit e = key 8 g + e)."""
+    tp = (T + 127) // 128 * 128
+    by = buf.cpu().numpy().reshape(B * H, tp, tp // 8)           # [bh, i, g]
+    bits = np.unpackbits(by[..., None], axis=-1, bitorder="little")  # [bh, i, g, e]
+    m = bits.reshape(B * H, tp, tp)                              # [bh, i, 8 g + e]
+    return m[:, :T, :T].reshape(B, H, T, T)
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("causal", [True, False])
+def test_kept_mask_bits_equal_oracle(D, causal):
+    """The forward stores exactly the oracle's keep bits for every tile it
+    draws (with the mask, the tiles at or below the diagonal)."""
+    import decoder_only_transformer_sdpa_b200 as A
+    B, H, T, p, seed, offset = 2, 3, 300, 0.3, 0x5EED0123456789, 9
+    inp = random_qkv(71 + D, B, H, T, D, dtype=torch.bfloat16)
+    dev = torch.device("cuda", 0)
+    buf = torch.full((A.attn_dropout_mask_bytes(B, H, T),), 0xA5, dtype=torch.uint8, device=dev)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    A.attn_fwd_ex(q, k, v, causal=causal, dropout_p=p, seed=seed, offset=offset, dropout_mask=buf)
+    torch.cuda.synchronize()
+    assert A.attn_device_error() == 0
+    got = _unpack_kept_mask(buf, B, H, T)
+    ref = oracle.dropout_mask(B, H, T, p, seed, offset)
+    drawn = np.ones((T, T), dtype=bool)
+    if causal:  # tiles of 128 x 128 at or below the diagonal
+        tq = np.arange(T)[:, None] // 128
+        tk = np.arange(T)[None, :] // 128
+        drawn = tk <= tq
+    assert np.array_equal(got[..., drawn], ref[..., drawn]), \
+        f"{np.sum(got[..., drawn] != ref[..., drawn])} kept bits differ from the oracle's"
+
+
+@pytest.mark.parametrize("D,T", [(64, 333), (64, 1024), (128, 333), (32, 200)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_kept_mask_backward_matches_redraw(D, T, causal):
+    """The backward that reads the forward's kept mask gives what the one that
+    draws the mask again gives (dK, dV bit for bit; dQ, summed by float32
+    reduce-adds in whatever order they land, within its rounding), and both
+    match the oracle."""
+    import decoder_only_transformer_sdpa_b200 as A
+    B, H = 2, 2
+    inp = random_qkv(900 + T + D, B, H, T, D, dtype=torch.bfloat16, do_std=1e-2)
+    dev = torch.device("cuda", 0)
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    kw = dict(causal=causal, dropout_p=0.1, seed=123, offset=4)
+    buf = torch.zeros(A.attn_dropout_mask_bytes(B, H, T), dtype=torch.uint8, device=dev)
+    o1, lse1 = A.attn_fwd_ex(q, k, v, dropout_mask=buf, **kw)
+    g1 = A.attn_bwd_ex(q, k, v, o1, lse1, do, dropout_mask=buf, **kw)
+    o0, lse0 = A.attn_fwd_ex(q, k, v, **kw)
+    g0 = A.attn_bwd_ex(q, k, v, o0, lse0, do, **kw)
+    torch.cuda.synchronize()
+    assert A.attn_device_error() == 0
+    assert torch.equal(o1, o0) and torch.equal(lse1, lse0)
+    assert torch.equal(g1[1], g0[1]) and torch.equal(g1[2], g0[2])
+    assert torch.allclose(g1[0].float(), g0[0].float(), rtol=1e-2, atol=1e-6)
+    cpu = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    got = dict(o=cpu(o1), lse=cpu(lse1), dq=cpu(g1[0]), dk=cpu(g1[1]), dv=cpu(g1[2]))
+    parity.assert_close(got, parity.run_oracle(inp, causal=causal, dropout_p=0.1, seed=123, offset=4),
+                        torch.bfloat16, f"kept mask D={D} T={T} causal={causal}")
