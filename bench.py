@@ -534,8 +534,9 @@ def run_ours(args, w):
     # results (O, dQ, dK, dV).  Uploads run on one copy stream, downloads on
     # another, the kernels on the launching stream; events order each layer's
     # upload before its forward and its downloads after its forward /
-    # backward.  Two device buffer sets alternate between steps, so a step's
-    # uploads overlap the previous step's downloads (the link is full duplex).
+    # backward.  Three device buffer sets rotate between steps, so a step's
+    # uploads overlap the previous step's downloads (the link is full duplex)
+    # without waiting for the downloads of the step before that.
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
         host = [{n: b[n].cpu().pin_memory() for n in ("q", "k", "v", "do")} for b in layers]
@@ -543,16 +544,18 @@ def run_ours(args, w):
                      for n in ("o", "dq", "dk", "dv")} for b in layers]
         h2d = sum(t.numel() * t.element_size() for hb in host for t in hb.values())
         d2h = sum(t.numel() * t.element_size() for hb in out_host for t in hb.values())
-        sets = [layers, [{n: torch.empty_like(t) for n, t in b.items()} for b in layers]]
+        n_sets = 3
+        sets = [layers] + [[{n: torch.empty_like(t) for n, t in b.items()} for b in layers]
+                           for _ in range(n_sets - 1)]
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        released = [None, None]  # per buffer set: its last downloads are done
+        released = [None] * n_sets  # per buffer set: its last downloads are done
 
         def e2e_step(it):
-            bs = sets[it % 2]
+            bs = sets[it % n_sets]
             ev_in, ev_f, ev_b = [], [], [None] * L
             with torch.cuda.stream(up):
-                if released[it % 2] is not None:
-                    up.wait_event(released[it % 2])
+                if released[it % n_sets] is not None:
+                    up.wait_event(released[it % n_sets])
                 for l, b in enumerate(bs):
                     for n in ("q", "k", "v", "do"):
                         b[n].copy_(host[l][n], non_blocking=True)
@@ -577,9 +580,9 @@ def run_ours(args, w):
                     down.wait_event(ev_b[l])
                     for n in ("dq", "dk", "dv"):
                         out_host[l][n].copy_(bs[l][n], non_blocking=True)
-                released[it % 2] = torch.cuda.Event()
-                released[it % 2].record(down)
-        for it in range(2):
+                released[it % n_sets] = torch.cuda.Event()
+                released[it % n_sets].record(down)
+        for it in range(n_sets):
             e2e_step(it)
         stream.wait_stream(down)
         barrier()
@@ -596,8 +599,8 @@ def run_ours(args, w):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
                "copies": "uploads and downloads on two copy streams, overlapping the kernels and each "
-                         "other; two device buffer sets alternate between steps"}
-        del sets[1]
+                         "other; three device buffer sets rotate between steps"}
+        del sets[1:]
 
     # ---- secondary: the same step on the layouts nanoGPT's attention sees
     # (q, k, v slices of a [B, T, 3C] c_attn output; O, dO as [B, T, C];
