@@ -19,6 +19,10 @@ from typing import Optional
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn.so")
+# ATTN_LIBRARY selects another build of the same library, e.g. libattn_debug.so
+# (the kernels with device-side bounds checks, see build.py --debug).
+if os.environ.get("ATTN_LIBRARY"):
+    LIB_PATH = os.path.abspath(os.environ["ATTN_LIBRARY"])
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -85,13 +89,15 @@ _lib.attn_device_error.argtypes = [_vp]
 _lib.attn_device_error.restype = _i
 _lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _vp]
 _lib.attn_selftest_wait_timeout.restype = _i
+_lib.attn_selftest_device_check.argtypes = [_vp]
+_lib.attn_selftest_device_check.restype = _i
 _lib.attn_profile_next_call.argtypes = [_vp, _vp]
 _lib.attn_profile_next_call.restype = _i
 
 EXPORTED = ("attn_status_string", "attn_version", "attn_last_launch_count", "attn_fwd",
             "attn_bwd_workspace_bytes", "attn_bwd", "attn_fwd_f32", "attn_bwd_f32_workspace_bytes",
             "attn_bwd_f32", "attn_device_error", "attn_profile_next_call",
-            "attn_selftest_wait_timeout", "attn_bwd_noalloc", "attn_fwd_strided",
+            "attn_selftest_wait_timeout", "attn_selftest_device_check", "attn_bwd_noalloc", "attn_fwd_strided",
             "attn_bwd_strided", "attn_fwd_ex", "attn_bwd_ex", "attn_fwd_f32_ex", "attn_bwd_f32_ex",
             "attn_decode", "attn_dropout_mask_bytes")
 

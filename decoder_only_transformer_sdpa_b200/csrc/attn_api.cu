@@ -111,6 +111,7 @@ ATTN_API const char *attn_status_string(int status) {
         case ATTN_ERR_DEVICE: return "current device is not sm_100 (B200 class)";
         case ATTN_ERR_SCALE: return "scale must be finite and positive";
         case ATTN_ERR_OPTION: return "unsupported attn_options value";
+        case ATTN_ERR_DEVICE_CHECK: return "a device-side bounds check failed (debug build)";
         default: return "unknown status";
     }
 }
@@ -456,7 +457,7 @@ ATTN_API int attn_device_error(cudaStream_t stream) {
         const int zero = 0;
         if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
             return ATTN_ERR_CUDA;
-        return ATTN_ERR_TIMEOUT;
+        return h == kErrBounds ? ATTN_ERR_DEVICE_CHECK : ATTN_ERR_TIMEOUT;
     }
     return ATTN_OK;
 }
@@ -467,6 +468,13 @@ ATTN_API int attn_selftest_wait_timeout(uint32_t polls, cudaStream_t stream) {
     int st = device_setup(&err);
     if (st != ATTN_OK) return st;
     return selftest_wait_timeout(polls, err, stream) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+ATTN_API int attn_selftest_device_check(cudaStream_t stream) {
+    int *err = nullptr;
+    int st = device_setup(&err);
+    if (st != ATTN_OK) return st;
+    return selftest_failed_check(err, stream) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 namespace attn {

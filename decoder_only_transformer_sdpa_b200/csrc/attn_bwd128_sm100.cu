@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dep_wait();
     grid_dep_launch();
     const uint32_t tmem = sm.tmem_slot;
+    ATTN_DCHECK(tmem == 0u, err);  // all 512 columns, from lane 0 column 0
     const uint32_t tS = tmem, tdP = tmem + 64, tdV = tmem + 128, tdK = tmem + 256;
     const uint32_t tdQ = tmem + 384, tP = tmem + 448;
 
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_4d_e(sm.dO[st][sl], &tdo, &sm.qdo_full[st], 64 * sl, i * kBQ, hh, bb);
             }
             const size_t prow = (size_t)bh * Tpad + (size_t)i * kBQ;
+            ATTN_DCHECK(kt * kBK < T && prow + kBQ <= (size_t)BH * Tpad && i * kBQ < T, err);
             bulk_load_e(sm.lse2[st], lse2 + prow, kBQ * 4, &sm.qdo_full[st]);
             bulk_load_e(sm.delta[st], delta + prow, kBQ * 4, &sm.qdo_full[st]);
             issued = idx + 1;
@@ -390,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (leader) {
+                ATTN_DCHECK((q_first + idx) * kBQ < T, err);
                 for (int db = 0; db < 4; ++db)
                     tma_reduce_add_3d(&tdq, sm.stage[db], 32 * db, (q_first + idx) * kBQ, bh);
                 bulk_commit();

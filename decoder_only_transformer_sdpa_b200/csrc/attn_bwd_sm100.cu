@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dep_wait();
     grid_dep_launch();
     const uint32_t tmem = sm.tmem_slot;
+    ATTN_DCHECK(tmem == 0u, err);  // all 512 columns, from lane 0 column 0
     const uint32_t tS = tmem, tdP = tmem + 128;
     const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D, tdQ = tmem + 256 + 2 * D;
     const uint32_t tP = tmem + 256 + 3 * D;
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kt = w / BH, bh = w % BH, hh = bh % H, bb = bh / H;
             const int q_first = Causal ? kt : 0;
             const int kb = n & 1;
+            ATTN_DCHECK(kt >= 0 && kt < nt && bh >= 0 && bh < BH && kt * kBT < T, err);
             if (n >= 2 && !(ok = mbar_wait_warp(&sm.kv_empty[kb], (uint32_t)((n >> 1) - 1) & 1u, err, abort)))
                 break;
             mbar_arrive_expect_tx_e(&sm.kv_full[kb], 2 * Smem::kTileBytes);
@@ -298,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_4d_e(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, hh, bb);
                 tma_load_4d_e(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, hh, bb);
                 const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
+                ATTN_DCHECK(prow + kBT <= (size_t)BH * Tpad && i * kBT < T, err);
                 bulk_load_e(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
                 bulk_load_e(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
             }
@@ -449,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool diag = Causal && (idx == 0);
             const uint32_t lse_addr = smem_u32(sm.lse2[st]), dl_addr = smem_u32(sm.delta[st]);
             const uint32_t ds_row = smem_u32(sm.ds[b][half]) + (uint32_t)kr * 128;
+            ATTN_DCHECK(kr < kBT && (kr + 1) * 128 <= (int)sizeof(sm.ds[0][0]), err);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {  // 32 query columns per chunk
                 const int q0 = 64 * half + 32 * c;
@@ -576,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
                 if (leader) {
+                    ATTN_DCHECK((q_first + idx) * kBT < T && bh < BH, err);
                     tma_reduce_add_3d(&tdq, sm.stage, 32 * h, (q_first + idx) * kBT, bh);
                     bulk_commit();
                 }

@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kThreads)
     // This CTA's tiles: rank, rank + cs, ... (tile 0, which every query sees,
     // is always in CTA 0).
     const int my_tiles = rank < ntiles ? (ntiles - 1 - rank) / cs + 1 : 0;
+    ATTN_DCHECK(bb >= 0 && hh >= 0 && hh < H && cs <= kMaxCluster, err);
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(kThreads)
         // The first tiles start streaming before anything else happens.
         for (int n = 0; n < kStages && n < my_tiles; ++n) {
             const int tile = rank + n * cs;
+            ATTN_DCHECK(tile >= 0 && tile < ntiles, err);
             mbar_arrive_expect_tx(&sm.full[n], 2 * Smem::kTileBytes);
             tma_load_4d(sm.k[n], &tk, &sm.full[n], 0, tile * kTile, hh, bb);
             tma_load_4d(sm.v[n], &tv, &sm.full[n], 0, tile * kTile, hh, bb);
@@ -162,6 +164,7 @@ __global__ void __launch_bounds__(kThreads)
                 const int s = n % kStages;
                 if (!mbar_wait(&sm.empty[s], (uint32_t)((n / kStages) - 1) & 1u, err, abort)) break;
                 const int tile = rank + n * cs;
+                ATTN_DCHECK(tile >= 0 && tile < ntiles, err);
                 mbar_arrive_expect_tx(&sm.full[s], 2 * Smem::kTileBytes);
                 tma_load_4d(sm.k[s], &tk, &sm.full[s], 0, tile * kTile, hh, bb);
                 tma_load_4d(sm.v[s], &tv, &sm.full[s], 0, tile * kTile, hh, bb);
@@ -181,6 +184,7 @@ __global__ void __launch_bounds__(kThreads)
         for (int n = 0; n < my_tiles; ++n) {
             const int s = n % kStages;
             const int tile = rank + n * cs;
+            ATTN_DCHECK(tile >= 0 && tile < ntiles, err);
             if (!(ok = mbar_wait_warp(&sm.full[s], (uint32_t)(n / kStages) & 1u, err, abort))) break;
             const int row = warp * kKeys + kk;  // this lane pair's key row in the tile
             // ---- scores of the warp's 16 keys (two lanes per row)

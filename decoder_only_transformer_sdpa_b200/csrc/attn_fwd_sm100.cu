@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
     grid_dep_wait();
     grid_dep_launch();
     const uint32_t tmem = sm.tmem_slot;
+    ATTN_DCHECK((tmem >> 16) == 0u && (tmem & 0xFFFFu) + kTmemCols <= 512u, err);  // lane 0, within TMEM
     const uint32_t tS = tmem;
     const uint32_t tP = tmem + 128;
     const uint32_t tO = tmem + 192;
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 const int qt = ntiles - 1 - w / BH, bh = w % BH;
                 const int hh = bh % H, bb = bh / H;
                 const int qb = n & 1;
+                ATTN_DCHECK(qt >= 0 && qt < ntiles && bh >= 0 && bh < BH, err);
                 if (!(ok = mbar_wait_warp(&sm.q_empty[qb], (uint32_t)((n >> 1) & 1) ^ 1u, err, abort))) break;
                 mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
 #pragma unroll
@@ -218,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 nq = n + 1;
                 const int nk = Causal ? qt + 1 : ntiles;  // key tiles this item reads
                 for (int j = 0; j < nk; ++j, ++gt) {
+                    ATTN_DCHECK(j * kBN < T, err);  // the key tile holds at least one key
                     const int s = gt % kStages;
                     const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
                     if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
@@ -253,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 const int qt = ntiles - 1 - w / BH, bh = w % BH;
                 const int hh = bh % H, bb = bh / H;
                 const int qb = n & 1;
+                ATTN_DCHECK(qt >= 0 && qt < ntiles && bh >= 0 && bh < BH, err);
                 if (!(ok = mbar_wait_warp(&sm.q_empty[qb], (uint32_t)((n >> 1) & 1) ^ 1u, err, abort))) break;
                 mbar_arrive_expect_tx_e(&sm.q_full[qb], Smem::kTileBytes);
 #pragma unroll
@@ -262,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 nq = n + 1;
                 const int nk = Causal ? qt + 1 : ntiles;  // key tiles this item reads
                 for (int j = 0; j < nk; ++j, ++gt) {
+                    ATTN_DCHECK(j * kBN < T, err);  // the key tile holds at least one key
                     const int s = gt % kStages;
                     const uint32_t ph = (uint32_t)(gt / kStages) & 1u;
                     if (!(ok = mbar_wait_warp(&sm.k_empty[s], ph ^ 1u, err, abort))) break;
@@ -423,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                     const int col0 = 32 * (h0 + h);  // first column of this load
                     const int sl = col0 / kSlabCols;
                     const uint32_t base = smem_u32(qbuf + sl * kSlabBytes) + (uint32_t)row * kRowBytes;
+                    ATTN_DCHECK(sl * kSlabBytes + (row + 1) * kRowBytes <= (int)sizeof(sm.q[0]), err);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {  // 16-byte chunks of 8 columns
                         const uint32_t chunk = (uint32_t)((col0 % kSlabCols) / 8 + c);
@@ -451,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 }
             }
             const int t = pqt * kBM + row;
+            ATTN_DCHECK(pbh >= 0 && pbh < BH && row < kBM, err);
             if (t < T) lse[(size_t)pbh * T + t] = (pm + log2f(pl)) * 0.69314718055994531f;
             return true;
         };

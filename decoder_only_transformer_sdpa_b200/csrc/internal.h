@@ -18,6 +18,21 @@ namespace attn {
 // roughly 0.1 s to a few seconds; legitimate waits last microseconds.
 constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr int kErrTimeout = 1;
+// The debug build (-DATTN_DEVICE_CHECKS) checks tile coordinates, TMEM column
+// ranges and shared-memory offsets inside the kernels; a failed check records
+// kErrBounds in the device error word and the kernel carries on (nothing
+// traps).  The release build compiles the checks away.
+constexpr int kErrBounds = 3;
+#ifdef ATTN_DEVICE_CHECKS
+#define ATTN_DCHECK(cond, err)                           \
+    do {                                                 \
+        if (!(cond)) atomicExch((err), ::attn::kErrBounds); \
+    } while (0)
+#else
+#define ATTN_DCHECK(cond, err) \
+    do {                       \
+    } while (0)
+#endif
 
 struct Shape {
     int B, H, T, D;
@@ -144,6 +159,9 @@ inline BwdWorkspace bwd_workspace_layout(int B, int H, int T, int D) {
 // Launches one thread that waits on an mbarrier nobody arrives at, polling at
 // most `polls` times, so the timeout path can be exercised without a fault.
 cudaError_t selftest_wait_timeout(uint32_t polls, int *err, cudaStream_t st);
+// Runs one device-side bounds check that cannot hold (recorded by the debug
+// build, compiled away by the release build).
+cudaError_t selftest_failed_check(int *err, cudaStream_t st);
 
 // The argument checks attn_bwd runs before it looks at its workspace
 // (pointers, shape, head_dim, scale, alignment, in that order): ATTN_OK or the

@@ -1,7 +1,11 @@
-// selftest.cu -- exercises the bounded-wait error path: a single thread waits
-// on a fresh mbarrier that no one arrives at, gives up after a given number
-// of polls and records the timeout in the device error word, exactly as the
-// attention kernels do when a wait runs out.  Nothing faults or hangs.
+// selftest.cu -- exercises the kernels' error paths without a fault:
+//  * the bounded wait: a single thread waits on a fresh mbarrier that no one
+//    arrives at, gives up after a given number of polls and records the
+//    timeout in the device error word, exactly as the attention kernels do
+//    when a wait runs out;
+//  * the debug build's bounds checks: one check that cannot hold, which the
+//    debug build records like any failed check (and the release build
+//    compiles away).  Nothing faults or hangs.
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -18,10 +22,19 @@ __global__ void wait_timeout_kernel(uint32_t polls, int *err) {
     atomicExch(err, kErrTimeout);
 }
 
+__global__ void failed_check_kernel(int *err) {
+    ATTN_DCHECK(threadIdx.x >= blockDim.x, err);  // never holds; touches no memory
+}
+
 }  // namespace
 
 cudaError_t selftest_wait_timeout(uint32_t polls, int *err, cudaStream_t st) {
     wait_timeout_kernel<<<1, 32, 0, st>>>(polls, err);
+    return cudaGetLastError();
+}
+
+cudaError_t selftest_failed_check(int *err, cudaStream_t st) {
+    failed_check_kernel<<<1, 32, 0, st>>>(err);
     return cudaGetLastError();
 }
 

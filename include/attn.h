@@ -73,7 +73,9 @@ typedef enum {
     ATTN_ERR_WORKSPACE = -7,     /* workspace NULL or smaller than required         */
     ATTN_ERR_DEVICE = -8,        /* current device is not sm_100 (B200 class)       */
     ATTN_ERR_SCALE = -9,         /* scale is not finite and positive                */
-    ATTN_ERR_OPTION = -10        /* an attn_options field holds an unsupported value */
+    ATTN_ERR_OPTION = -10,       /* an attn_options field holds an unsupported value */
+    ATTN_ERR_DEVICE_CHECK = -11  /* a device-side bounds check failed (the debug
+                                    build, libattn_debug.so, only)               */
 } attn_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -290,7 +292,10 @@ int attn_bwd_f32_ex(const float *q, const float *k, const float *v, const float 
 
 /* Synchronises `stream`, then reads and clears the current device's
  * in-kernel error flag.  Returns ATTN_OK, ATTN_ERR_TIMEOUT (a bounded wait
- * ran out since the last call) or ATTN_ERR_CUDA (the sync itself failed). */
+ * ran out since the last call), ATTN_ERR_DEVICE_CHECK (the debug build
+ * libattn_debug.so only: a kernel's bounds check on a tile coordinate, TMEM
+ * column or shared-memory offset failed; the kernel records it and carries
+ * on) or ATTN_ERR_CUDA (the sync itself failed). */
 int attn_device_error(cudaStream_t stream);
 
 /* Failure-path self test: enqueues one thread that waits on an in-kernel
@@ -299,6 +304,13 @@ int attn_device_error(cudaStream_t stream);
  * does.  A following attn_device_error() then returns ATTN_ERR_TIMEOUT.
  * Faults nothing and never hangs. */
 int attn_selftest_wait_timeout(uint32_t polls, cudaStream_t stream);
+
+/* Self test of the device-side bounds checks: enqueues one kernel that runs
+ * a single check that cannot hold and touches no memory.  In the debug build
+ * (libattn_debug.so) a following attn_device_error() returns
+ * ATTN_ERR_DEVICE_CHECK; the release build compiles the check away, and it
+ * returns ATTN_OK. */
+int attn_selftest_device_check(cudaStream_t stream);
 
 /* Number of kernels the most recent successful call on this host thread
  * enqueued (for launch accounting). */

@@ -251,3 +251,18 @@ def test_dropout_mask_bytes_and_rejection():
     # without dropout the mask fields are ignored: the ordinary checks decide
     off = ctypes.byref(lib_mod.attn_options(1, 0.0, 7, 0, 0, P, 1))
     assert lib.attn_fwd_ex(P, P, P, P, P, 1, 1, 1, 48, 0.125, None, off, None) == E_D
+
+
+def test_debug_library_exports_the_same_abi():
+    """build() also makes libattn_debug.so (the kernels with the device-side
+    bounds checks); it exports exactly the release library's symbols, and its
+    failed-check status has its own message."""
+    import subprocess
+    dbg = os.path.join(os.path.dirname(lib_mod.LIB_PATH), "libattn_debug.so")
+    assert os.path.exists(dbg), "libattn_debug.so is not built (build.py --debug)"
+    names = lambda p: {ln.split()[-1] for ln in subprocess.run(
+        ["nm", "-D", "--defined-only", p], capture_output=True, text=True, check=True).stdout.splitlines()
+        if ln.split()[-1].startswith("attn_")}
+    assert names(dbg) == names(lib_mod.LIB_PATH)
+    E_CHECK = -11
+    assert "bounds check" in lib_mod.attn_status_string(E_CHECK)
