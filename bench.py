@@ -649,19 +649,26 @@ def run_ours(args, w):
         # with dropout, each layer's forward keeps its drawn mask for its backward
         masks = [torch.empty(A.attn_dropout_mask_bytes(w.B, w.H, w.T), dtype=torch.uint8, device=dev)
                  if dropout_p > 0 else None for _ in range(L)]
-        evn = [((mk(), mk()), (mk(), mk())) for _ in range(n_v + 1)]
+        evn = [((mk(), mk()), (mk(), mk()), (mk(), mk())) for _ in range(n_v + 1)]
         for e in evn:
             for pair in e:
                 for x in pair:
                     x.record(stream)
+        # whole forward call (with a lent mask: the mask draw, then the forward
+        # kernel) on another layer than the one whose kernels are bracketed
+        CL = (PL + 1) % L
 
-        def v_step(it, ev_fwd=None, ev_bwd=None):
+        def v_step(it, ev_fwd=None, ev_bwd=None, ev_call=None):
             for l, b in enumerate(layers):
                 if ev_fwd is not None and l == PL:
                     A.attn_profile_next_call(*ev_fwd)
+                if ev_call is not None and l == CL and CL != PL:
+                    ev_call[0].record(stream)
                 A.attn_fwd_ex(b["q"], b["k"], b["v"], b["o"], b["lse"], causal=causal,
                               dropout_p=dropout_p, seed=args.seed + 1, offset=it * L + l,
                               dropout_mask=masks[l])
+                if ev_call is not None and l == CL and CL != PL:
+                    ev_call[1].record(stream)
             for l in range(L - 1, -1, -1):
                 b = layers[l]
                 if ev_bwd is not None and l == PL:
@@ -683,6 +690,7 @@ def run_ours(args, w):
         pairs_v = w.causal_pairs() if causal else w.B * w.H * w.T * w.T
         nf = statistics.mean(e[0][0].elapsed_time(e[0][1]) for e in evn[:n_v])
         nb = statistics.mean(e[1][0].elapsed_time(e[1][1]) for e in evn[:n_v])
+        nc = statistics.mean(e[2][0].elapsed_time(e[2][1]) for e in evn[:n_v]) if CL != PL else None
         tf = lambda fl, ms_: fl / (ms_ * 1e-3) / 1e12
         del masks
         return {"value": whole_job_tflops(12 * w.D * pairs_v * L, world, n_v, v_ms),
@@ -692,6 +700,10 @@ def run_ours(args, w):
                 "flops_per_layer": 12 * w.D * pairs_v,
                 "fwd_main": {"avg_launch_ms": nf, "tflops": tf(4 * w.D * pairs_v, nf),
                              "frac": tf(4 * w.D * pairs_v, nf) / peak},
+                "fwd_call": None if nc is None else
+                            {"avg_ms": nc, "tflops": tf(4 * w.D * pairs_v, nc),
+                             "note": "events around the whole forward call (mask draw + forward kernel "
+                                     "when a mask is lent); events between launches cost the PDL overlap"},
                 "bwd_main": {"avg_launch_ms": nb, "tflops": tf(8 * w.D * pairs_v, nb),
                              "frac": tf(8 * w.D * pairs_v, nb) / peak}}
 

@@ -238,9 +238,16 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, i
     if ((st = attach_mask(op, B, H, T)) != ATTN_OK) return st;
     int *err = nullptr;
     if ((st = device_setup(&err)) != ATTN_OK) return st;
+    const Shape sh = make_shape(B, H, T, D, scale, op);
+    if (sh.drop.mask) {
+        // A lent mask buffer: draw the keep bits into it first; the forward
+        // (and later the backward) load them.
+        const cudaError_t em = draw_dropout_mask(sh, err, stream, li);
+        if (em != cudaSuccess) return finish(em, li);
+    }
     cudaError_t e = sm100_fwd(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
                               static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), lse,
-                              make_shape(B, H, T, D, scale, op), str, err, stream, li);
+                              sh, str, err, stream, li);
     return finish(e, li);
 }
 

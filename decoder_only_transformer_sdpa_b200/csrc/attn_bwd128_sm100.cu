@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!dp.mask) {
 #pragma unroll
                     for (int r = 0; r < 4; ++r)
-                        wbits |= philox::keep_byte(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
+                        wbits |= philox::keep_byte_lanes(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
                 }
                 keepm = 0;
 #pragma unroll
@@ -365,7 +365,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // swizzled [64 query][32 d] block, then one thread adds the four
         // blocks into the float32 accumulator.
         const int quad = warp & 3;
-        const int d = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const bool leader = (warp == 10 && lane == 0);
         const uint32_t blk = smem_u32(sm.stage[quad]);

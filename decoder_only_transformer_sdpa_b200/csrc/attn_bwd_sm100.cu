@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!dp.mask) {
 #pragma unroll
                         for (int r = 0; r < 4; ++r)
-                            wbits |= philox::keep_byte(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
+                            wbits |= philox::keep_byte_lanes(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
                     }
                     keepm = 0;
 #pragma unroll

@@ -40,16 +40,18 @@
 //               item boundary.  O / l is staged in the item's Q buffer, no
 //               longer read by then.
 // At D <= 64 (two CTAs per SM, 128 registers per thread at launch) the first
-// warpgroup hands registers to the softmax warpgroup with setmaxnreg: 56 and
-// 200 per thread, 128 x 56 + 128 x 200 = the block's 256 x 128; the launch
+// warpgroup hands registers to the softmax warpgroup with setmaxnreg: 48 and
+// 208 per thread, 128 x 48 + 128 x 208 = the block's 256 x 128; the launch
 // checks that the kernel was built with exactly 128 registers per thread.
 // Key tiles wholly above the diagonal are never loaded; only the diagonal
 // tile applies the element mask.  The score matrix never leaves the SM.
 // Without the mask (Causal = false) every query tile runs over all key tiles
 // and only the last key tile masks the keys past T.  With dropout (Drop) each
-// softmax thread draws its row's keep bits from Philox4x32-10, eight keys per
-// call (philox.cuh): the row sum l takes every weight, P_j in TMEM only the
-// kept ones, and the final O is scaled by keep_scale / l.
+// softmax thread takes its row's 16 keep bytes of a key tile before waiting for
+// the tile's S: one 16-byte load from the kept mask when the caller lent one
+// (drawn beforehand by dropout_mask.cu), else drawn here from Philox4x32-10,
+// eight keys per call (philox.cuh).  The row sum l takes every weight, P_j in
+// TMEM only the kept ones, and the final O is scaled by keep_scale / l.
 //
 // TMEM columns: S [0,128), P (bf16 pairs) [128,192), O [192, 192+D).
 #include "internal.h"
@@ -68,8 +70,8 @@ constexpr int kStages = 2;        // K/V ring depth
 constexpr int kThreads = 256;     // 8 warps (two warpgroups)
 constexpr int kSoftmaxWarp0 = 4;  // first softmax warp (the second warpgroup)
 constexpr int kRegsLaunch = 128;  // registers per thread at launch (D <= 64)
-constexpr int kRegsLow = 56;      // first warpgroup after the hand-over
-constexpr int kRegsHigh = 200;    // softmax warpgroup after the hand-over
+constexpr int kRegsLow = 48;      // first warpgroup after the hand-over
+constexpr int kRegsHigh = 208;    // softmax warpgroup after the hand-over
 static_assert(kRegsLow + kRegsHigh == 2 * kRegsLaunch, "the register split must add up");
 // TMEM columns: 256 at D <= 64, 512 (of which 320 used) at D = 128
 template <int D>
@@ -99,6 +101,18 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void 
         " [%0, {%1, %2, %3, %4}], [%5];" ::"l"(reinterpret_cast<uint64_t>(map)),
         "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(src))
         : "memory");
+}
+
+// The bf16-pair mask of keys e0 and e0 + 1 (e0 even, < 32) of a word W of keep
+// bits, given sh[t] = W << t: the sign bit of byte b of sh[t] is bit 8b + 7 - t
+// of W, and prmt with a sign-replicating selector copies a byte's sign bit over
+// a whole byte; the low half takes key e0, the high half key e0 + 1.
+__device__ __forceinline__ uint32_t keep_pair_mask(const uint32_t (&sh)[8], int e0) {
+    const int b = e0 >> 3;
+    const uint32_t sel = (uint32_t)(8 + b) * 0x0011u | (uint32_t)(12 + b) * 0x1100u;
+    uint32_t m;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m) : "r"(sh[7 - (e0 & 7)]), "r"(sh[6 - (e0 & 7)]), "r"(sel));
+    return m;
 }
 
 // The n-th work item of CTA c in a grid of G CTAs over W items (snake order),
@@ -472,6 +486,33 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
             float m_used = -INFINITY, l = 0.f;
             const int nk = Causal ? qt + 1 : ntiles;
             for (int j = 0; j < nk; ++j, ++gt) {
+                // This row's keep bits against key tile j (Drop), four 8-key
+                // groups (bytes) per word, ready before S is: loaded from the
+                // kept mask, or drawn here, eight keys per generator call.
+                [[maybe_unused]] uint32_t kwv[kBN / 32];
+                if constexpr (Drop) {
+                    const uint32_t ti = (uint32_t)(qt * kBM + row);
+                    if (dp.mask) {
+                        ATTN_DCHECK(ti < dp.mask_ld && (uint32_t)(j + 1) * kBN <= dp.mask_ld, err);
+                        const uint4 mw = __ldg(reinterpret_cast<const uint4 *>(
+                            dp.mask + philox::mask_at(dp, (uint32_t)bh, (uint32_t)(j * (kBN / 8)), ti)));
+                        kwv[0] = mw.x;
+                        kwv[1] = mw.y;
+                        kwv[2] = mw.z;
+                        kwv[3] = mw.w;
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < kBN / 32; ++q) {
+                            uint32_t w4 = 0u;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                w4 |= philox::keep_byte(dp, ti, (uint32_t)(j * (kBN / 8) + 4 * q + e),
+                                                        (uint32_t)bh)
+                                      << (8 * e);
+                            kwv[q] = w4;
+                        }
+                    }
+                }
                 ok = mbar_wait_warp(&sm.s_full, (uint32_t)gt & 1u, err, abort);
                 if (!ok) break;
                 tc_fence_after();
@@ -559,31 +600,23 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 uint32_t pk[kBN / 2];
                 float la = 0.f, lb = 0.f;
                 if constexpr (Drop) {
-                    // Keep bits of this row, eight keys per generator call.
-                    const uint32_t ti = (uint32_t)(qt * kBM + row);
-                    uint32_t kw = 0u;  // keep bytes of four key groups, kept for the backward
-                    uint32_t *mrow = dp.mask ? reinterpret_cast<uint32_t *>(
-                                                   dp.mask + philox::mask_at(dp, (uint32_t)bh,
-                                                                             (uint32_t)(j * (kBN / 8)), ti))
-                                             : nullptr;
+                    // Word q of keep bits covers keys 32q .. 32q+31 (bit e = key
+                    // 32q + e); its left shifts by 0..7 put every key's bit in the
+                    // sign position of some byte, so a byte permute turns the two
+                    // bits of a key pair into the pair's bf16 mask.
 #pragma unroll
-                    for (int g = 0; g < kBN / 8; ++g) {
-                        const uint32_t kb = philox::keep_byte(dp, ti, (uint32_t)(j * (kBN / 8) + g),
-                                                              (uint32_t)bh);
-                        kw |= kb << (8 * (g & 3));
-                        if ((g & 3) == 3) {
-                            if (mrow) mrow[g >> 2] = kw;
-                            kw = 0u;
-                        }
+                    for (int q = 0; q < kBN / 32; ++q) {
+                        uint32_t sh[8];
 #pragma unroll
-                        for (int y = 0; y < 4; ++y) {
-                            const int x = 4 * g + y;
+                        for (int t = 0; t < 8; ++t) sh[t] = kwv[q] << t;
+#pragma unroll
+                        for (int y = 0; y < 16; ++y) {
+                            const int x = 16 * q + y;
                             const float p0 = ex2(fmaf(s[2 * x], scale_log2, neg_m));
                             const float p1 = ex2(fmaf(s[2 * x + 1], scale_log2, neg_m));
                             la += p0;
                             lb += p1;
-                            pk[x] = pack_bf16x2((kb >> (2 * y)) & 1u ? p0 : 0.f,
-                                                (kb >> (2 * y + 1)) & 1u ? p1 : 0.f);
+                            pk[x] = pack_bf16x2(p0, p1) & keep_pair_mask(sh, 2 * y);
                         }
                     }
                 } else {

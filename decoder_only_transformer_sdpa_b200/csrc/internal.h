@@ -130,6 +130,11 @@ cudaError_t sm100_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                       float *dq_acc, float *lse2, float *delta, Shape s, const BwdStrides &str,
                       int *err, cudaStream_t st, LaunchInfo &li);
 
+// Draws the keep bytes of every tile the bf16 kernels visit into s.drop.mask
+// (laid out as philox.cuh describes); launched ahead of the forward when the
+// caller lends a mask buffer.
+cudaError_t draw_dropout_mask(const Shape &s, int *err, cudaStream_t st, LaunchInfo &li);
+
 // The backward main kernel at D = 128 (prep and post kernels run around it in
 // sm100_bwd).
 cudaError_t sm100_bwd128_main(const __nv_bfloat16 *q, const __nv_bfloat16 *k,

@@ -192,12 +192,14 @@ int attn_bwd_strided(const void *q, const void *k, const void *v, const void *o,
  *
  * dropout_mask, dropout_mask_bytes: optional device buffer of at least
  *   attn_dropout_mask_bytes(B,H,T) bytes that keeps the drawn mask, so that
- *   the backward does not draw it again (the generator's ten rounds per eight
- *   weights otherwise cost the backward as much as the forward).  With
- *   dropout on and dropout_mask != NULL, attn_fwd_ex stores the keep bits of
- *   every weight it draws there, and attn_bwd_ex loads them instead of drawing
- *   them; the buffer must then hold what the forward of the same q, k, shape
- *   and options stored (the results equal those of drawing the mask again).
+ *   neither the forward's softmax nor the backward runs the generator (its
+ *   ten rounds per eight weights otherwise cost each of them about as much
+ *   as the attention itself).  With dropout on and dropout_mask != NULL,
+ *   attn_fwd_ex first draws the keep bits of every weight the kernels visit
+ *   into the buffer (one extra kernel on the same stream) and its attention
+ *   kernel loads them; attn_bwd_ex loads them instead of drawing them.  The
+ *   buffer must then hold what the forward of the same shape and options
+ *   stored (the results equal those of drawing the mask in the kernels).
  *   Layout, for the curious: byte (query i, key group g = j / 8) of head
  *   b*H + h is at ((b*H + h) * Tp + i) * Tp/8 + g with Tp = T rounded up to a
  *   multiple of 128, bit e = key 8 g + e, 1 = kept.  The buffer must be

@@ -153,8 +153,8 @@ def _unpack_kept_mask(buf, B, H, T):
 @pytest.mark.parametrize("D", [32, 64, 128])
 @pytest.mark.parametrize("causal", [True, False])
 def test_kept_mask_bits_equal_oracle(D, causal):
-    """The forward stores exactly the oracle's keep bits for every tile it
-    draws (with the mask, the tiles at or below the diagonal)."""
+    """The forward call stores exactly the oracle's keep bits for every tile
+    the kernels visit (with the mask, the tiles at or below the diagonal)."""
     import decoder_only_transformer_sdpa_b200 as A
     B, H, T, p, seed, offset = 2, 3, 300, 0.3, 0x5EED0123456789, 9
     inp = random_qkv(71 + D, B, H, T, D, dtype=torch.bfloat16)
