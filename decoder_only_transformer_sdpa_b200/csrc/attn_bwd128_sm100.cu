@@ -274,12 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int r = 0; r < 4; ++r)
                         wbits |= philox::keep_byte_lanes(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
                 }
-                keepm = 0;
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t w = __shfl_sync(0xffffffffu, wbits, (lane & ~7) | s);
-                    keepm |= ((w >> sub) & 0x01010101u) << s;
-                }
+                keepm = philox::transpose_keep_bits(wbits, lane);
             }
             uint32_t pw[16], dw[16];
 #pragma unroll
@@ -294,9 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float pv = ex2(fmaf(__uint_as_float(rs[x + y]), scale_log2, -lv[y]));
                     if (diag && (qg0 + x + y) < kr) pv = 0.f;  // query before key: masked
                     if constexpr (Drop) {
-                        const bool keep = (keepm >> (x + y)) & 1u;
-                        pp[y] = keep ? pv : 0.f;
-                        dd[y] = pv * ((keep ? dp.keep_scale * __uint_as_float(rp[x + y]) : 0.f) - dvv[y]);
+                        // kept weight p~ = keep ? p : 0; dS / keep_scale = p~ dP - p Delta'
+                        pp[y] = (keepm >> (x + y)) & 1u ? pv : 0.f;
+                        dd[y] = fmaf(pp[y], __uint_as_float(rp[x + y]), -pv * dvv[y]);
                     } else {
                         pp[y] = pv;
                         dd[y] = pv * (__uint_as_float(rp[x + y]) - dvv[y]);
@@ -335,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int t = kt * kBK + kr;
             const uint32_t src = half == 0 ? tdK : tdV;
-            const float mul = half == 0 ? scale : (Drop ? dp.keep_scale : 1.f);
+            const float mul = Drop ? (half == 0 ? scale : 1.f) * dp.keep_scale : (half == 0 ? scale : 1.f);
             const TStrides so = half == 0 ? sdk : sdv;
             __nv_bfloat16 *out = (half == 0 ? dk : dv) + (long long)bb * so.b + (long long)hh * so.h +
                                  (long long)t * so.t;

@@ -55,9 +55,12 @@
 //
 // With attention dropout (Drop) the keep bit of (query i, key j) is the one
 // the forward drew (philox.cuh): the eight lanes holding keys 8g .. 8g+7 each
-// draw the bits of four queries for all eight keys and trade them with
-// shuffles; P^T in TMEM keeps only the kept weights (dV is scaled by the keep
-// scale at the end) and dS^T = P^T (keep_scale M dP^T - Delta).
+// load (from a kept mask) or draw the bits of four queries for all eight keys
+// and trade them in a three-stage shuffle butterfly; P^T in TMEM keeps only the kept weights (dV is scaled by the keep
+// scale at the end), and the kernel forms dS^T / keep_scale =
+// P^T (M dP^T - Delta / keep_scale) with Delta / keep_scale from the prep
+// kernel, so the keep scale enters once per output element (dK here, dQ in
+// the post kernel) instead of once per weight.
 //
 // TMEM columns: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D),
 // dQ [256+2D, 256+3D), P^T (bf16 pairs) [256+3D, 256+3D+64).
@@ -119,8 +122,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
                                                        const float *__restrict__ lse,
                                                        float *__restrict__ lse2,
                                                        float *__restrict__ delta,
-                                                       float *__restrict__ dq_acc, int T, int Tpad,
-                                                       int BH, int H, TStrides so, TStrides sdo) {
+                                                       float *__restrict__ dq_acc, float dscale, int T,
+                                                       int Tpad, int BH, int H, TStrides so, TStrides sdo) {
     constexpr int kTpr = D / 8;           // threads per row (a power of two dividing 32)
     constexpr int kRows = 256 / kTpr;     // rows per block
     grid_dep_wait();
@@ -152,7 +155,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
         for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (c == 0) {
             const size_t prow = (size_t)bh * Tpad + t;
-            delta[prow] = live ? acc : 0.f;
+            delta[prow] = live ? acc * dscale : 0.f;
             lse2[prow] = live ? lse[row] * kLog2e : INFINITY;
         }
     }
@@ -186,6 +189,12 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float4 *__restrict_
         *reinterpret_cast<uint4 *>(dq + hb * sdq.b + hh * sdq.h + (long long)t * sdq.t + 8 * c) = r;
     }
 }
+
+// With dropout the main kernels compute dS / keep_scale (the keep scale is
+// taken out of the per-weight arithmetic): the prep kernel stores
+// Delta / keep_scale, and dK and dQ take keep_scale in their output scale.
+inline float delta_scale(const Shape &s) { return s.dropout ? 1.f / s.drop.keep_scale : 1.f; }
+inline float dq_scale(const Shape &s) { return s.dropout ? s.scale * s.drop.keep_scale : s.scale; }
 
 // The (token blocks, heads) grid of the prep and post kernels.
 template <int D>
@@ -478,12 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int r = 0; r < 4; ++r)
                             wbits |= philox::keep_byte_lanes(dp, ib + 8u * r, jg, (uint32_t)bh) << (8 * r);
                     }
-                    keepm = 0;
-#pragma unroll
-                    for (int s = 0; s < 8; ++s) {
-                        const uint32_t w = __shfl_sync(0xffffffffu, wbits, (lane & ~7) | s);
-                        keepm |= ((w >> sub) & 0x01010101u) << s;
-                    }
+                    keepm = philox::transpose_keep_bits(wbits, lane);
                 }
                 uint32_t pw[16], dw[16];
 #pragma unroll
@@ -498,9 +502,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float pv = ex2(fmaf(__uint_as_float(rs[x + y]), scale_log2, -lv[y]));
                         if (diag && (q0 + x + y) < kr) pv = 0.f;  // query before key: masked
                         if constexpr (Drop) {
-                            const bool keep = (keepm >> (x + y)) & 1u;
-                            pp[y] = keep ? pv : 0.f;
-                            dd[y] = pv * ((keep ? dp.keep_scale * __uint_as_float(rp[x + y]) : 0.f) - dvv[y]);
+                            // kept weight p~ = keep ? p : 0; dS / keep_scale = p~ dP - p Delta'
+                            pp[y] = (keepm >> (x + y)) & 1u ? pv : 0.f;
+                            dd[y] = fmaf(pp[y], __uint_as_float(rp[x + y]), -pv * dvv[y]);
                         } else {
                             pp[y] = pv;
                             dd[y] = pv * (__uint_as_float(rp[x + y]) - dvv[y]);
@@ -599,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const uint32_t src = which == 0 ? tdK : tdV;
-                const float mul = which == 0 ? scale : (Drop ? dp.keep_scale : 1.f);
+                const float mul = Drop ? (which == 0 ? scale : 1.f) * dp.keep_scale : (which == 0 ? scale : 1.f);
                 const TStrides so = which == 0 ? sdk : sdv;
                 __nv_bfloat16 *out = (which == 0 ? dk : dv) + (long long)bb * so.b +
                                      (long long)hh * so.h + (long long)t * so.t;
@@ -685,7 +689,7 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if ((e = make_map(&mdq, dq_acc, BH, s.T, D, true, 32)) != cudaSuccess) return e;
 
     if ((e = launch_pdl(bwd_prep_kernel<D>, rows_grid<D>(Tpad, BH), dim3(256), 0, st, o, dO, lse, lse2,
-                        delta, dq_acc, s.T, Tpad, BH, s.H, str.o, str.dO)) != cudaSuccess)
+                        delta, dq_acc, delta_scale(s), s.T, Tpad, BH, s.H, str.o, str.dO)) != cudaSuccess)
         return e;
     li.kernels += 1;
 
@@ -713,7 +717,7 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if ((e = mark_main_end(li, st)) != cudaSuccess) return e;
 
     if ((e = launch_pdl(bwd_post_kernel<D>, rows_grid<D>(s.T, BH), dim3(256), 0, st,
-                        reinterpret_cast<const float4 *>(dq_acc), dq, s.scale, s.T, BH, s.H, str.dq)) !=
+                        reinterpret_cast<const float4 *>(dq_acc), dq, dq_scale(s), s.T, BH, s.H, str.dq)) !=
         cudaSuccess)
         return e;
     li.kernels += 1;
@@ -732,14 +736,14 @@ cudaError_t launch_bwd128(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const 
     const int Tpad = (s.T + kBT - 1) / kBT * kBT;
     cudaError_t e;
     if ((e = launch_pdl(bwd_prep_kernel<D>, rows_grid<D>(Tpad, BH), dim3(256), 0, st, o, dO, lse, lse2,
-                        delta, dq_acc, s.T, Tpad, BH, s.H, str.o, str.dO)) != cudaSuccess)
+                        delta, dq_acc, delta_scale(s), s.T, Tpad, BH, s.H, str.o, str.dO)) != cudaSuccess)
         return e;
     li.kernels += 1;
     if ((e = sm100_bwd128_main(q, k, v, dO, dk, dv, dq_acc, lse2, delta, s, str, err, st, li)) !=
         cudaSuccess)
         return e;
     if ((e = launch_pdl(bwd_post_kernel<D>, rows_grid<D>(s.T, BH), dim3(256), 0, st,
-                        reinterpret_cast<const float4 *>(dq_acc), dq, s.scale, s.T, BH, s.H, str.dq)) !=
+                        reinterpret_cast<const float4 *>(dq_acc), dq, dq_scale(s), s.T, BH, s.H, str.dq)) !=
         cudaSuccess)
         return e;
     li.kernels += 1;

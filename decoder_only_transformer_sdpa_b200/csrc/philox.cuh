@@ -106,6 +106,28 @@ __device__ __forceinline__ uint32_t keep_byte_lanes(const DropoutParams &dp, uin
     return bits;
 }
 
+// The backward holds keep bits by key: within each group of eight lanes (the
+// keys 8g .. 8g+7), lane s has in byte r the keep bits of those eight keys
+// for query (base + s + 8r).  Returns the lane's own key's bits: bit 8r + s =
+// keep bit of query (base + s + 8r) for key 8g + (lane & 7).  That is four
+// 8 x 8 bit-matrix transposes across the group at once, done in three
+// butterfly stages: exchange with lane ^ d (d = 4, 2, 1) and swap the
+// off-diagonal d x d blocks, a rotate by +-d bringing the partner's block
+// into place and a bit select keeping the lane's own.
+__device__ __forceinline__ uint32_t transpose_keep_bits(uint32_t x, int lane) {
+#pragma unroll
+    for (int st = 0; st < 3; ++st) {
+        const int d = 4 >> st;
+        const uint32_t m = st == 0 ? 0x0F0F0F0Fu : (st == 1 ? 0x33333333u : 0x55555555u);
+        const uint32_t t = __shfl_xor_sync(0xffffffffu, x, d);
+        const bool lo = (lane & d) == 0;
+        const uint32_t u = __funnelshift_l(t, t, lo ? d : 32 - d);  // rotate left
+        const uint32_t own = lo ? m : ~m;
+        x = (x & own) | (u & ~own);
+    }
+    return x;
+}
+
 // Offset of the kept byte of query i, key group g, head bh.
 __device__ __forceinline__ size_t mask_at(const DropoutParams &dp, uint32_t bh, uint32_t g, uint32_t i) {
     return ((size_t)bh * dp.mask_ld + i) * (dp.mask_ld >> 3) + g;
