@@ -31,6 +31,7 @@
 #include "sm100.cuh"
 
 #include <cudaTypedefs.h>
+#include <type_traits>
 
 namespace attn {
 namespace {
@@ -277,31 +278,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 keepm = philox::transpose_keep_bits(wbits, lane);
             }
             uint32_t pw[16], dw[16];
+            const uint64_t sc2 = f2pack(scale_log2, scale_log2);
+            // lse2 and delta hold -lse * log2(e) and -Delta' (prep kernel); the
+            // arithmetic runs on float32 pairs, and only the diagonal sub-tile
+            // takes the per-weight causal test.
+            auto elementwise = [&](auto diag_c) {
+                constexpr bool kDiag = decltype(diag_c)::value;
 #pragma unroll
-            for (int x = 0; x < 32; x += 4) {
-                const float4 l4 = ld_shared_f4(lse_addr + (q0 + x) * 4);
-                const float4 d4 = ld_shared_f4(dl_addr + (q0 + x) * 4);
-                const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
-                float pp[4], dd[4];
+                for (int x = 0; x < 32; x += 4) {
+                    const float4 l4 = ld_shared_f4(lse_addr + (q0 + x) * 4);
+                    const float4 d4 = ld_shared_f4(dl_addr + (q0 + x) * 4);
 #pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    float pv = ex2(fmaf(__uint_as_float(rs[x + y]), scale_log2, -lv[y]));
-                    if (diag && (qg0 + x + y) < kr) pv = 0.f;  // query before key: masked
-                    if constexpr (Drop) {
-                        // kept weight p~ = keep ? p : 0; dS / keep_scale = p~ dP - p Delta'
-                        pp[y] = (keepm >> (x + y)) & 1u ? pv : 0.f;
-                        dd[y] = fmaf(pp[y], __uint_as_float(rp[x + y]), -pv * dvv[y]);
-                    } else {
-                        pp[y] = pv;
-                        dd[y] = pv * (__uint_as_float(rp[x + y]) - dvv[y]);
+                    for (int h = 0; h < 2; ++h) {
+                        const int e = x + 2 * h;
+                        const uint64_t nl = h ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y);
+                        const uint64_t nd = h ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y);
+                        const float2 t =
+                            f2unpack(ffma2(f2pack(__uint_as_float(rs[e]), __uint_as_float(rs[e + 1])), sc2, nl));
+                        float p0 = ex2(t.x), p1 = ex2(t.y);
+                        if constexpr (kDiag) {  // query before key: masked
+                            if (qg0 + e < kr) p0 = 0.f;
+                            if (qg0 + e + 1 < kr) p1 = 0.f;
+                        }
+                        const uint64_t rp2 = f2pack(__uint_as_float(rp[e]), __uint_as_float(rp[e + 1]));
+                        float2 dd;
+                        if constexpr (Drop) {
+                            // kept weight p~ = keep ? p : 0; dS / keep_scale = p~ dP - p Delta'
+                            const float k0 = (keepm >> e) & 1u ? p0 : 0.f;
+                            const float k1 = (keepm >> (e + 1)) & 1u ? p1 : 0.f;
+                            dd = f2unpack(ffma2(f2pack(p0, p1), nd, fmul2(f2pack(k0, k1), rp2)));
+                            pw[e / 2] = pack_bf16x2(k0, k1);
+                        } else {
+                            dd = f2unpack(fmul2(f2pack(p0, p1), fadd2(rp2, nd)));
+                            pw[e / 2] = pack_bf16x2(p0, p1);
+                        }
+                        dw[e / 2] = pack_bf16x2(dd.x, dd.y);
                     }
                 }
-                pw[x / 2] = pack_bf16x2(pp[0], pp[1]);
-                pw[x / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
-                dw[x / 2] = pack_bf16x2(dd[0], dd[1]);
-                dw[x / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
-            }
+            };
+            if (diag)
+                elementwise(std::true_type{});
+            else
+                elementwise(std::false_type{});
             // P^T in TMEM is free once dV of the previous sub-tile completed;
             // this dS^T buffer once dK / dQ^T of two sub-tiles ago completed.
             bool w = true;

@@ -13,9 +13,10 @@
 //   dK_j  = scale sum_{i>=j} dS_ij q_i,   dQ_i = scale sum_{j<=i} dS_ij k_j
 //
 // Three launches on the caller's stream:
-//   prep   Delta_i and lse_i * log2(e) into tile-padded float32 arrays (pad rows
-//          get Delta = 0 and lse = +inf, so they contribute exactly 0), and the
-//          float32 dQ accumulator zeroed;
+//   prep   -Delta_i and -lse_i * log2(e) into tile-padded float32 arrays
+//          (negated, so that the main kernels add them: pad rows get 0 and
+//          -inf and contribute exactly 0), and the float32 dQ accumulator
+//          zeroed;
 //   main   one CTA per (128-row key tile j, head), looping over the query
 //          tiles i >= j (all query tiles without the mask, where keys past T
 //          are zero rows of K and V and so add nothing to dQ); dK_j and dV_j
@@ -33,8 +34,10 @@
 //   warp 3      tcgen05 issuer of dV, dK and dQ
 //   warps 4..11 softmax gradient, two warps per TMEM lane quadrant (one per
 //               64-query half): per key row (TMEM lane) P^T = exp2(S^T - lse),
-//               dS^T = P^T (dP^T - Delta); P^T to TMEM (bf16), dS^T to shared
-//               memory (bf16, double buffered)
+//               dS^T = P^T (dP^T - Delta), in packed float32 pairs (two queries
+//               per instruction); only the diagonal tile runs the causal test;
+//               P^T to TMEM (bf16), dS^T to shared memory (bf16, double
+//               buffered)
 //   warps 12..15 dQ drain: TMEM -> swizzled shared staging -> TMA reduce-add;
 //               at the end of each item the dK and dV epilogue, so that the
 //               softmax-gradient warps go straight on to the next item
@@ -68,6 +71,7 @@
 #include "sm100.cuh"
 
 #include <cudaTypedefs.h>
+#include <type_traits>
 
 namespace attn {
 namespace {
@@ -155,8 +159,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16 *__re
         for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (c == 0) {
             const size_t prow = (size_t)bh * Tpad + t;
-            delta[prow] = live ? acc * dscale : 0.f;
-            lse2[prow] = live ? lse[row] * kLog2e : INFINITY;
+            delta[prow] = live ? -(acc * dscale) : 0.f;
+            lse2[prow] = live ? -(lse[row] * kLog2e) : -INFINITY;
         }
     }
 }
@@ -192,7 +196,7 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float4 *__restrict_
 
 // With dropout the main kernels compute dS / keep_scale (the keep scale is
 // taken out of the per-weight arithmetic): the prep kernel stores
-// Delta / keep_scale, and dK and dQ take keep_scale in their output scale.
+// -Delta / keep_scale, and dK and dQ take keep_scale in their output scale.
 inline float delta_scale(const Shape &s) { return s.dropout ? 1.f / s.drop.keep_scale : 1.f; }
 inline float dq_scale(const Shape &s) { return s.dropout ? s.scale * s.drop.keep_scale : s.scale; }
 
@@ -490,31 +494,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                     keepm = philox::transpose_keep_bits(wbits, lane);
                 }
                 uint32_t pw[16], dw[16];
+                const uint64_t sc2 = f2pack(scale_log2, scale_log2);
+                // lse2 and delta hold -lse * log2(e) and -Delta' (prep kernel)
+                auto elementwise = [&](auto diag_c) {
+                    constexpr bool kDiag = decltype(diag_c)::value;
 #pragma unroll
-                for (int x = 0; x < 32; x += 4) {
-                    const float4 l4 = ld_shared_f4(lse_addr + (q0 + x) * 4);
-                    const float4 d4 = ld_shared_f4(dl_addr + (q0 + x) * 4);
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pp[4], dd[4];
+                    for (int x = 0; x < 32; x += 4) {
+                        const float4 l4 = ld_shared_f4(lse_addr + (q0 + x) * 4);
+                        const float4 d4 = ld_shared_f4(dl_addr + (q0 + x) * 4);
 #pragma unroll
-                    for (int y = 0; y < 4; ++y) {
-                        float pv = ex2(fmaf(__uint_as_float(rs[x + y]), scale_log2, -lv[y]));
-                        if (diag && (q0 + x + y) < kr) pv = 0.f;  // query before key: masked
-                        if constexpr (Drop) {
-                            // kept weight p~ = keep ? p : 0; dS / keep_scale = p~ dP - p Delta'
-                            pp[y] = (keepm >> (x + y)) & 1u ? pv : 0.f;
-                            dd[y] = fmaf(pp[y], __uint_as_float(rp[x + y]), -pv * dvv[y]);
-                        } else {
-                            pp[y] = pv;
-                            dd[y] = pv * (__uint_as_float(rp[x + y]) - dvv[y]);
+                        for (int h = 0; h < 2; ++h) {
+                            const int e = x + 2 * h;
+                            const uint64_t nl = h ? f2pack(l4.z, l4.w) : f2pack(l4.x, l4.y);
+                            const uint64_t nd = h ? f2pack(d4.z, d4.w) : f2pack(d4.x, d4.y);
+                            const float2 t = f2unpack(
+                                ffma2(f2pack(__uint_as_float(rs[e]), __uint_as_float(rs[e + 1])), sc2, nl));
+                            float p0 = ex2(t.x), p1 = ex2(t.y);
+                            if constexpr (kDiag) {  // query before key: masked
+                                if (q0 + e < kr) p0 = 0.f;
+                                if (q0 + e + 1 < kr) p1 = 0.f;
+                            }
+                            const uint64_t rp2 = f2pack(__uint_as_float(rp[e]), __uint_as_float(rp[e + 1]));
+                            float2 dd;
+                            if constexpr (Drop) {
+                                // kept weight p~ = keep ? p : 0; dS / keep_scale = p~ dP - p Delta'
+                                const float k0 = (keepm >> e) & 1u ? p0 : 0.f;
+                                const float k1 = (keepm >> (e + 1)) & 1u ? p1 : 0.f;
+                                dd = f2unpack(ffma2(f2pack(p0, p1), nd, fmul2(f2pack(k0, k1), rp2)));
+                                pw[e / 2] = pack_bf16x2(k0, k1);
+                            } else {
+                                dd = f2unpack(fmul2(f2pack(p0, p1), fadd2(rp2, nd)));
+                                pw[e / 2] = pack_bf16x2(p0, p1);
+                            }
+                            dw[e / 2] = pack_bf16x2(dd.x, dd.y);
                         }
                     }
-                    pw[x / 2] = pack_bf16x2(pp[0], pp[1]);
-                    pw[x / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
-                    dw[x / 2] = pack_bf16x2(dd[0], dd[1]);
-                    dw[x / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
-                }
+                };
+                if (diag)
+                    elementwise(std::true_type{});
+                else
+                    elementwise(std::false_type{});
                 if (c == 0) {
                     // P^T in TMEM is free once dV of the previous tile completed;
                     // this dS^T buffer once dK/dQ of two tiles ago completed.

@@ -597,8 +597,11 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
                 // All exponentials first (packed bf16 pairs), then wait for the
                 // previous PV to release the P region: the wait sits at the end
                 // of the tile, where the previous PV has had the most time.
+                // Exponent arguments and the two running row sums (even and odd
+                // keys) are float32 pairs, one packed instruction per key pair.
                 uint32_t pk[kBN / 2];
-                float la = 0.f, lb = 0.f;
+                const uint64_t sc2 = f2pack(scale_log2, scale_log2), nm2 = f2pack(neg_m, neg_m);
+                uint64_t l2 = f2pack(0.f, 0.f);
                 if constexpr (Drop) {
                     // Word q of keep bits covers keys 32q .. 32q+31 (bit e = key
                     // 32q + e); its left shifts by 0..7 put every key's bit in the
@@ -612,24 +615,25 @@ __global__ void __launch_bounds__(kThreads, D > 64 ? 1 : 2)
 #pragma unroll
                         for (int y = 0; y < 16; ++y) {
                             const int x = 16 * q + y;
-                            const float p0 = ex2(fmaf(s[2 * x], scale_log2, neg_m));
-                            const float p1 = ex2(fmaf(s[2 * x + 1], scale_log2, neg_m));
-                            la += p0;
-                            lb += p1;
+                            const float2 t = f2unpack(ffma2(f2pack(s[2 * x], s[2 * x + 1]), sc2, nm2));
+                            const float p0 = ex2(t.x);
+                            const float p1 = ex2(t.y);
+                            l2 = fadd2(l2, f2pack(p0, p1));
                             pk[x] = pack_bf16x2(p0, p1) & keep_pair_mask(sh, 2 * y);
                         }
                     }
                 } else {
 #pragma unroll
                     for (int x = 0; x < kBN / 2; ++x) {
-                        const float p0 = ex2(fmaf(s[2 * x], scale_log2, neg_m));
-                        const float p1 = ex2(fmaf(s[2 * x + 1], scale_log2, neg_m));
-                        la += p0;
-                        lb += p1;
+                        const float2 t = f2unpack(ffma2(f2pack(s[2 * x], s[2 * x + 1]), sc2, nm2));
+                        const float p0 = ex2(t.x);
+                        const float p1 = ex2(t.y);
+                        l2 = fadd2(l2, f2pack(p0, p1));
                         pk[x] = pack_bf16x2(p0, p1);
                     }
                 }
-                l += la + lb;
+                const float2 lab = f2unpack(l2);
+                l += lab.x + lab.y;
                 if (kDeferEpilogue && j == 0 && pn >= 0) {
                     // The previous item's epilogue, off the item boundary: its
                     // last PV has had this tile's exponentials to complete (its
