@@ -464,7 +464,8 @@ ATTN_API int attn_device_error(cudaStream_t stream) {
         const int zero = 0;
         if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
             return ATTN_ERR_CUDA;
-        return h == kErrBounds ? ATTN_ERR_DEVICE_CHECK : ATTN_ERR_TIMEOUT;
+        if (h == kErrBounds) return ATTN_ERR_DEVICE_CHECK;
+        return h == kErrLayout ? ATTN_ERR_CUDA : ATTN_ERR_TIMEOUT;
     }
     return ATTN_OK;
 }

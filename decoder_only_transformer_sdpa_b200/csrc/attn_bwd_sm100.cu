@@ -26,11 +26,13 @@
 //   post   dQ = scale * accumulator, rounded to bf16.
 //
 // Main kernel, sixteen warps in four warpgroups:
-//   warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse_i, Delta_i per tile
-//               into a 2-stage ring (a stage is released after dK_i, since
-//               dQ_i reads neither Q nor dO)
+//   warp 0      TMA producer: K_j (and V_j) once; Q_i, dO_i (and lse_i,
+//               Delta_i) per tile into a 2-stage ring (a stage is released
+//               after dK_i, since dQ_i reads neither Q nor dO); without the
+//               causal mask and dropout the ring has 3 stages (BwdSmem)
 //   warp 1      tcgen05 issuer of S^T and dP^T, TMEM owner
-//   warp 2      idle (it completes the first warpgroup)
+//   warp 2      in the 3-stage layout, V_j and lse_i, Delta_i (their own
+//               2-slot ring); idle otherwise
 //   warp 3      tcgen05 issuer of dV, dK and dQ
 //   warps 4..11 softmax gradient, two warps per TMEM lane quadrant (one per
 //               64-query half): per key row (TMEM lane) P^T = exp2(S^T - lse),
@@ -71,6 +73,7 @@
 #include "sm100.cuh"
 
 #include <cudaTypedefs.h>
+#include <cstddef>
 #include <type_traits>
 
 namespace attn {
@@ -88,29 +91,49 @@ constexpr int kRegsIssue = 56;    // producer / MMA warpgroup after the hand-ove
 constexpr int kRegsEw = 176;      // softmax-gradient warpgroups
 constexpr int kRegsDrain = 104;   // drain warpgroup
 static_assert(kRegsIssue + kRegsDrain + 2 * kRegsEw == 4 * kRegsLaunch, "the register split must add up");
-constexpr int kQStages = 2;       // Q / dO / lse / Delta ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D>
+// Two layouts.  Under the causal mask (short items, 4.5 query tiles on
+// average at T = 1024), and with dropout (whose longer softmax-gradient work
+// sets the tile period): a 2-stage Q / dO / lse / Delta ring and K, V double
+// buffered across items.  Without the mask and without dropout (every item
+// runs over all query tiles, and the ring's reload sits on the tile period):
+// a 3-stage Q / dO ring, paid for by a single V buffer (its last reader is the
+// item's last dP^T) and by lse / Delta in a 2-slot ring of their own, loaded
+// with V by warp 2.
+template <int D, bool R3>
 struct BwdSmem {
     static constexpr int kTileBytes = kBT * D * 2;
-    alignas(1024) __nv_bfloat16 q[kQStages][kBT * D];
-    alignas(1024) __nv_bfloat16 dO[kQStages][kBT * D];
+    static constexpr int kQS = R3 ? 3 : 2;    // Q / dO stages
+    static constexpr int kLS = R3 ? 2 : kQS;  // lse / Delta slots (the Q / dO stages without R3)
+    static constexpr int kVB = R3 ? 1 : 2;    // V buffers
+    alignas(1024) __nv_bfloat16 q[kQS][kBT * D];
+    alignas(1024) __nv_bfloat16 dO[kQS][kBT * D];
     alignas(1024) __nv_bfloat16 k[2][kBT * D];   // double buffered across work items
-    alignas(1024) __nv_bfloat16 v[2][kBT * D];
+    alignas(1024) __nv_bfloat16 v[kVB][kBT * D];
     // dS^T, [buffer][query half][key row][64 queries], 128-byte swizzled rows
     alignas(1024) __nv_bfloat16 ds[2][2][kBT * 64];
     // dQ staging for the TMA reduce: one 32-column box [row][32 floats], swizzled
     alignas(1024) float stage[kBT * 32];
-    alignas(16) float lse2[kQStages][kBT];
-    alignas(16) float delta[kQStages][kBT];
-    uint64_t kv_full[2], kv_empty[2], qdo_full[kQStages], qdo_empty[kQStages];
+    alignas(16) float lse2[kLS][kBT];
+    alignas(16) float delta[kLS][kBT];
+    uint64_t kv_full[2], kv_empty[2], qdo_full[kQS], qdo_empty[kQS];
+    uint64_t v_full, v_empty, ld_full[kLS], ld_empty[kLS];  // the R3 layout's V and lse / Delta
     uint64_t sdp_full, sdp_free, p_ready[2], ds_ready[2], p_free, ds_free[2];
     uint64_t dq_full, dq_free, acc_done, acc_free, drain;
     uint32_t tmem_slot;
     int abort;
 };
+
+// Bytes of a layout in use (without the tail padding to its alignment).
+template <int D, bool R3>
+struct SmemUsed {
+    using S = BwdSmem<D, R3>;
+    static constexpr size_t value = offsetof(S, abort) + sizeof(int);
+};
+template <int D, bool R3>
+constexpr size_t kSmemUsed = SmemUsed<D, R3>::value;
 
 // ------------------------------------------------------------------ prep
 
@@ -225,7 +248,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __nv_bfloat16 *__restrict__ dv, const TStrides sdk, const TStrides sdv,
                     int T, int Tpad, int H, int BH, int nt, float scale_log2, float scale,
                     const DropoutParams dp, int *err) {
-    using Smem = BwdSmem<D>;
+    constexpr bool R3 = !Causal && !Drop;
+    using Smem = BwdSmem<D, R3>;
+    constexpr int kQStages = Smem::kQS, kLStages = Smem::kLS;
     constexpr int kRowBytes = D * 2;
     constexpr uint32_t kSwz = (D == 64) ? kSwizzle128B : kSwizzle64B;
     constexpr uint32_t kAtom = 8 * kRowBytes;
@@ -234,6 +259,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                          ~uintptr_t(1023));
     volatile int *abort = &sm.abort;
+    if constexpr (R3) {
+        // The launch allocates only the padding the layout leaves below the
+        // per-block limit: a base that needs more leaves before touching
+        // shared memory and reports it.
+        uint32_t dyn;
+        asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+        const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+        if (pad + (uint32_t)kSmemUsed<D, R3> > dyn) {
+            if (threadIdx.x == 0) atomicExch(err, kErrLayout);
+            return;
+        }
+    }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = (int)gridDim.x, cta = (int)blockIdx.x;
@@ -247,6 +284,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kQStages; ++s) {
             mbar_init(&sm.qdo_full[s], 1);
             mbar_init(&sm.qdo_empty[s], 1);
+        }
+        if constexpr (R3) {
+            mbar_init(&sm.v_full, 1);
+            mbar_init(&sm.v_empty, 1);  // the score stream, after the item's last dP^T
+            for (int s = 0; s < kLStages; ++s) {
+                mbar_init(&sm.ld_full[s], 1);
+                mbar_init(&sm.ld_empty[s], kEwThreads);
+            }
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.p_ready[s], kEwThreads);
@@ -302,20 +347,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             ATTN_DCHECK(kt >= 0 && kt < nt && bh >= 0 && bh < BH && kt * kBT < T, err);
             if (n >= 2 && !(ok = mbar_wait_warp(&sm.kv_empty[kb], (uint32_t)((n >> 1) - 1) & 1u, err, abort)))
                 break;
-            mbar_arrive_expect_tx_e(&sm.kv_full[kb], 2 * Smem::kTileBytes);
-            tma_load_4d_e(sm.k[kb], &tk, &sm.kv_full[kb], 0, kt * kBT, hh, bb);
-            tma_load_4d_e(sm.v[kb], &tv, &sm.kv_full[kb], 0, kt * kBT, hh, bb);
+            if constexpr (R3) {  // V comes from warp 2
+                mbar_arrive_expect_tx_e(&sm.kv_full[kb], Smem::kTileBytes);
+                tma_load_4d_e(sm.k[kb], &tk, &sm.kv_full[kb], 0, kt * kBT, hh, bb);
+            } else {
+                mbar_arrive_expect_tx_e(&sm.kv_full[kb], 2 * Smem::kTileBytes);
+                tma_load_4d_e(sm.k[kb], &tk, &sm.kv_full[kb], 0, kt * kBT, hh, bb);
+                tma_load_4d_e(sm.v[kb], &tv, &sm.kv_full[kb], 0, kt * kBT, hh, bb);
+            }
             n_items = n + 1;
             for (int i = q_first; i < nt; ++i, ++g) {
                 const int st = g % kQStages;
                 if (!(ok = mbar_wait_warp(&sm.qdo_empty[st], (uint32_t)((g / kQStages) & 1) ^ 1u, err, abort))) break;
-                mbar_arrive_expect_tx_e(&sm.qdo_full[st], 2 * Smem::kTileBytes + 2 * kBT * 4);
+                mbar_arrive_expect_tx_e(&sm.qdo_full[st], 2 * Smem::kTileBytes + (R3 ? 0 : 2 * kBT * 4));
                 tma_load_4d_e(sm.q[st], &tq, &sm.qdo_full[st], 0, i * kBT, hh, bb);
                 tma_load_4d_e(sm.dO[st], &tdo, &sm.qdo_full[st], 0, i * kBT, hh, bb);
-                const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
-                ATTN_DCHECK(prow + kBT <= (size_t)BH * Tpad && i * kBT < T, err);
-                bulk_load_e(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
-                bulk_load_e(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
+                if constexpr (!R3) {  // lse and Delta travel with the stage
+                    const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
+                    ATTN_DCHECK(prow + kBT <= (size_t)BH * Tpad && i * kBT < T, err);
+                    bulk_load_e(sm.lse2[st], lse2 + prow, kBT * 4, &sm.qdo_full[st]);
+                    bulk_load_e(sm.delta[st], delta + prow, kBT * 4, &sm.qdo_full[st]);
+                }
             }
         }
         // The last loads issued have landed before the CTA leaves.
@@ -323,6 +375,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (uint32_t m = 0; m < kWaitLimit && !mbar_try_wait(&sm.qdo_full[x % kQStages], (uint32_t)(x / kQStages) & 1u); ++m) {}
         for (int n = (n_items > 2 ? n_items - 2 : 0); n < n_items; ++n)
             for (uint32_t m = 0; m < kWaitLimit && !mbar_try_wait(&sm.kv_full[n & 1], (uint32_t)(n >> 1) & 1u); ++m) {}
+    } else if (warp == 2) {
+        if constexpr (R3) {
+            // ------------------------------------------------ second loader (R3
+            // layout): V of each item (single buffer, once the score stream is
+            // done with the previous item) and the lse / Delta rows of each
+            // tile into their 2-slot ring (once the softmax-gradient warps are
+            // done with the tile two back), so the Q / dO producer never waits
+            // on either.
+            if (lane == 0) prefetch_tensormap(&tv);
+            __syncwarp();
+            int g = 0, n_v = 0;
+            bool ok = true;
+            for (int n = 0; ok; ++n) {
+                const int w = item_of(cta, n, G, W);
+                if (w < 0) break;
+                const int kt = w / BH, bh = w % BH;
+                if (n >= 1 && !(ok = mbar_wait_warp(&sm.v_empty, (uint32_t)(n - 1) & 1u, err, abort))) break;
+                mbar_arrive_expect_tx_e(&sm.v_full, Smem::kTileBytes);
+                tma_load_4d_e(sm.v[0], &tv, &sm.v_full, 0, kt * kBT, bh % H, bh / H);
+                n_v = n + 1;
+                for (int i = 0; i < nt; ++i, ++g) {
+                    const int sl = g % kLStages;
+                    if (g >= kLStages &&
+                        !(ok = mbar_wait_warp(&sm.ld_empty[sl], (uint32_t)(g / kLStages - 1) & 1u, err, abort)))
+                        break;
+                    const size_t prow = (size_t)bh * Tpad + (size_t)i * kBT;
+                    ATTN_DCHECK(prow + kBT <= (size_t)BH * Tpad && i * kBT < T, err);
+                    mbar_arrive_expect_tx_e(&sm.ld_full[sl], 2 * kBT * 4);
+                    bulk_load_e(sm.lse2[sl], lse2 + prow, kBT * 4, &sm.ld_full[sl]);
+                    bulk_load_e(sm.delta[sl], delta + prow, kBT * 4, &sm.ld_full[sl]);
+                }
+            }
+            // The last loads issued have landed before the CTA leaves.
+            for (int x = (g > kLStages ? g - kLStages : 0); x < g; ++x)
+                mbar_wait_drain(&sm.ld_full[x % kLStages], (uint32_t)(x / kLStages) & 1u);
+            if (n_v > 0) mbar_wait_drain(&sm.v_full, (uint32_t)(n_v - 1) & 1u);
+        }
     } else if (warp == 1 || warp == 3) {
         // ------------------------------------------------ tcgen05 issuers (whole
         // warp, one elected lane issues).  Two independent streams share the
@@ -346,9 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (warp == 1) {
                 // ---- score stream
                 if (!(ok = mbar_wait_warp(&sm.kv_full[kb], (uint32_t)(n >> 1) & 1u, err, abort))) break;
+                if (R3 && !(ok = mbar_wait_warp(&sm.v_full, (uint32_t)n & 1u, err, abort))) break;
                 // K and V as K-major operands.
                 const uint64_t kd_k = smem_desc(smem_u32(sm.k[kb]), 16, kAtom, kSwz);
-                const uint64_t vd_k = smem_desc(smem_u32(sm.v[kb]), 16, kAtom, kSwz);
+                const uint64_t vd_k = smem_desc(smem_u32(sm.v[R3 ? 0 : kb]), 16, kAtom, kSwz);
                 for (int idx = 0; idx < n_q; ++idx, ++g) {
                     const int st = g % kQStages;
                     if (!(ok = mbar_wait_warp(&sm.qdo_full[st], (uint32_t)(g / kQStages) & 1u, err, abort))) break;
@@ -368,7 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_commit_e(&sm.sdp_full);
                 }
                 if (!ok) break;
-                mma_commit_e(&sm.kv_empty[kb]);  // this stream's reads of the item's K, V
+                if constexpr (R3) mma_commit_e(&sm.v_empty);  // the item's reads of V
+                mma_commit_e(&sm.kv_empty[kb]);  // this stream's reads of the item's K (and V)
             } else {
                 // ---- gradient stream.  K needs no wait of its own: the first
                 // tile's dS^T exists only after that tile's S^T, which waited
@@ -442,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int idx = 0; idx < n_q; ++idx) {
             const int g = g0 + idx;
             const int st = g % kQStages, b = g & 1;
+            const int sl = R3 ? g % kLStages : st;  // lse / Delta slot
             // With a kept dropout mask, this tile's keep bytes are loaded
             // before the wait for S^T, so their latency overlaps it: byte r of
             // kept[c] is keys 8 jg .. +7 of query ib + 8 r (as drawn below).
@@ -459,11 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            ok = mbar_wait_warp(&sm.sdp_full, (uint32_t)g & 1u, err, abort);
+            ok = (!R3 || mbar_wait_warp(&sm.ld_full[sl], (uint32_t)(g / kLStages) & 1u, err, abort)) &&
+                 mbar_wait_warp(&sm.sdp_full, (uint32_t)g & 1u, err, abort);
             if (!ok) break;
             tc_fence_after();
             const bool diag = Causal && (idx == 0);
-            const uint32_t lse_addr = smem_u32(sm.lse2[st]), dl_addr = smem_u32(sm.delta[st]);
+            const uint32_t lse_addr = smem_u32(sm.lse2[sl]), dl_addr = smem_u32(sm.delta[sl]);
             const uint32_t ds_row = smem_u32(sm.ds[b][half]) + (uint32_t)kr * 128;
             ATTN_DCHECK(kr < kBT && (kr + 1) * 128 <= (int)sizeof(sm.ds[0][0]), err);
 #pragma unroll
@@ -553,6 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok) break;
+            if constexpr (R3) mbar_arrive(&sm.ld_empty[sl]);  // this tile's lse / Delta are read
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
@@ -712,7 +806,19 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
         return e;
     li.kernels += 1;
 
-    const size_t smem = sizeof(BwdSmem<D>) + 1024;
+    // The layout plus the padding a 1024-byte alignment of the base may need;
+    // the R3 layout caps that at the per-block limit (the kernel checks the
+    // base it gets).
+    constexpr bool R3 = !Causal && !Drop;
+    size_t smem = sizeof(BwdSmem<D, R3>) + 1024;
+    if constexpr (R3) {
+        int smem_max = 0;
+        if ((e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+            return e;
+        smem = kSmemUsed<D, R3> + 1023;
+        if (smem > (size_t)smem_max) smem = (size_t)smem_max;
+        if (kSmemUsed<D, R3> > smem) return cudaErrorInvalidConfiguration;
+    }
     {
         // The setmaxnreg hand-over assumes the block holds 512 x 128
         // registers; any other build would make the increases wait forever.

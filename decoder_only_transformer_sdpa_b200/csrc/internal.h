@@ -23,6 +23,10 @@ constexpr int kErrTimeout = 1;
 // kErrBounds in the device error word and the kernel carries on (nothing
 // traps).  The release build compiles the checks away.
 constexpr int kErrBounds = 3;
+// A kernel whose tile layout leaves less alignment padding than its dynamic
+// shared-memory base needs records kErrLayout and leaves before touching
+// shared memory.
+constexpr int kErrLayout = 4;
 #ifdef ATTN_DEVICE_CHECKS
 #define ATTN_DCHECK(cond, err)                           \
     do {                                                 \

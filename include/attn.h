@@ -297,7 +297,9 @@ int attn_bwd_f32_ex(const float *q, const float *k, const float *v, const float 
  * ran out since the last call), ATTN_ERR_DEVICE_CHECK (the debug build
  * libattn_debug.so only: a kernel's bounds check on a tile coordinate, TMEM
  * column or shared-memory offset failed; the kernel records it and carries
- * on) or ATTN_ERR_CUDA (the sync itself failed). */
+ * on) or ATTN_ERR_CUDA (the sync itself failed, or a kernel found its dynamic
+ * shared memory placed too far from a 1024-byte boundary for its tile layout
+ * and left without computing). */
 int attn_device_error(cudaStream_t stream);
 
 /* Failure-path self test: enqueues one thread that waits on an in-kernel
