@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx_e(&sm.v_full, Smem::kTileBytes);
                 tma_load_4d_e(sm.v[0], &tv, &sm.v_full, 0, kt * kBT, bh % H, bh / H);
                 n_v = n + 1;
-                for (int i = 0; i < nt; ++i, ++g) {
+                for (int i = Causal ? kt : 0; i < nt; ++i, ++g) {  // the item's query tiles
                     const int sl = g % kLStages;
                     if (g >= kLStages &&
                         !(ok = mbar_wait_warp(&sm.ld_empty[sl], (uint32_t)(g / kLStages - 1) & 1u, err, abort)))
