@@ -132,13 +132,48 @@ def _torch():
 
 
 def _stream_handle(stream) -> int:
+    """The raw handle of `stream`, or of torch's current stream on the current
+    device (read without building a Stream object when torch offers that)."""
     torch = _torch()
     if stream is None:
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:
+            return int(raw(torch.cuda.current_device()))
         stream = torch.cuda.current_stream()
     return int(stream.cuda_stream)
 
 
+class _device:
+    """Makes `device` current for the call, switching only when it is not
+    (a plain torch.cuda.device() switches and restores every time)."""
+    __slots__ = ("idx", "prev")
+
+    def __init__(self, device):
+        self.idx = device.index
+
+    def __enter__(self):
+        torch = _torch()
+        cur = torch.cuda.current_device()
+        self.prev = None if cur == self.idx else cur
+        if self.prev is not None:
+            torch.cuda.set_device(self.idx)
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            _torch().cuda.set_device(self.prev)
+        return False
+
+
 def _check(t, name, dtype, shape=None):
+    """The tensor's device address, after checking that it is a contiguous
+    CUDA tensor of `dtype` (and `shape`); one combined test on the common
+    path, the specific error otherwise."""
+    try:
+        if t.is_cuda and t.dtype == dtype and (shape is None or t.shape == shape) and t.is_contiguous():
+            return t.data_ptr()
+    except AttributeError:
+        pass
     torch = _torch()
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -156,7 +191,8 @@ def _check(t, name, dtype, shape=None):
 def _shape4(q):
     if q.dim() != 4:
         raise ValueError("expected [B, H, T, D]")
-    return tuple(int(s) for s in q.shape)
+    B, H, T, D = q.shape
+    return B, H, T, D
 
 
 def _raise(status: int, where: str):
@@ -174,7 +210,7 @@ def _fwd(cfn, dtype, q, k, v, o, lse, scale, stream):
         lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
     ptrs = [_check(q, "q", dtype), _check(k, "k", dtype, q.shape), _check(v, "v", dtype, q.shape),
             _check(o, "o", dtype, q.shape), _check(lse, "lse", torch.float32, (B, H, T))]
-    with torch.cuda.device(q.device):
+    with _device(q.device):
         _raise(cfn(*ptrs, B, H, T, D, scale, _stream_handle(stream)), cfn.__name__)
     return o, lse
 
@@ -196,7 +232,7 @@ def _bwd(cfn, ws_fn, dtype, q, k, v, o, lse, dO, dq, dk, dv, scale, workspace, s
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
-    with torch.cuda.device(q.device):
+    with _device(q.device):
         _raise(cfn(*ptrs, B, H, T, D, scale, workspace.data_ptr(), ws_bytes, _stream_handle(stream)),
                cfn.__name__)
     return dq, dk, dv
@@ -234,7 +270,7 @@ def attn_bwd_noalloc(q, k, v, o, lse, dO, dq=None, dk=None, dv=None,
             _check(o, "o", bf, q.shape), _check(lse, "lse", torch.float32, (B, H, T)),
             _check(dO, "dO", bf, q.shape), _check(dq, "dq", bf, q.shape),
             _check(dk, "dk", bf, q.shape), _check(dv, "dv", bf, q.shape)]
-    with torch.cuda.device(q.device):
+    with _device(q.device):
         _raise(_lib.attn_bwd_noalloc(*ptrs, B, H, T, D, scale, _stream_handle(stream)),
                "attn_bwd_noalloc")
     return dq, dk, dv
@@ -321,7 +357,7 @@ def attn_fwd_strided(q, k, v, o=None, lse=None, scale: Optional[float] = None, s
             _check_view(v, "v", q.shape), _check_view(o, "o", q.shape),
             _check(lse, "lse", torch.float32, (B, H, T))]
     st = _strides_of(q, k, v, o)
-    with torch.cuda.device(q.device):
+    with _device(q.device):
         _raise(_lib.attn_fwd_strided(*ptrs, B, H, T, D, scale, st, _stream_handle(stream)),
                "attn_fwd_strided")
     return o, lse
@@ -347,7 +383,7 @@ def attn_bwd_strided(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Opti
             _check_view(dv, "dv", q.shape)]
     st = _strides_of(q, k, v, o, dO, dq, dk, dv)
     ws_bytes = workspace.numel() * workspace.element_size()
-    with torch.cuda.device(q.device):
+    with _device(q.device):
         _raise(_lib.attn_bwd_strided(*ptrs, B, H, T, D, scale, st, workspace.data_ptr(), ws_bytes,
                                      _stream_handle(stream)), "attn_bwd_strided")
     return dq, dk, dv
@@ -392,7 +428,7 @@ def attn_fwd_ex(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal
             _check(lse, "lse", torch.float32, (B, H, T))]
     st = None if _all_contiguous(q, k, v, o) else _strides_of(q, k, v, o)
     opts = _options(causal, dropout_p, seed, offset, dropout_mask)
-    with torch.cuda.device(q.device):
+    with _device(q.device):
         _raise(_lib.attn_fwd_ex(*ptrs, B, H, T, D, scale, st, ctypes.byref(opts),
                                 _stream_handle(stream)), "attn_fwd_ex")
     return o, lse
@@ -425,7 +461,7 @@ def attn_bwd_ex(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, scale: Optional[
     st = None if _all_contiguous(*views) else _strides_of(*views)
     opts = _options(causal, dropout_p, seed, offset, dropout_mask)
     ws_bytes = workspace.numel() * workspace.element_size()
-    with torch.cuda.device(q.device):
+    with _device(q.device):
         _raise(_lib.attn_bwd_ex(*ptrs, B, H, T, D, scale, st, ctypes.byref(opts),
                                 workspace.data_ptr(), ws_bytes, _stream_handle(stream)),
                "attn_bwd_ex")
@@ -468,7 +504,7 @@ def attn_decode(q, k, v, o=None, lse=None, scale: Optional[float] = None, stream
             _check_view(v, "v", (B, H, Tk, D)), _check_view(o, "o", (B, H, Tq, D)),
             _check(lse, "lse", torch.float32, (B, H, Tq))]
     st = None if _all_contiguous(q, k, v, o) else _strides_of(q, k, v, o)
-    with torch.cuda.device(q.device):
+    with _device(q.device):
         _raise(_lib.attn_decode(*ptrs, B, H, Tq, Tk, D, scale, st, _stream_handle(stream)),
                "attn_decode")
     return o, lse

@@ -472,8 +472,11 @@ cudaError_t launch128(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     if ((e = make_map_rows(&mdo, dO, s, str.dO, kBQ)) != cudaSuccess) return e;
     if ((e = make_map_dq(&mdq, dq_acc, BH, s.T)) != cudaSuccess) return e;
     const size_t smem = sizeof(Smem128) + 1024;
-    if ((e = cudaFuncSetAttribute(bwd128_main_kernel<Causal, Drop>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    static std::atomic<unsigned long long> smem_set{0};
+    if ((e = set_max_smem_once(reinterpret_cast<const void *>(bwd128_main_kernel<Causal, Drop>), smem, dev,
+                               smem_set)) != cudaSuccess)
         return e;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     if ((e = launch_pdl(bwd128_main_kernel<Causal, Drop>, dim3((unsigned)blocks), dim3(kThreads), smem,

@@ -830,8 +830,9 @@ cudaError_t launch_bwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
         }
         if (checked < 0) return cudaErrorInvalidConfiguration;
     }
-    if ((e = cudaFuncSetAttribute(bwd_main_kernel<D, Causal, Drop>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem)) != cudaSuccess)
+    static std::atomic<unsigned long long> smem_set{0};
+    if ((e = set_max_smem_once(reinterpret_cast<const void *>(bwd_main_kernel<D, Causal, Drop>), smem, dev,
+                               smem_set)) != cudaSuccess)
         return e;
     if ((e = mark_main_start(li, st)) != cudaSuccess) return e;
     if ((e = launch_pdl(bwd_main_kernel<D, Causal, Drop>, dim3((unsigned)blocks), dim3(kThreads), smem, st,

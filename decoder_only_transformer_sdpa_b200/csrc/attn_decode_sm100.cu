@@ -381,8 +381,9 @@ cudaError_t launch_decode(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const 
     if ((e = make_map_bf16(&mk, k, kv, str.k)) != cudaSuccess) return e;
     if ((e = make_map_bf16(&mv, v, kv, str.v)) != cudaSuccess) return e;
     const size_t smem = sizeof(DecSmem<D, NQ>) + 1024;
-    if ((e = cudaFuncSetAttribute(decode_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem)) != cudaSuccess)
+    static std::atomic<unsigned long long> smem_set{0};
+    if ((e = set_max_smem_once(reinterpret_cast<const void *>(decode_kernel<D, NQ>), smem, dev, smem_set)) !=
+        cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);

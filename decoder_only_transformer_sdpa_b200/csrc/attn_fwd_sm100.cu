@@ -723,8 +723,9 @@ cudaError_t launch_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __n
     if ((e = make_map_bf16(&mv, v, s, str.v)) != cudaSuccess) return e;
     if ((e = make_map_bf16(&mo, o, s, str.o)) != cudaSuccess) return e;
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
-    if ((e = cudaFuncSetAttribute(fwd_kernel<D, Causal, Drop>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem)) != cudaSuccess)
+    static std::atomic<unsigned long long> smem_set{0};
+    if ((e = set_max_smem_once(reinterpret_cast<const void *>(fwd_kernel<D, Causal, Drop>), smem, dev,
+                               smem_set)) != cudaSuccess)
         return e;
     if constexpr (D <= 64) {
         // The setmaxnreg hand-over assumes the block holds 256 x 128

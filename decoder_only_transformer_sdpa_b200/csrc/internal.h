@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "philox.cuh"
 
 namespace attn {
@@ -94,6 +96,18 @@ inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on device `dev`
+// once per call site: the attribute lasts for the process, so later calls on
+// a device whose bit is set in `done` skip the runtime call.
+inline cudaError_t set_max_smem_once(const void *kernel, size_t bytes, int dev,
+                                     std::atomic<unsigned long long> &done) {
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_relaxed);
+    return e;
 }
 
 // Records li.main_start / li.main_end (when armed) around a main kernel.
