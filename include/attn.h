@@ -90,9 +90,10 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              int B, int H, int T, int D, float scale, cudaStream_t stream);
 
 /* Bytes of device workspace attn_bwd needs: a float32 dQ accumulator
- * [B,H,T,D], then lse * log2(e) and Delta_i = <dO_i, O_i>, each [B*H] rows of
- * T rounded up to a multiple of 128 floats; each part 256-byte aligned.
- * 0 on a bad shape or unsupported D. */
+ * [B,H,T,D], then -lse * log2(e) and -Delta_i = -<dO_i, O_i> (with dropout,
+ * divided by the keep scale), each [B*H] rows of T rounded up to a multiple
+ * of 128 floats; each part 256-byte aligned.  0 on a bad shape or
+ * unsupported D. */
 size_t attn_bwd_workspace_bytes(int B, int H, int T, int D);
 
 /* Backward.  q, k, v, o, lse: as given to / returned by attn_fwd; dO: bf16
